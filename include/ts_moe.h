@@ -1,0 +1,166 @@
+/*
+ * ts_moe.h -- C ABI of the B200 (sm_100a) routed MoE half of a decoder layer.
+ *
+ * One call of ts_moe_forward runs, for a micro-batch of M <= 16 tokens, the
+ * routed half that the turbospark-runtime family-state pages describe:
+ *   router GEMV to FP32 logits -> family top-k rule -> each selected expert's
+ *   gate/up GEMV, SwiGLU (or clamped SwiGLU), down GEMV -> weighted sum
+ *   (+ optional shared expert) -> added back to the residual stream.
+ * Every step runs in this library's CUDA kernels on the caller's stream; the
+ * host does no per-call arithmetic, no allocation and no synchronisation.
+ *
+ * Conventions
+ *   - "device" pointers are CUDA device addresses on cfg->device; "host"
+ *     pointers are ordinary process memory.
+ *   - Matrices are row-major.  Quantised matrices are rows of 32-element
+ *     blocks:  Q8_0 block = { uint16 d (IEEE fp16 bits); int8 q[32] } (34 B),
+ *     element i = d * q[i];  MXFP4 block = { uint8 e (E8M0, 2^(e-127));
+ *     uint8 qs[16] } (17 B), element 2j = low nibble of qs[j], element 2j+1 =
+ *     high nibble, each an E2M1 code (bit 3 sign; magnitudes 0,.5,1,1.5,2,3,4,6).
+ *   - BF16 values are passed as their 16-bit patterns (little-endian uint16).
+ *   - Every function returns a ts_moe_status; on failure ts_moe_last_error()
+ *     gives a one-line reason.  Nothing aborts, prints or throws.
+ */
+#ifndef TS_MOE_H
+#define TS_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TS_MOE_ABI_VERSION 1u
+#define TS_MOE_MAX_TOKENS 16 /* micro-batch cap: MAX_PREFILL_BATCH = 16 (llama / gpt-oss state pages) */
+#define TS_MOE_MAX_TOPK 8    /* PHASE2_FIXED_SLOTS = 8 (deepseek2 state page, `build`) */
+#define TS_MOE_MAX_EXPERTS 256
+
+typedef enum {
+  TS_MOE_OK = 0,
+  TS_MOE_EINVAL = 1,       /* bad argument: NULL, out-of-range size or index, non-finite bias */
+  TS_MOE_EUNSUPPORTED = 2, /* well-formed but outside what the kernels implement */
+  TS_MOE_ENOMEM = 3,       /* device allocation failed at open */
+  TS_MOE_ECUDA = 4,        /* a CUDA runtime call failed (message in last_error) */
+  TS_MOE_EDEVICE = 5       /* a kernel reported an error through the device error word */
+} ts_moe_status;
+
+enum { TS_FMT_Q8_0 = 0, TS_FMT_MXFP4 = 1 };
+/* Top-k rule.  SOFTMAX_SELECTED: softmax over the K selected experts (llama /
+ * gpt-oss state pages, `per_expert_ones`: "selection reduces to softmax over the
+ * selected").  SOFTMAX_ALL_NORENORM: softmax over all E experts, the K largest
+ * kept with no renormalisation (deepseek2 state page, layer sketch). */
+enum { TS_SCORE_SOFTMAX_SELECTED = 0, TS_SCORE_SOFTMAX_ALL_NORENORM = 1 };
+/* Router bias (gpt-oss state page, `router_bias`: added to the logits BEFORE
+ * top-k).  LOGITS: selection and weights both use l + b.  SELECT_ONLY: l + b
+ * selects, the weights use the unbiased l. */
+enum { TS_BIAS_NONE = 0, TS_BIAS_LOGITS = 1, TS_BIAS_SELECT_ONLY = 2 };
+/* SWIGLU: silu(g) * u.  SWIGLU_CLAMPED (gpt-oss state page header, "clamped
+ * SwiGLU"): g' = min(g, limit), u' = clamp(u, -limit, limit),
+ * a = g' * sigmoid(alpha * g') * (u' + 1). */
+enum { TS_ACT_SWIGLU = 0, TS_ACT_SWIGLU_CLAMPED = 1 };
+/* Where the bulk weight blobs passed to ts_moe_open live. */
+enum { TS_MEM_HOST = 0, TS_MEM_DEVICE = 1 };
+
+typedef struct {
+  uint32_t abi_version;  /* TS_MOE_ABI_VERSION */
+  int32_t hidden;        /* H, multiple of 32, <= 16384 */
+  int32_t moe_inter;     /* I, routed expert width, multiple of 32, <= 65536 */
+  int32_t num_experts;   /* E, 1..256 */
+  int32_t top_k;         /* K, 1..min(8, E) */
+  int32_t num_layers;    /* layers held by this handle, 1..1024 */
+  int32_t max_tokens;    /* largest M any call will pass, 1..16 */
+  int32_t expert_fmt;    /* TS_FMT_*; router and shared expert are always Q8_0 */
+  int32_t score;         /* TS_SCORE_* */
+  int32_t bias_mode;     /* TS_BIAS_* */
+  int32_t act;           /* TS_ACT_* (the shared expert uses the same rule) */
+  float act_alpha;       /* clamped SwiGLU alpha (1.702 for gpt-oss) */
+  float act_limit;       /* clamped SwiGLU limit (7.0 for gpt-oss), > 0 */
+  int32_t shared_inter;  /* S, 0 = no shared expert; else multiple of 32 (Q8_0 only) */
+  int32_t device;        /* CUDA device ordinal */
+  int32_t weights_mem;   /* TS_MEM_HOST or TS_MEM_DEVICE for the blobs below */
+} ts_moe_config;
+
+/* One layer's weights, read (copied and repacked) by ts_moe_open only; the
+ * caller may free them when it returns.  router_xscale, router_bias and
+ * per_expert_scale are always HOST memory; the other blobs live where
+ * cfg->weights_mem says. */
+typedef struct {
+  const void* router;             /* [E][H] Q8_0 (llama state page: "INT8 router kernel" with an fp16 block scale) */
+  const uint16_t* router_xscale;  /* [H] BF16 per-element x scale, or NULL = ones (`router_ones`) */
+  const float* router_bias;       /* [E], finite; required iff bias_mode != NONE (`router_bias`) */
+  const float* per_expert_scale;  /* [E], or NULL = ones (`per_expert_ones`); multiplies the weights */
+  const void* gate;               /* [E][I][H] expert_fmt */
+  const void* up;                 /* [E][I][H] expert_fmt */
+  const void* down;               /* [E][H][I] expert_fmt */
+  const void* sh_gate;            /* [S][H] Q8_0, required iff shared_inter > 0 */
+  const void* sh_up;              /* [S][H] Q8_0 */
+  const void* sh_down;            /* [H][S] Q8_0 */
+} ts_moe_layer_weights;
+
+typedef struct ts_moe ts_moe;
+
+/* Validates cfg and layers[0 .. num_layers-1] (shapes, enums, finiteness of
+ * the bias, E8M0 = 255 and non-finite Q8_0 scales are refused), then on
+ * cfg->device allocates the repacked weight arena and the per-call workspace
+ * (sized once for max_tokens) and repacks every layer.  All refusals happen
+ * before any device memory exists (deepseek2 state page: errors at open, "not
+ * at token 1").  *out is set only on TS_MOE_OK.  Synchronises the device. */
+ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* layers, ts_moe** out);
+
+/* Router GEMV + top-k only (steps a1-a3).  x: device [M][H] BF16 (row-major).
+ * idx: device [M][K] int32 selected experts in slot order (descending
+ * selection logit, lower index first on ties); w: device [M][K] float32
+ * weights; logits: device [M][E] float32 router logits before any bias, or
+ * NULL.  0 <= M <= max_tokens (M = 0 is a no-op).  Asynchronous on `stream`
+ * (a cudaStream_t, NULL = legacy default stream). */
+ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
+                           void* stream);
+
+/* The whole routed half for one layer.  x: device [M][H] BF16 (the
+ * post-attention-norm activations, `moe_x`).  resid: device [M][H] BF16,
+ * updated in place to bf16(resid + y), or NULL.  y: device [M][H] float32
+ * routed(+shared) sum (`h2`), or NULL.  At least one of resid / y must be
+ * non-NULL.  Asynchronous on `stream`; allocates nothing; calls on one handle
+ * must not overlap on the device (they share the handle's workspace). */
+ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * kernels set on a bounded wait that gave up or an index found out of range.
+ * Returns TS_MOE_EDEVICE (with the bits in last_error) if any was set; in that
+ * case the handle's inter-block counters are re-zeroed so later calls start
+ * clean. */
+ts_moe_status ts_moe_device_status(ts_moe* h, void* stream);
+
+/* Sizes the caller may need: arena bytes, per-expert algorithmic bytes in the
+ * input format (gate + up + down), router bytes per layer, shared expert bytes
+ * per layer, number of CTAs the expert kernels launch. */
+typedef struct {
+  uint64_t arena_bytes;
+  uint64_t workspace_bytes;
+  uint64_t expert_bytes;
+  uint64_t router_bytes;
+  uint64_t shared_bytes;
+  int32_t num_ctas;
+  int32_t sm_count;
+} ts_moe_info;
+ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
+
+/* Optional per-phase timing hooks for profiling: when set, ts_moe_forward
+ * records events[0] before the gate/up kernel and events[1] after it, and
+ * events[2] / events[3] around the down+combine kernel, on the call's stream
+ * (cudaEvent_t values; NULL clears).  Events between the kernels serialise
+ * them, so a timed run without hooks is the throughput number. */
+ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4);
+
+/* Reason for the last failure on this handle; with h == NULL, the last
+ * failure of ts_moe_open on the calling thread.  Never NULL. */
+const char* ts_moe_last_error(const ts_moe* h);
+
+/* Frees the arena and workspace.  NULL is a no-op.  The caller must make sure
+ * no call on the handle is still running on the device. */
+ts_moe_status ts_moe_close(ts_moe* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TS_MOE_H */

@@ -1,0 +1,34 @@
+/*
+ * ts_moe_debug.h -- host-only helpers exported for tests.  They expose the
+ * pure arithmetic the kernels use to split work between CTAs and the open-time
+ * validation, so both can be checked on a machine without a GPU.  None of
+ * them touches device memory or the CUDA runtime.
+ */
+#ifndef TS_MOE_DEBUG_H
+#define TS_MOE_DEBUG_H
+
+#include <stdint.h>
+
+#include "ts_moe.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* First unit of CTA b when U units are cut into NB contiguous ranges:
+ * floor(b * U / NB).  Range of CTA b = [start(b), start(b + 1)). */
+uint64_t ts_moe_debug_range_start(uint64_t U, int NB, int b);
+/* The CTA whose range holds unit u (0 <= u < U, U >= 1). */
+int ts_moe_debug_owner_of(uint64_t U, int NB, uint64_t u);
+/* Partial-sum slot (0 or 1) CTA b uses for the group whose first unit is g0. */
+int ts_moe_debug_partial_slot(uint64_t U, int NB, int b, uint64_t g0);
+/* Tiles per group chosen for an expert matrix of `tiles` 16-row tiles. */
+int ts_moe_debug_group_size(int tiles);
+/* The validation ts_moe_open performs before any CUDA call; same status and
+ * message (ts_moe_last_error(NULL)). */
+ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TS_MOE_DEBUG_H */

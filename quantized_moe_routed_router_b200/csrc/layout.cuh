@@ -1,0 +1,86 @@
+// Repacked weight layout and the work partition shared by host and device code.
+//
+// Repacked expert matrix ("tile-major for the tensor-core fragment"):
+//   A tile is 16 MMA rows.  Gate/up tiles interleave 8 gate rows (tile rows
+//   0..7) with the same 8 rows of up (tile rows 8..15), so one thread holds
+//   gate and up of the same act row and forms the activation in registers.
+//   Down tiles are 16 consecutive rows of the [H][I] matrix.
+//   K is cut into chunks of KC elements (64 for MXFP4, 32 for Q8_0); one
+//   (tile, chunk) unit is 544 bytes: 512 bytes of quants, lane l of a warp
+//   owning bytes [16 l, 16 l + 16) (its whole A fragment for the chunk),
+//   followed by 32 bytes of block scales, 4 per lane quad.
+//   Tiles are grouped (GS tiles per group, the last group may be short) and a
+//   group is stored chunk-major: [chunk][tile in group][544 B], so any run of
+//   chunks of one group is one contiguous range -- one bulk copy.
+#pragma once
+#include <stdint.h>
+
+#ifndef TSM_HD
+#define TSM_HD __host__ __device__ __forceinline__
+#endif
+
+namespace tsm {
+
+constexpr int UNIT_BYTES = 544;       // one (tile, chunk): 512 B quants + 32 B scales
+constexpr int QUANT_BYTES = 512;
+constexpr int GS_MAX = 16;            // tiles per group (= consumer warps x tiles per warp)
+constexpr int MAX_TOK = 16;
+constexpr int MAX_K = 8;
+constexpr int MAX_E = 256;
+constexpr int MAX_ENTRIES = MAX_E + 1;  // touched routed experts + the shared pseudo-expert
+
+TSM_HD int chunk_k(int fmt) { return fmt == 1 ? 64 : 32; }  // elements of K per chunk
+TSM_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
+
+struct MatGeom {
+  int tiles;       // 16-row MMA tiles per expert
+  int chunks;      // K chunks
+  int gs;          // tiles per group
+  int ngroups;     // groups per expert
+  int kdim;        // K (unpadded)
+  int fmt;         // 0 Q8_0, 1 MXFP4
+  uint64_t bytes;  // bytes per expert matrix = tiles * chunks * 544
+};
+
+// Largest tile count per group in [8, 16] that divides `tiles` (equal groups
+// keep the work partition balanced); otherwise 16 with a short last group.
+inline int pick_group_size(int tiles) {
+  if (tiles <= GS_MAX) return tiles;
+  for (int g = GS_MAX; g >= 8; --g)
+    if (tiles % g == 0) return g;
+  return GS_MAX;
+}
+
+inline MatGeom make_geom(int rows_tiles, int kdim, int fmt) {
+  MatGeom m;
+  m.tiles = rows_tiles;
+  m.kdim = kdim;
+  m.fmt = fmt;
+  m.chunks = (kdim + chunk_k(fmt) - 1) / chunk_k(fmt);
+  m.gs = pick_group_size(rows_tiles);
+  m.ngroups = (rows_tiles + m.gs - 1) / m.gs;
+  m.bytes = (uint64_t)rows_tiles * m.chunks * UNIT_BYTES;
+  return m;
+}
+
+TSM_HD uint64_t group_offset(int gs, int chunks, int grp) { return (uint64_t)grp * gs * chunks * UNIT_BYTES; }
+TSM_HD int group_tiles(int tiles, int gs, int grp) {
+  int t = tiles - grp * gs;
+  return t < gs ? t : gs;
+}
+
+// ----------------------------------------------------------------------------- stream-K partition
+// The units of one launch (all touched entries' (group, chunk) pairs, entries
+// in order, groups in order, chunks in order) are split into NB contiguous
+// ranges: block b owns [range_start(b), range_start(b + 1)).
+TSM_HD uint64_t range_start(uint64_t U, int NB, int b) { return (uint64_t)b * U / (uint64_t)NB; }
+
+// The block whose range contains unit u (0 <= u < U): the largest b with
+// range_start(b) <= u, i.e. floor(((u + 1) * NB - 1) / U).
+TSM_HD int owner_of(uint64_t U, int NB, uint64_t u) { return (int)(((u + 1) * (uint64_t)NB - 1) / U); }
+
+// Partial-sum slot of block b for the group starting at unit g0: 0 when the
+// group is b's first segment (b's range starts inside it), else 1 (its last).
+TSM_HD int partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return range_start(U, NB, b) >= g0 ? 0 : 1; }
+
+}  // namespace tsm

@@ -1,0 +1,656 @@
+// C-ABI library: open-time validation, device allocation and repack; per-call
+// launch of the route kernel and the two expert kernels on the caller's
+// stream with programmatic dependent launch (each kernel's prologue overlaps
+// the previous kernel's tail; griddepcontrol.wait orders the data).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/ts_moe.h"
+#include "../../include/ts_moe_debug.h"
+#include "common.cuh"
+#include "expert.cuh"
+#include "layout.cuh"
+#include "repack.cuh"
+#include "route.cuh"
+
+using namespace tsm;
+
+namespace {
+
+thread_local std::string g_open_error;
+
+struct LayerDev {
+  int8_t* rq = nullptr;
+  float* rd = nullptr;
+  float* bias = nullptr;
+  float* pes = nullptr;
+  float* xscale = nullptr;
+  uint8_t* wB = nullptr;   // routed gate/up, E matrices
+  uint8_t* wC = nullptr;   // routed down
+  uint8_t* wBs = nullptr;  // shared gate/up
+  uint8_t* wCs = nullptr;  // shared down
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t blob_row_bytes(int fmt, int cols) { return (size_t)(cols / 32) * (fmt == TS_FMT_Q8_0 ? 34 : 17); }
+
+}  // namespace
+
+struct ts_moe {
+  ts_moe_config cfg{};
+  int sm_count = 0, nb = 0;
+  int Hp = 0, Ip = 0, Sp = 0;
+  MatGeom gB{}, gC{}, gBs{}, gCs{};
+  int ng_max_B = 0, ng_max_C = 0;
+  uint8_t* arena = nullptr;
+  size_t arena_bytes = 0;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  std::vector<LayerDev> layers;
+  // workspace views
+  float* logits = nullptr;
+  int* idx = nullptr;
+  float* w = nullptr;
+  int* rpos = nullptr;
+  int* shift = nullptr;
+  int* meta = nullptr;
+  Route* routes = nullptr;
+  __half* xh = nullptr;
+  __half* acts = nullptr;
+  __half* acts_sh = nullptr;
+  float* P = nullptr;
+  float* partial = nullptr;
+  unsigned* cnt_route = nullptr;
+  unsigned* cnt_gB = nullptr;
+  unsigned* cnt_gC = nullptr;
+  unsigned* cnt_rg = nullptr;
+  unsigned* err = nullptr;
+  size_t counters_bytes = 0;
+  uint8_t* counters = nullptr;
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  bool timing = false;
+  std::string error;
+  uint64_t expert_bytes = 0, router_bytes = 0, shared_bytes = 0;
+};
+
+namespace {
+
+ts_moe_status fail(ts_moe* h, ts_moe_status st, const std::string& msg) {
+  if (h)
+    h->error = msg;
+  else
+    g_open_error = msg;
+  return st;
+}
+
+ts_moe_status cuda_fail(ts_moe* h, cudaError_t e, const char* what) {
+  return fail(h, TS_MOE_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define TSM_CUDA(h, call)                                     \
+  do {                                                        \
+    cudaError_t e_ = (call);                                  \
+    if (e_ != cudaSuccess) return cuda_fail((h), e_, #call);  \
+  } while (0)
+
+// Host-side validation: everything that can be refused before device memory exists.
+ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
+  if (!c) return fail(nullptr, TS_MOE_EINVAL, "config is NULL");
+  if (c->abi_version != TS_MOE_ABI_VERSION) return fail(nullptr, TS_MOE_EINVAL, "abi_version mismatch");
+  auto bad = [&](const std::string& m) { return fail(nullptr, TS_MOE_EINVAL, m); };
+  auto uns = [&](const std::string& m) { return fail(nullptr, TS_MOE_EUNSUPPORTED, m); };
+  if (c->hidden <= 0 || c->hidden % 32) return bad("hidden must be a positive multiple of 32 (whole Q8_0/MXFP4 blocks)");
+  if (c->hidden > 16384) return uns("hidden > 16384 is not supported");
+  if (c->moe_inter <= 0 || c->moe_inter % 32) return bad("moe_inter must be a positive multiple of 32");
+  if (c->moe_inter > 65536) return uns("moe_inter > 65536 is not supported");
+  if (c->num_experts < 1 || c->num_experts > TS_MOE_MAX_EXPERTS) return bad("num_experts must be in [1, 256]");
+  if (c->top_k < 1 || c->top_k > TS_MOE_MAX_TOPK || c->top_k > c->num_experts)
+    return bad("top_k must be in [1, min(8, num_experts)] (the 8-slot phase-2 reduce)");
+  if (c->num_layers < 1 || c->num_layers > 1024) return bad("num_layers must be in [1, 1024]");
+  if (c->max_tokens < 1 || c->max_tokens > TS_MOE_MAX_TOKENS) return bad("max_tokens must be in [1, 16]");
+  if (c->expert_fmt != TS_FMT_Q8_0 && c->expert_fmt != TS_FMT_MXFP4) return bad("unknown expert_fmt");
+  if (c->score != TS_SCORE_SOFTMAX_SELECTED && c->score != TS_SCORE_SOFTMAX_ALL_NORENORM) return bad("unknown score");
+  if (c->bias_mode < TS_BIAS_NONE || c->bias_mode > TS_BIAS_SELECT_ONLY) return bad("unknown bias_mode");
+  if (c->act != TS_ACT_SWIGLU && c->act != TS_ACT_SWIGLU_CLAMPED) return bad("unknown act");
+  if (c->act == TS_ACT_SWIGLU_CLAMPED &&
+      (!std::isfinite(c->act_alpha) || !std::isfinite(c->act_limit) || c->act_limit <= 0.f))
+    return bad("clamped SwiGLU needs a finite alpha and a finite limit > 0");
+  if (c->shared_inter < 0 || c->shared_inter % 32) return bad("shared_inter must be 0 or a multiple of 32");
+  if (c->shared_inter > 65536) return uns("shared_inter > 65536 is not supported");
+  if (c->shared_inter > 0 && c->expert_fmt != TS_FMT_Q8_0)
+    return uns("a shared expert is only supported with Q8_0 routed experts (no family on the pages mixes them)");
+  if (c->weights_mem != TS_MEM_HOST && c->weights_mem != TS_MEM_DEVICE) return bad("unknown weights_mem");
+  if (c->device < 0) return bad("device must be >= 0");
+  if (!L) return bad("layers is NULL");
+  for (int l = 0; l < c->num_layers; ++l) {
+    const ts_moe_layer_weights& w = L[l];
+    const std::string at = " (layer " + std::to_string(l) + ")";
+    if (!w.router || !w.gate || !w.up || !w.down) return bad("router/gate/up/down must be non-NULL" + at);
+    if ((c->bias_mode != TS_BIAS_NONE) != (w.router_bias != nullptr))
+      return bad("router_bias must be given iff bias_mode != NONE" + at);
+    if (w.router_bias)
+      for (int e = 0; e < c->num_experts; ++e)
+        if (!std::isfinite(w.router_bias[e])) return bad("non-finite router bias" + at);
+    if (w.per_expert_scale)
+      for (int e = 0; e < c->num_experts; ++e)
+        if (!std::isfinite(w.per_expert_scale[e])) return bad("non-finite per_expert_scale" + at);
+    if (w.router_xscale)
+      for (int n = 0; n < c->hidden; ++n)
+        if ((w.router_xscale[n] & 0x7F80u) == 0x7F80u) return bad("non-finite router_xscale" + at);
+    const bool sh = w.sh_gate || w.sh_up || w.sh_down;
+    if (c->shared_inter > 0 && !(w.sh_gate && w.sh_up && w.sh_down))
+      return bad("shared_inter > 0 needs sh_gate, sh_up and sh_down" + at);
+    if (c->shared_inter == 0 && sh) return bad("shared expert blobs given with shared_inter == 0" + at);
+  }
+  return TS_MOE_OK;
+}
+
+template <typename... Args>
+cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(block);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, k, args...);
+}
+
+ts_moe_status set_smem_attrs(ts_moe* h) {
+  const int bytes = (int)sizeof(PhaseSmem);
+  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  const int rbytes = (h->cfg.hidden + h->cfg.num_experts) * 4;
+  if (rbytes > 48 * 1024)
+    TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rbytes));
+  return TS_MOE_OK;
+}
+
+template <int PHASE>
+void launch_repack(int fmt, const uint8_t* a, const uint8_t* b, int row_bytes, int nblocks, const MatGeom& g,
+                   uint8_t* dst, unsigned* bad, cudaStream_t st) {
+  const long long units = (long long)g.tiles * g.chunks;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((units + 7) / 8, 65535LL * 8);
+  if (fmt == TS_FMT_MXFP4)
+    repack_kernel<1, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
+                                                                                      g.chunks, g.gs, dst, bad);
+  else
+    repack_kernel<0, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
+                                                                                      g.chunks, g.gs, dst, bad);
+}
+
+}  // namespace
+
+extern "C" {
+
+ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* layers, ts_moe** out) {
+  if (!out) return fail(nullptr, TS_MOE_EINVAL, "out is NULL");
+  *out = nullptr;
+  ts_moe_status st = validate(cfg, layers);
+  if (st != TS_MOE_OK) return st;
+
+  int ndev = 0;
+  cudaError_t ce = cudaGetDeviceCount(&ndev);
+  if (ce != cudaSuccess || ndev == 0)
+    return fail(nullptr, TS_MOE_ECUDA, std::string("no CUDA device: ") + cudaGetErrorString(ce));
+  if (cfg->device >= ndev) return fail(nullptr, TS_MOE_EINVAL, "device ordinal out of range");
+  ce = cudaSetDevice(cfg->device);
+  if (ce != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaSetDevice: ") + cudaGetErrorString(ce));
+  cudaDeviceProp prop;
+  ce = cudaGetDeviceProperties(&prop, cfg->device);
+  if (ce != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, cudaGetErrorString(ce));
+  if (prop.major != 10)
+    return fail(nullptr, TS_MOE_EUNSUPPORTED, "the kernels are built for sm_100a (B200); this device is sm_" +
+                                                  std::to_string(prop.major) + std::to_string(prop.minor));
+
+  ts_moe* h = new ts_moe();
+  h->cfg = *cfg;
+  const ts_moe_config& c = h->cfg;
+  const int H = c.hidden, I = c.moe_inter, E = c.num_experts, K = c.top_k, S = c.shared_inter, Mx = c.max_tokens;
+  const int fmt = c.expert_fmt;
+  h->sm_count = prop.multiProcessorCount;
+  h->nb = h->sm_count;
+  h->Hp = round_up(H, 64);
+  h->Ip = round_up(I, 64);
+  h->Sp = S ? round_up(S, 64) : 0;
+  h->gB = make_geom(I / 8, H, fmt);
+  h->gC = make_geom(H / 16, I, fmt);
+  if (S) {
+    h->gBs = make_geom(S / 8, H, TS_FMT_Q8_0);
+    h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
+  }
+  h->ng_max_B = std::max(h->gB.ngroups, S ? h->gBs.ngroups : 0);
+  h->ng_max_C = std::max(h->gC.ngroups, S ? h->gCs.ngroups : 0);
+  h->expert_bytes = 2ull * I * blob_row_bytes(fmt, H) + (uint64_t)H * blob_row_bytes(fmt, I);
+  h->router_bytes = (uint64_t)E * blob_row_bytes(TS_FMT_Q8_0, H);
+  h->shared_bytes = S ? 2ull * S * blob_row_bytes(TS_FMT_Q8_0, H) + (uint64_t)H * blob_row_bytes(TS_FMT_Q8_0, S) : 0;
+
+  auto cleanup = [&](ts_moe_status s2) {
+    ts_moe_close(h);
+    return s2;
+  };
+
+  // ---- arena
+  size_t per_layer = 0;
+  per_layer += align256((size_t)E * H);            // rq
+  per_layer += align256((size_t)E * (H / 32) * 4); // rd
+  per_layer += align256((size_t)E * 4) * 2;        // bias, pes
+  per_layer += align256((size_t)H * 4);            // xscale
+  per_layer += align256(h->gB.bytes * E);
+  per_layer += align256(h->gC.bytes * E);
+  if (S) per_layer += align256(h->gBs.bytes) + align256(h->gCs.bytes);
+  h->arena_bytes = per_layer * c.num_layers;
+  ce = cudaMalloc(&h->arena, h->arena_bytes);
+  if (ce != cudaSuccess) {
+    g_open_error = "arena allocation of " + std::to_string(h->arena_bytes) + " bytes failed";
+    ts_moe_close(h);
+    return TS_MOE_ENOMEM;
+  }
+  h->layers.resize(c.num_layers);
+  {
+    uint8_t* p = h->arena;
+    auto take = [&](size_t n) {
+      uint8_t* r = p;
+      p += align256(n);
+      return r;
+    };
+    for (int l = 0; l < c.num_layers; ++l) {
+      LayerDev& d = h->layers[l];
+      d.rq = (int8_t*)take((size_t)E * H);
+      d.rd = (float*)take((size_t)E * (H / 32) * 4);
+      d.bias = (float*)take((size_t)E * 4);
+      d.pes = (float*)take((size_t)E * 4);
+      d.xscale = (float*)take((size_t)H * 4);
+      d.wB = take(h->gB.bytes * E);
+      d.wC = take(h->gC.bytes * E);
+      if (S) {
+        d.wBs = take(h->gBs.bytes);
+        d.wCs = take(h->gCs.bytes);
+      }
+    }
+  }
+
+  // ---- workspace (sized once for max_tokens; the calls allocate nothing)
+  {
+    size_t off = 0;
+    auto slot = [&](size_t n) {
+      size_t r = off;
+      off += align256(n);
+      return r;
+    };
+    const size_t o_logits = slot((size_t)Mx * E * 4);
+    const size_t o_idx = slot((size_t)Mx * K * 4);
+    const size_t o_w = slot((size_t)Mx * K * 4);
+    const size_t o_rpos = slot((size_t)Mx * K * 4);
+    const size_t o_shift = slot((size_t)Mx * 4);
+    const size_t o_meta = slot((size_t)META_INTS * 4);
+    const size_t o_routes = slot((size_t)Mx * K * sizeof(Route));
+    const size_t o_xh = slot((size_t)Mx * h->Hp * 2);
+    const size_t o_acts = slot((size_t)Mx * K * h->Ip * 2);
+    const size_t o_acts_sh = slot((size_t)Mx * std::max(h->Sp, 64) * 2);
+    const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
+    const size_t o_partial = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
+    const size_t o_cnt = off;
+    const size_t n_cnt = 1 + (size_t)(E + 1) * h->ng_max_B + (size_t)(E + 1) * h->ng_max_C + h->gC.ngroups + 1;
+    slot(n_cnt * 4);
+    h->ws_bytes = off;
+    ce = cudaMalloc(&h->ws, h->ws_bytes);
+    if (ce != cudaSuccess) {
+      g_open_error = "workspace allocation failed";
+      ts_moe_close(h);
+      return TS_MOE_ENOMEM;
+    }
+    h->logits = (float*)(h->ws + o_logits);
+    h->idx = (int*)(h->ws + o_idx);
+    h->w = (float*)(h->ws + o_w);
+    h->rpos = (int*)(h->ws + o_rpos);
+    h->shift = (int*)(h->ws + o_shift);
+    h->meta = (int*)(h->ws + o_meta);
+    h->routes = (Route*)(h->ws + o_routes);
+    h->xh = (__half*)(h->ws + o_xh);
+    h->acts = (__half*)(h->ws + o_acts);
+    h->acts_sh = (__half*)(h->ws + o_acts_sh);
+    h->P = (float*)(h->ws + o_P);
+    h->partial = (float*)(h->ws + o_partial);
+    unsigned* cn = (unsigned*)(h->ws + o_cnt);
+    h->counters = (uint8_t*)cn;
+    h->counters_bytes = n_cnt * 4;
+    h->cnt_route = cn;
+    h->cnt_gB = cn + 1;
+    h->cnt_gC = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
+    h->cnt_rg = h->cnt_gC + (size_t)(E + 1) * h->ng_max_C;
+    h->err = h->cnt_rg + h->gC.ngroups;
+    // zeros: counters, error word, and the padding columns of x / acts
+    ce = cudaMemset(h->ws, 0, h->ws_bytes);
+    if (ce != cudaSuccess) {
+      g_open_error = std::string("workspace memset: ") + cudaGetErrorString(ce);
+      return cleanup(TS_MOE_ECUDA);
+    }
+  }
+  if ((st = set_smem_attrs(h)) != TS_MOE_OK) {
+    g_open_error = h->error;
+    return cleanup(st);
+  }
+
+  // ---- upload + repack every layer
+  unsigned* d_bad = nullptr;
+  uint8_t* stage = nullptr;
+  size_t stage_bytes = 0;
+  const size_t gate_bytes = (size_t)E * I * blob_row_bytes(fmt, H);
+  const size_t down_bytes = (size_t)E * H * blob_row_bytes(fmt, I);
+  const size_t router_b = (size_t)E * blob_row_bytes(TS_FMT_Q8_0, H);
+  const size_t shg = S ? (size_t)S * blob_row_bytes(TS_FMT_Q8_0, H) : 0;
+  const size_t shd = S ? (size_t)H * blob_row_bytes(TS_FMT_Q8_0, S) : 0;
+  ce = cudaMalloc(&d_bad, 4);
+  if (ce == cudaSuccess) ce = cudaMemset(d_bad, 0, 4);
+  if (ce == cudaSuccess && c.weights_mem == TS_MEM_HOST) {
+    stage_bytes = std::max({2 * gate_bytes, down_bytes, router_b, 2 * shg, shd});
+    ce = cudaMalloc(&stage, stage_bytes);
+  }
+  if (ce != cudaSuccess) {
+    g_open_error = std::string("repack staging: ") + cudaGetErrorString(ce);
+    cudaFree(d_bad);
+    cudaFree(stage);
+    ts_moe_close(h);
+    return TS_MOE_ENOMEM;
+  }
+  cudaStream_t st0 = 0;
+  std::vector<float> ones((size_t)std::max(H, E), 1.0f);
+  std::vector<float> tmp((size_t)std::max(H, E));
+  for (int l = 0; l < c.num_layers && ce == cudaSuccess; ++l) {
+    const ts_moe_layer_weights& w = layers[l];
+    LayerDev& d = h->layers[l];
+    auto src = [&](const void* p, size_t bytes, size_t at) -> const uint8_t* {
+      if (c.weights_mem == TS_MEM_DEVICE) return (const uint8_t*)p;
+      if (ce == cudaSuccess) ce = cudaMemcpy(stage + at, p, bytes, cudaMemcpyHostToDevice);
+      return stage + at;
+    };
+    // router + small vectors
+    const uint8_t* r = src(w.router, router_b, 0);
+    if (ce != cudaSuccess) break;
+    repack_router_kernel<<<std::max<int>(1, (int)std::min<long long>(((long long)E * (H / 32) + 255) / 256, 65535)),
+                           256, 0, st0>>>(r, E, H, d.rq, d.rd, d_bad);
+    if (ce == cudaSuccess) ce = cudaDeviceSynchronize();  // the staging buffer is reused next
+    if (w.router_bias && ce == cudaSuccess) ce = cudaMemcpy(d.bias, w.router_bias, E * 4, cudaMemcpyHostToDevice);
+    if (ce == cudaSuccess)
+      ce = cudaMemcpy(d.pes, w.per_expert_scale ? w.per_expert_scale : ones.data(), E * 4, cudaMemcpyHostToDevice);
+    if (w.router_xscale) {
+      for (int n = 0; n < H; ++n) {
+        uint32_t u = (uint32_t)w.router_xscale[n] << 16;
+        std::memcpy(&tmp[n], &u, 4);
+      }
+    } else {
+      std::fill(tmp.begin(), tmp.begin() + H, 1.0f);
+    }
+    if (ce == cudaSuccess) ce = cudaMemcpy(d.xscale, tmp.data(), (size_t)H * 4, cudaMemcpyHostToDevice);
+    // gate/up -> phase-1 layout, per expert
+    const uint8_t* gsrc = src(w.gate, gate_bytes, 0);
+    const uint8_t* usrc = src(w.up, gate_bytes, gate_bytes);
+    if (ce != cudaSuccess) break;
+    const int rbH = (int)blob_row_bytes(fmt, H), rbI = (int)blob_row_bytes(fmt, I);
+    for (int e = 0; e < E; ++e)
+      launch_repack<0>(fmt, gsrc + (size_t)e * I * rbH, usrc + (size_t)e * I * rbH, rbH, H / 32, h->gB,
+                       d.wB + (size_t)e * h->gB.bytes, d_bad, st0);
+    ce = cudaDeviceSynchronize();
+    if (ce != cudaSuccess) break;
+    const uint8_t* dsrc = src(w.down, down_bytes, 0);
+    if (ce != cudaSuccess) break;
+    for (int e = 0; e < E; ++e)
+      launch_repack<1>(fmt, dsrc + (size_t)e * H * rbI, nullptr, rbI, I / 32, h->gC, d.wC + (size_t)e * h->gC.bytes,
+                       d_bad, st0);
+    ce = cudaDeviceSynchronize();
+    if (ce != cudaSuccess) break;
+    if (S) {
+      const int rbHq = (int)blob_row_bytes(TS_FMT_Q8_0, H), rbS = (int)blob_row_bytes(TS_FMT_Q8_0, S);
+      const uint8_t* sg = src(w.sh_gate, shg, 0);
+      const uint8_t* su = src(w.sh_up, shg, shg);
+      if (ce != cudaSuccess) break;
+      launch_repack<0>(TS_FMT_Q8_0, sg, su, rbHq, H / 32, h->gBs, d.wBs, d_bad, st0);
+      ce = cudaDeviceSynchronize();
+      if (ce != cudaSuccess) break;
+      const uint8_t* sd = src(w.sh_down, shd, 0);
+      if (ce != cudaSuccess) break;
+      launch_repack<1>(TS_FMT_Q8_0, sd, nullptr, rbS, S / 32, h->gCs, d.wCs, d_bad, st0);
+      ce = cudaDeviceSynchronize();
+    }
+  }
+  unsigned bad = 0;
+  if (ce == cudaSuccess) ce = cudaMemcpy(&bad, d_bad, 4, cudaMemcpyDeviceToHost);
+  cudaFree(d_bad);
+  cudaFree(stage);
+  if (ce != cudaSuccess) {
+    g_open_error = std::string("repack: ") + cudaGetErrorString(ce);
+    ts_moe_close(h);
+    return TS_MOE_ECUDA;
+  }
+  if (bad) {
+    g_open_error = std::string("refused at open: ") + ((bad & BAD_E8M0_NAN) ? "MXFP4 block scale e8m0 = 255 (NaN); " : "") +
+                   ((bad & BAD_Q8_SCALE) ? "non-finite Q8_0 block scale; " : "") +
+                   ((bad & BAD_ROUTER_SCALE) ? "non-finite router block scale; " : "");
+    ts_moe_close(h);
+    return TS_MOE_EINVAL;
+  }
+  *out = h;
+  return TS_MOE_OK;
+}
+
+static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
+  const ts_moe_config& c = h->cfg;
+  const LayerDev& d = h->layers[layer];
+  RouteParams rp;
+  rp.x = (const __nv_bfloat16*)x;
+  rp.M = M;
+  rp.H = c.hidden;
+  rp.Hp = h->Hp;
+  rp.E = c.num_experts;
+  rp.K = c.top_k;
+  rp.rq = d.rq;
+  rp.rd = d.rd;
+  rp.xscale = d.xscale;
+  rp.bias = c.bias_mode != TS_BIAS_NONE ? d.bias : nullptr;
+  rp.pes = d.pes;
+  rp.bias_mode = c.bias_mode;
+  rp.score = c.score;
+  rp.has_shared = c.shared_inter > 0;
+  rp.logits = h->logits;
+  rp.idx = h->idx;
+  rp.w = h->w;
+  rp.shift = h->shift;
+  rp.xh = h->xh;
+  rp.meta = h->meta;
+  rp.routes = h->routes;
+  rp.rpos = h->rpos;
+  rp.cnt = h->cnt_route;
+  rp.err = h->err;
+  rp.idx_out = nullptr;
+  rp.w_out = nullptr;
+  rp.logits_out = nullptr;
+  return rp;
+}
+
+static ts_moe_status check_call(ts_moe* h, int layer, const void* x, int M) {
+  if (!h) return TS_MOE_EINVAL;
+  if (layer < 0 || layer >= h->cfg.num_layers) return fail(h, TS_MOE_EINVAL, "layer out of range");
+  if (M < 0 || M > h->cfg.max_tokens) return fail(h, TS_MOE_EINVAL, "M out of range [0, max_tokens]");
+  if (M > 0 && !x) return fail(h, TS_MOE_EINVAL, "x is NULL");
+  return TS_MOE_OK;
+}
+
+static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t st) {
+  const size_t smem = (size_t)(h->cfg.hidden + h->cfg.num_experts) * 4;
+  cudaError_t e = launch_pdl(route_kernel, rp.M, ROUTE_THREADS, smem, st, rp);
+  if (e != cudaSuccess) return cuda_fail(h, e, "route_kernel launch");
+  return TS_MOE_OK;
+}
+
+ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
+                           void* stream) {
+  ts_moe_status s = check_call(h, layer, x, M);
+  if (s != TS_MOE_OK) return s;
+  if (M == 0) return TS_MOE_OK;
+  if (!idx || !w) return fail(h, TS_MOE_EINVAL, "idx and w must be non-NULL");
+  RouteParams rp = route_params(h, layer, x, M);
+  rp.idx_out = idx;
+  rp.w_out = w;
+  rp.logits_out = logits;
+  return launch_route(h, rp, (cudaStream_t)stream);
+}
+
+ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream) {
+  ts_moe_status s = check_call(h, layer, x, M);
+  if (s != TS_MOE_OK) return s;
+  if (!resid && !y) return fail(h, TS_MOE_EINVAL, "resid and y are both NULL");
+  if (M == 0) return TS_MOE_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const ts_moe_config& c = h->cfg;
+  const LayerDev& d = h->layers[layer];
+  RouteParams rp = route_params(h, layer, x, M);
+  if ((s = launch_route(h, rp, st)) != TS_MOE_OK) return s;
+
+  PhaseParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.meta = h->meta;
+  pp.routes = h->routes;
+  pp.shift = h->shift;
+  pp.wts = h->w;
+  pp.rpos = h->rpos;
+  pp.partial = h->partial;
+  pp.err = h->err;
+  pp.H = c.hidden;
+  pp.K = c.top_k;
+  pp.E = c.num_experts;
+  pp.act = c.act;
+  pp.alpha = c.act_alpha;
+  pp.limit = c.act_limit;
+  pp.acts = h->acts;
+  pp.acts_ld = h->Ip;
+  pp.acts_sh = h->acts_sh;
+  pp.acts_sh_ld = h->Sp;
+  pp.P = h->P;
+  pp.y = y;
+  pp.resid = (__nv_bfloat16*)resid;
+  pp.cnt_rg = h->cnt_rg;
+
+  // phase 1: gate/up + activation
+  PhaseParams p1 = pp;
+  p1.w_routed = d.wB;
+  p1.w_stride = h->gB.bytes;
+  p1.w_shared = d.wBs;
+  p1.gr = h->gB;
+  p1.gsh = h->gBs;
+  p1.b_routed = h->xh;
+  p1.b_routed_ld = h->Hp;
+  p1.b_shared = h->xh;
+  p1.b_shared_ld = h->Hp;
+  p1.cnt_group = h->cnt_gB;
+  p1.ng_max = h->ng_max_B;
+  // phase 2: down + combine
+  PhaseParams p2 = pp;
+  p2.w_routed = d.wC;
+  p2.w_stride = h->gC.bytes;
+  p2.w_shared = d.wCs;
+  p2.gr = h->gC;
+  p2.gsh = h->gCs;
+  p2.b_routed = h->acts;
+  p2.b_routed_ld = h->Ip;
+  p2.b_shared = h->acts_sh;
+  p2.b_shared_ld = h->Sp;
+  p2.cnt_group = h->cnt_gC;
+  p2.ng_max = h->ng_max_C;
+
+  const size_t smem = sizeof(PhaseSmem);
+  cudaError_t e;
+  if (h->timing) cudaEventRecord(h->ev[0], st);
+  if (c.expert_fmt == TS_FMT_MXFP4)
+    e = launch_pdl(expert_kernel<1, 0>, h->nb, NTHREADS, smem, st, p1);
+  else
+    e = launch_pdl(expert_kernel<0, 0>, h->nb, NTHREADS, smem, st, p1);
+  if (e != cudaSuccess) return cuda_fail(h, e, "gate/up kernel launch");
+  if (h->timing) {
+    cudaEventRecord(h->ev[1], st);
+    cudaEventRecord(h->ev[2], st);
+  }
+  if (c.expert_fmt == TS_FMT_MXFP4)
+    e = launch_pdl(expert_kernel<1, 1>, h->nb, NTHREADS, smem, st, p2);
+  else
+    e = launch_pdl(expert_kernel<0, 1>, h->nb, NTHREADS, smem, st, p2);
+  if (e != cudaSuccess) return cuda_fail(h, e, "down kernel launch");
+  if (h->timing) cudaEventRecord(h->ev[3], st);
+  return TS_MOE_OK;
+}
+
+ts_moe_status ts_moe_device_status(ts_moe* h, void* stream) {
+  if (!h) return TS_MOE_EINVAL;
+  TSM_CUDA(h, cudaSetDevice(h->cfg.device));
+  TSM_CUDA(h, cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned err = 0;
+  TSM_CUDA(h, cudaMemcpy(&err, h->err, 4, cudaMemcpyDeviceToHost));
+  if (!err) return TS_MOE_OK;
+  TSM_CUDA(h, cudaMemset(h->counters, 0, h->counters_bytes));
+  char buf[160];
+  std::snprintf(buf, sizeof buf, "device error word 0x%x (bit0/1: weight-stage wait gave up, bit2/3: activation-window "
+                "wait gave up, bit4: bad index, bit5: bad route metadata)", err);
+  return fail(h, TS_MOE_EDEVICE, buf);
+}
+
+ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info) {
+  if (!h || !info) return TS_MOE_EINVAL;
+  info->arena_bytes = h->arena_bytes;
+  info->workspace_bytes = h->ws_bytes;
+  info->expert_bytes = h->expert_bytes;
+  info->router_bytes = h->router_bytes;
+  info->shared_bytes = h->shared_bytes;
+  info->num_ctas = h->nb;
+  info->sm_count = h->sm_count;
+  return TS_MOE_OK;
+}
+
+ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4) {
+  if (!h) return TS_MOE_EINVAL;
+  if (!events4) {
+    h->timing = false;
+    return TS_MOE_OK;
+  }
+  for (int i = 0; i < 4; ++i) {
+    if (!events4[i]) return fail(h, TS_MOE_EINVAL, "timing events must be non-NULL");
+    h->ev[i] = (cudaEvent_t)events4[i];
+  }
+  h->timing = true;
+  return TS_MOE_OK;
+}
+
+const char* ts_moe_last_error(const ts_moe* h) { return h ? h->error.c_str() : g_open_error.c_str(); }
+
+ts_moe_status ts_moe_close(ts_moe* h) {
+  if (!h) return TS_MOE_OK;
+  cudaSetDevice(h->cfg.device);
+  if (h->arena) cudaFree(h->arena);
+  if (h->ws) cudaFree(h->ws);
+  delete h;
+  return TS_MOE_OK;
+}
+
+// ----------------------------------------------------------------------------- debug helpers (host-only arithmetic)
+uint64_t ts_moe_debug_range_start(uint64_t U, int NB, int b) { return range_start(U, NB, b); }
+int ts_moe_debug_owner_of(uint64_t U, int NB, uint64_t u) { return owner_of(U, NB, u); }
+int ts_moe_debug_partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return partial_slot(U, NB, b, g0); }
+int ts_moe_debug_group_size(int tiles) { return pick_group_size(tiles); }
+ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers) {
+  return validate(cfg, layers);
+}
+
+}  // extern "C"

@@ -1,0 +1,157 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every
+declared symbol, refuses bad configurations before touching CUDA, and its
+work-partition arithmetic covers every unit exactly once."""
+import ctypes as C
+import glob
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from quantized_moe_routed_router_b200 import build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    build.build()
+    from quantized_moe_routed_router_b200 import binding
+    return binding
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(ts_moe_\w+)\s*\(", txt))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(B):
+    names = declared_functions()
+    assert {"ts_moe_open", "ts_moe_route", "ts_moe_forward", "ts_moe_close", "ts_moe_last_error",
+            "ts_moe_device_status"} <= set(names)
+    lib = C.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _small_layers(shape, n=None):
+    n = n or shape.num_layers
+    return [synth.make_layer(shape, l) for l in range(n)]
+
+
+SHAPE = synth.MoEShape("t", 64, 64, 4, 2, cfg_id=77, max_tokens=4)
+
+
+@pytest.mark.parametrize("over,status,frag", [
+    (dict(abi_version=99), 1, "abi"),
+    (dict(hidden=48), 1, "hidden"),
+    (dict(moe_inter=0), 1, "moe_inter"),
+    (dict(num_experts=0), 1, "num_experts"),
+    (dict(num_experts=300), 1, "num_experts"),
+    (dict(top_k=9), 1, "top_k"),
+    (dict(top_k=5), 1, "top_k"),           # > num_experts (4)
+    (dict(max_tokens=17), 1, "max_tokens"),
+    (dict(max_tokens=0), 1, "max_tokens"),
+    (dict(expert_fmt=2), 1, "expert_fmt"),
+    (dict(score=3), 1, "score"),
+    (dict(bias_mode=7), 1, "bias_mode"),
+    (dict(act=5), 1, "act"),
+    (dict(act=1, act_limit=-1.0), 1, "clamped"),
+    (dict(shared_inter=40), 1, "shared_inter"),
+    (dict(hidden=32768), 2, "hidden"),
+    (dict(weights_mem=3), 1, "weights_mem"),
+])
+def test_open_time_refusals(B, over, status, frag):
+    st, msg = B.validate(SHAPE, _small_layers(SHAPE), **over)
+    assert st == status, msg
+    assert frag in msg
+
+
+def test_bias_and_shared_consistency(B):
+    L = _small_layers(SHAPE)
+    st, msg = B.validate(SHAPE, L, bias_mode=1)
+    assert st == 1 and "router_bias" in msg
+    L[0].bias = np.array([0.1, np.inf, 0.0, 0.0], np.float32)
+    st, msg = B.validate(SHAPE.replace(bias_mode=1), L, bias_mode=1)
+    assert st == 1 and "non-finite" in msg
+    L[0].bias = np.zeros(4, np.float32)
+    st, msg = B.validate(SHAPE.replace(bias_mode=1), L, bias_mode=1)
+    assert st == 0, msg
+    # shared expert: flags and blobs must agree; MXFP4 + shared is refused as unsupported
+    Ls = _small_layers(SHAPE.replace(shared_inter=64))
+    st, msg = B.validate(SHAPE, Ls)
+    assert st == 1 and "shared" in msg
+    st, msg = B.validate(SHAPE, _small_layers(SHAPE), shared_inter=64)
+    assert st == 1 and "shared" in msg
+    shm = SHAPE.replace(shared_inter=64, expert_fmt=synth.FMT_MXFP4, cfg_id=78)
+    st, msg = B.validate(shm, _small_layers(shm))
+    assert st == 2 and "shared" in msg
+    ok = SHAPE.replace(shared_inter=64)
+    assert B.validate(ok, _small_layers(ok))[0] == 0
+
+
+def test_open_without_gpu_fails_cleanly(B):
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(B.TsMoeError) as ei:
+        B.MoE(SHAPE, _small_layers(SHAPE))
+    assert ei.value.status == 4
+
+
+@pytest.mark.parametrize("U,NB", [(1, 148), (7, 148), (147, 148), (148, 148), (149, 148), (1000, 148), (5040, 148),
+                                  (32, 3), (100, 7), (123457, 148)])
+def test_partition_covers_every_unit_once(B, U, NB):
+    lib = B.lib
+    starts = [lib.ts_moe_debug_range_start(U, NB, b) for b in range(NB + 1)]
+    assert starts[0] == 0 and starts[-1] == U
+    assert all(starts[b] <= starts[b + 1] for b in range(NB))
+    sizes = [starts[b + 1] - starts[b] for b in range(NB)]
+    assert max(sizes) - min(sizes) <= 1               # balanced to one unit
+    for u in list(range(min(U, 400))) + [U - 1]:
+        b = lib.ts_moe_debug_owner_of(U, NB, u)
+        assert starts[b] <= u < starts[b + 1]
+
+
+@pytest.mark.parametrize("chunks,ngroups,NB", [(8, 4, 148), (45, 96, 148), (45, 672, 148), (44, 400, 148),
+                                                (448, 128, 148), (3, 5, 4), (64, 1, 148)])
+def test_split_groups_use_distinct_slots(B, chunks, ngroups, NB):
+    """Every CTA writes at most one partial per slot, and the last contributor of
+    a group finds exactly the CTAs that worked on it (empty ranges skipped)."""
+    lib = B.lib
+    U = chunks * ngroups
+    starts = [lib.ts_moe_debug_range_start(U, NB, b) for b in range(NB + 1)]
+    used = {}
+    for G in range(ngroups):
+        g0, g1 = G * chunks, (G + 1) * chunks
+        workers = [b for b in range(NB) if starts[b] < starts[b + 1] and starts[b] < g1 and starts[b + 1] > g0]
+        bf = lib.ts_moe_debug_owner_of(U, NB, g0)
+        bl = lib.ts_moe_debug_owner_of(U, NB, g1 - 1)
+        found = [b for b in range(bf, bl + 1) if starts[b] != starts[b + 1]]
+        assert found == workers
+        if len(workers) > 1:
+            for b in workers:
+                s = lib.ts_moe_debug_partial_slot(U, NB, b, g0)
+                assert (b, s) not in used, (b, s, G, used.get((b, s)))
+                used[(b, s)] = G
+                covered = min(g1, starts[b + 1]) - max(g0, starts[b])
+                assert covered > 0
+            assert sum(min(g1, starts[b + 1]) - max(g0, starts[b]) for b in workers) == chunks
+
+
+def test_group_sizes_divide_or_cap():
+    from quantized_moe_routed_router_b200 import binding as B
+    for tiles in (1, 8, 15, 16, 17, 32, 88, 176, 180, 352, 360, 1792, 97):
+        gs = B.lib.ts_moe_debug_group_size(tiles)
+        assert 1 <= gs <= 16
+        if tiles <= 16:
+            assert gs == tiles
+        elif any(tiles % g == 0 for g in range(8, 17)):
+            assert tiles % gs == 0 and gs >= 8
+        else:
+            assert gs == 16

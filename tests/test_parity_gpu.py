@@ -1,0 +1,162 @@
+"""GPU parity: the CUDA path (through the C ABI) against the FP64 oracle on
+seeded inputs -- small shapes that still span several tiles, groups and a
+ragged tail, every edge the kernels branch on, and the five workloads at full
+size (the 24-layer stack on sampled layers)."""
+import numpy as np
+import pytest
+import torch
+
+from quantized_moe_routed_router_b200 import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+S = synth.MoEShape
+Q8, MX = synth.FMT_Q8_0, synth.FMT_MXFP4
+
+SMALL = {
+    # name: shape  (cfg_id only seeds the draws)
+    "q8_sel": S("q8_sel", 256, 256, 8, 2, cfg_id=101),
+    "mx_odd_blocks_clamped_bias": S("mx", 96, 160, 5, 3, expert_fmt=MX, bias_mode=1, act=1, cfg_id=102),
+    "q8_select_only_bias": S("q8so", 128, 192, 16, 4, bias_mode=2, cfg_id=103),
+    "q8_all_norenorm_shared": S("ds", 128, 96, 16, 6, score=1, shared_inter=96, cfg_id=104),
+    "k_equals_e": S("kee", 64, 128, 4, 4, cfg_id=105),
+    "one_expert": S("one", 64, 64, 1, 1, cfg_id=106),
+    "e256_k8": S("e256", 128, 64, 256, 8, cfg_id=107),
+    "mx_large_k_window_split": S("mxk", 1088, 96, 4, 2, expert_fmt=MX, cfg_id=108),
+    "q8_wide_inter": S("q8w", 64, 2080, 3, 2, cfg_id=109),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from quantized_moe_routed_router_b200 import build
+    build.build()
+    from oracle import oracle
+    oracle.build()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("M", [1, 3, 9, 16])
+def test_small_shapes(name, M):
+    shape = SMALL[name]
+    rep = parity.check_shape(shape, M)
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
+def test_small_with_xscale_and_per_expert_scale():
+    from quantized_moe_routed_router_b200 import binding
+    shape = S("xs", 128, 128, 8, 3, bias_mode=1, cfg_id=110)
+    L = synth.make_layer(shape, 0, device="cuda")
+    rng = np.random.default_rng(3)
+    L.pes = rng.uniform(0.5, 1.5, 8).astype(np.float32)
+    L.xscale = synth.bf16_bits_np(torch.tensor(rng.uniform(0.5, 2.0, 128), dtype=torch.float32).to(torch.bfloat16))
+    moe = binding.MoE(shape, [L])
+    rep = parity.check_shape(shape, 16, moe=moe, layers=[L])
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
+def test_m0_is_a_noop_and_bad_calls_are_refused():
+    from quantized_moe_routed_router_b200 import binding
+    shape = SMALL["q8_sel"]
+    moe = binding.MoE(shape, [synth.make_layer(shape, 0, device="cuda")])
+    x = synth.make_x(shape, 0, 4, device="cuda")
+    y = torch.full((4, shape.hidden), 7.0, device="cuda")
+    moe.forward(0, x, None, y, M=0)
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+    with pytest.raises(binding.TsMoeError):
+        moe.forward(1, x, None, y)                       # layer out of range
+    with pytest.raises(binding.TsMoeError):
+        moe.forward(0, synth.make_x(shape, 0, 17, device="cuda"), None, torch.zeros(17, 256, device="cuda"))
+    with pytest.raises(binding.TsMoeError):
+        moe.forward(0, x, None, None)                    # no output
+    moe.device_status()
+
+
+def test_deterministic_and_route_consistent():
+    from quantized_moe_routed_router_b200 import binding
+    shape = synth.CONFIGS[3].replace(cfg_id=111)
+    L = [synth.make_layer(shape, 0, device="cuda")]
+    moe = binding.MoE(shape, L)
+    x = synth.make_x(shape, 0, 16, device="cuda")
+    ys = []
+    for _ in range(3):
+        y = torch.empty(16, shape.hidden, device="cuda")
+        moe.forward(0, x, None, y)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    idx = torch.empty(16, 4, dtype=torch.int32, device="cuda")
+    w = torch.empty(16, 4, device="cuda")
+    moe.route(0, x, idx, w)
+    y1 = torch.empty_like(ys[0])
+    moe.forward(0, x, None, y1)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, ys[0])
+
+
+def test_cuda_graph_capture_matches_eager():
+    from quantized_moe_routed_router_b200 import binding
+    shape = synth.CONFIGS[4].replace(cfg_id=112)
+    L = [synth.make_layer(shape, 0, device="cuda")]
+    moe = binding.MoE(shape, L)
+    x = synth.make_x(shape, 0, 16, device="cuda")
+    y_e = torch.empty(16, shape.hidden, device="cuda")
+    moe.forward(0, x, None, y_e)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    y_g = torch.zeros_like(y_e)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            moe.forward(0, x, None, y_g, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y_g, y_e)
+    moe.device_status()
+
+
+def test_batch_rows_match_single_token_calls():
+    from quantized_moe_routed_router_b200 import binding
+    shape = SMALL["mx_odd_blocks_clamped_bias"]
+    L = [synth.make_layer(shape, 0, device="cuda")]
+    moe = binding.MoE(shape, L)
+    x = synth.make_x(shape, 0, 16, device="cuda")
+    yb = torch.empty(16, shape.hidden, device="cuda")
+    moe.forward(0, x, None, yb)
+    rms = yb.pow(2).mean().sqrt()
+    for m in range(16):
+        y1 = torch.empty(1, shape.hidden, device="cuda")
+        moe.forward(0, x[m:m + 1].contiguous(), None, y1)
+        assert (y1[0] - yb[m]).abs().max() <= 1e-4 * rms
+
+
+# --------------------------------------------------------------------------- the five workloads at full size
+
+@pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 16), (4, 16)])
+def test_workload_full_size(cfg, M):
+    shape = synth.CONFIGS[cfg]
+    if M > shape.max_tokens:
+        shape = shape.replace(max_tokens=M)
+    rep = parity.check_shape(shape, M)
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
+def test_workload_24_layer_stack_sampled():
+    """The 24-layer gpt-oss-shaped stack in the launch configuration the
+    benchmark times (one handle, all layers resident, M = 16 and M = 1): every
+    layer's outputs are checked on sampled tokens against the oracle."""
+    from quantized_moe_routed_router_b200 import binding
+    shape = synth.CONFIGS[5]
+    layers = [synth.make_layer(shape, l, device="cuda") for l in range(shape.num_layers)]
+    moe = binding.MoE(shape, layers)
+    rng = np.random.default_rng(5)
+    for M in (16, 1):
+        for l in range(shape.num_layers):
+            rows = [0] if M == 1 else sorted(rng.choice(16, 2, replace=False).tolist())
+            if l in (0, 11, 23):
+                rows = None                              # whole micro-batch on three layers
+            rep = parity.check_shape(shape, M, layer=l, rows=rows, moe=moe, layers=layers)
+            assert rep.max_err_y <= 1e-2 * rep.rms_y
+    moe.close()
