@@ -167,6 +167,9 @@ class MoE:
             self._check(lib.ts_moe_set_timing_events(self.h, None))
             return
         self._evs = list(events)
+        for e in self._evs:
+            if not e.cuda_event:          # torch creates the CUDA event on first record
+                e.record()
         arr = (C.c_void_p * 4)(*[e.cuda_event for e in self._evs])
         self._check(lib.ts_moe_set_timing_events(self.h, arr))
 

@@ -23,7 +23,7 @@ namespace tsm {
 
 constexpr int UNIT_BYTES = 544;       // one (tile, chunk): 512 B quants + 32 B scales
 constexpr int QUANT_BYTES = 512;
-constexpr int GS_MAX = 16;            // tiles per group (= consumer warps x tiles per warp)
+constexpr int GS_MAX = 30;            // tiles per group (= consumer warps x tiles per warp)
 constexpr int MAX_TOK = 16;
 constexpr int MAX_K = 8;
 constexpr int MAX_E = 256;
@@ -42,11 +42,11 @@ struct MatGeom {
   uint64_t bytes;  // bytes per expert matrix = tiles * chunks * 544
 };
 
-// Largest tile count per group in [8, 16] that divides `tiles` (equal groups
-// keep the work partition balanced); otherwise 16 with a short last group.
+// Largest tile count per group in [15, 30] that divides `tiles` (equal groups
+// keep the work partition balanced); otherwise 30 with a short last group.
 inline int pick_group_size(int tiles) {
   if (tiles <= GS_MAX) return tiles;
-  for (int g = GS_MAX; g >= 8; --g)
+  for (int g = GS_MAX; g >= GS_MAX / 2; --g)
     if (tiles % g == 0) return g;
   return GS_MAX;
 }
@@ -70,9 +70,10 @@ TSM_HD int group_tiles(int tiles, int gs, int grp) {
 }
 
 // ----------------------------------------------------------------------------- stream-K partition
-// The units of one launch (all touched entries' (group, chunk) pairs, entries
-// in order, groups in order, chunks in order) are split into NB contiguous
-// ranges: block b owns [range_start(b), range_start(b + 1)).
+// The units of one launch -- every touched entry's (group, chunk) pairs, in
+// entry-major order (entry, group, chunk) for gate/up and group-major order
+// (group, entry, chunk) for down -- are split into NB contiguous ranges:
+// block b owns [range_start(b), range_start(b + 1)).
 TSM_HD uint64_t range_start(uint64_t U, int NB, int b) { return (uint64_t)b * U / (uint64_t)NB; }
 
 // The block whose range contains unit u (0 <= u < U): the largest b with

@@ -25,11 +25,13 @@ namespace tsm {
 enum : unsigned { BAD_E8M0_NAN = 1u, BAD_Q8_SCALE = 2u, BAD_ROUTER_SCALE = 4u };
 
 // PHASE 0: tile t rows 0..7 = gate rows 8t..8t+7, rows 8..15 = up rows
-// 8t..8t+7 (matrices [rows][row_bytes]); PHASE 1: tile t rows = down rows
-// 16t..16t+15.
+// 8t..8t+7 (matrices [rows][row_bytes]); PHASE 1: tile t rows = rows
+// 16t..16t+15 of a [nrows][row_bytes] matrix (down, or the router); tile rows
+// at or past nrows repack as zero weights with zero scale.
 template <int FMT, int PHASE>
 __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ b, int row_bytes,
-                              int nblocks, int tiles, int chunks, int gs, uint8_t* __restrict__ dst, unsigned* bad) {
+                              int nblocks, int tiles, int chunks, int gs, uint8_t* __restrict__ dst, unsigned* bad,
+                              int nrows) {
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const long long total = (long long)tiles * chunks;
@@ -42,12 +44,15 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
     uint8_t* unit = dst + group_offset(gs, chunks, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
     const uint8_t* rg;
     const uint8_t* rg8;
+    bool zg = false, zg8 = false;
     if (PHASE == 0) {
       rg = a + (size_t)(8 * t + g) * row_bytes;
       rg8 = b + (size_t)(8 * t + g) * row_bytes;
     } else {
-      rg = a + (size_t)(16 * t + g) * row_bytes;
-      rg8 = a + (size_t)(16 * t + g + 8) * row_bytes;
+      zg = 16 * t + g >= nrows;
+      zg8 = 16 * t + g + 8 >= nrows;
+      rg = a + (size_t)(zg ? 0 : 16 * t + g) * row_bytes;
+      rg8 = a + (size_t)(zg8 ? 0 : 16 * t + g + 8) * row_bytes;
     }
     uint32_t w[4];
     if (FMT == 1) {
@@ -58,6 +63,8 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
         if (blk < nblocks) {
           const int o = blk * 17 + 1 + 8 * (s % 2) + 2 * c;
           v = (uint32_t)rg[o] | ((uint32_t)rg8[o] << 8) | ((uint32_t)rg[o + 1] << 16) | ((uint32_t)rg8[o + 1] << 24);
+          if (zg) v &= 0xFF00FF00u;
+          if (zg8) v &= 0x00FF00FFu;
         }
         w[s] = v;
       }
@@ -71,6 +78,14 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
                     ((uint32_t)qg8[o + 1] << 24)) ^ 0x80808080u;
         w[2 * s + 1] = ((uint32_t)qg[o + 2] | ((uint32_t)qg[o + 3] << 8) | ((uint32_t)qg8[o + 2] << 16) |
                         ((uint32_t)qg8[o + 3] << 24)) ^ 0x80808080u;
+        if (zg) {  // q = 0 is stored as 0x80
+          w[2 * s] = (w[2 * s] & 0xFFFF0000u) | 0x8080u;
+          w[2 * s + 1] = (w[2 * s + 1] & 0xFFFF0000u) | 0x8080u;
+        }
+        if (zg8) {
+          w[2 * s] = (w[2 * s] & 0x0000FFFFu) | 0x80800000u;
+          w[2 * s + 1] = (w[2 * s + 1] & 0x0000FFFFu) | 0x80800000u;
+        }
       }
     }
     *reinterpret_cast<uint4*>(unit + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -78,12 +93,15 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
       // scales of the quad of rows (lane, lane + 8)
       const uint8_t* sg;
       const uint8_t* sg8;
+      bool zs = false, zs8 = false;
       if (PHASE == 0) {
         sg = a + (size_t)(8 * t + lane) * row_bytes;
         sg8 = b + (size_t)(8 * t + lane) * row_bytes;
       } else {
-        sg = a + (size_t)(16 * t + lane) * row_bytes;
-        sg8 = a + (size_t)(16 * t + lane + 8) * row_bytes;
+        zs = 16 * t + lane >= nrows;
+        zs8 = 16 * t + lane + 8 >= nrows;
+        sg = a + (size_t)(zs ? 0 : 16 * t + lane) * row_bytes;
+        sg8 = a + (size_t)(zs8 ? 0 : 16 * t + lane + 8) * row_bytes;
       }
       uint32_t sw;
       if (FMT == 1) {
@@ -96,34 +114,19 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
           e[2] = sg[(2 * ck + 1) * 17];
           e[3] = sg8[(2 * ck + 1) * 17];
         }
+        if (zs) e[0] = e[2] = 0;
+        if (zs8) e[1] = e[3] = 0;
         for (int i = 0; i < 4; ++i)
           if (e[i] == 255u) mybad |= BAD_E8M0_NAN;
         sw = e[0] | (e[1] << 8) | (e[2] << 16) | (e[3] << 24);
       } else {
-        const uint32_t d0 = (uint32_t)sg[ck * 34] | ((uint32_t)sg[ck * 34 + 1] << 8);
-        const uint32_t d1 = (uint32_t)sg8[ck * 34] | ((uint32_t)sg8[ck * 34 + 1] << 8);
+        const uint32_t d0 = zs ? 0u : (uint32_t)sg[ck * 34] | ((uint32_t)sg[ck * 34 + 1] << 8);
+        const uint32_t d1 = zs8 ? 0u : (uint32_t)sg8[ck * 34] | ((uint32_t)sg8[ck * 34 + 1] << 8);
         if ((d0 & 0x7C00u) == 0x7C00u || (d1 & 0x7C00u) == 0x7C00u) mybad |= BAD_Q8_SCALE;
         sw = d0 | (d1 << 16);
       }
       *reinterpret_cast<uint32_t*>(unit + QUANT_BYTES + lane * 4) = sw;
     }
-  }
-  if (mybad) atomicOr(bad, mybad);
-}
-
-// Router [E][H] Q8_0 -> int8 plane [E][H] + FP32 block scales [E][H/32].
-__global__ void repack_router_kernel(const uint8_t* __restrict__ src, int E, int H, int8_t* __restrict__ q,
-                                     float* __restrict__ d, unsigned* bad) {
-  const int nb = H / 32;
-  const long long total = (long long)E * nb;
-  unsigned mybad = 0;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
-    const int e = (int)(i / nb), blk = (int)(i % nb);
-    const uint8_t* p = src + ((size_t)e * nb + blk) * 34;
-    const unsigned short bits = (unsigned short)(p[0] | (p[1] << 8));
-    if ((bits & 0x7C00u) == 0x7C00u) mybad |= BAD_ROUTER_SCALE;
-    d[i] = __half2float(__ushort_as_half(bits));
-    for (int k = 0; k < 32; ++k) q[(size_t)e * H + blk * 32 + k] = (int8_t)p[2 + k];
   }
   if (mybad) atomicOr(bad, mybad);
 }

@@ -1,9 +1,14 @@
 // Route kernel: router GEMV -> (bias) -> top-k + weights -> route list.
 //
-// One CTA per token.  The router GEMV reads the Q8_0 router rows (int8 plane
-// + FP32 block scales, repacked at open) against x * router_xscale in FP32
-// (llama state page, `router_ones`: the INT8 router kernel scales x[n] per
-// element; `router_logits_f32`: one FP32 row of logits per token).  One warp
+// One CTA does the whole micro-batch.  The router GEMV runs on the tensor
+// cores: the Q8_0 router is repacked at open into the same 16-row MMA
+// fragment layout as the experts (rows past E are zero), x * router_xscale is
+// staged in shared memory as FP16 scaled by a per-token power of two (|x| max
+// lands in [2^13, 2^14); with a non-trivial xscale the product is split into
+// an FP16 hi + lo pair so it stays exact), and the FP32 logits come out of
+// m16n8k16 MMAs with the block scale folded in per 32-block (llama state page,
+// `router_ones`: the INT8 router kernel scales x[n] per element;
+// `router_logits_f32`: one FP32 row of logits per token).  One warp per token
 // then selects the top K by (selection logit desc, index asc), where the
 // selection logit is l + b when a router bias is present (gpt-oss state page,
 // `router_bias`: added BEFORE the top-k), and forms the weights:
@@ -13,16 +18,15 @@
 // times the per-expert scale.  The reference does this part on the host after
 // reading the logits back; here it never leaves the device.
 //
-// The last CTA to finish (one atomic counter, no waiting) groups the M*K
-// (token, slot) pairs by expert into the route list the expert kernels walk:
-// per touched expert its first route and count, routes sorted by (expert,
-// token) -- each expert's weights are then streamed once per micro-batch.
-// The pages' route list is a host-written 16-byte record per route
-// (gpt-oss state page, `batch_routes`); ours is built on the device.
+// The same CTA then groups the M*K (token, slot) pairs by expert into the
+// route list the expert kernels walk: per touched expert its first route and
+// count, routes sorted by (expert, token) -- each expert's weights are then
+// streamed once per micro-batch.  The pages' route list is a host-written
+// 16-byte record per route (gpt-oss state page, `batch_routes`); ours is
+// built on the device.
 //
-// Each CTA also writes its token's x as FP16 scaled by a power of two
-// 2^shift (|x| max lands in [2^13, 2^14)), the B operand of the gate/up
-// tensor-core MMA; the shift is undone exactly in that kernel's epilogue.
+// It also writes x as FP16 with the same per-token scale (no xscale), the B
+// operand of the gate/up MMA; that kernel undoes the shift exactly.
 #pragma once
 #include "common.cuh"
 #include "layout.cuh"
@@ -36,16 +40,16 @@ struct Route {
   float w;
 };
 
-// meta[] layout (int32), written by the route kernel's last CTA.
+// meta[] layout (int32), written by the route kernel.
 enum { META_M = 0, META_NT = 1, META_MK = 2, META_HAS_SHARED = 3, META_NE = 4, META_EX = 8,
        META_RO = META_EX + MAX_ENTRIES, META_NC = META_RO + MAX_ENTRIES, META_INTS = META_NC + MAX_ENTRIES };
 
 struct RouteParams {
   const __nv_bfloat16* x;  // [M][H]
   int M, H, Hp, E, K;
-  const int8_t* rq;        // [E][H] router quants
-  const float* rd;         // [E][H/32] router block scales
-  const float* xscale;     // [H] or null
+  const uint8_t* rw;       // router, repacked Q8_0 fragment tiles (rows padded to 16)
+  MatGeom rg;              // its geometry
+  const float* xscale;     // [H] or null (null = ones)
   const float* bias;       // [E] or null
   const float* pes;        // [E] or null
   int bias_mode, score, has_shared;
@@ -57,7 +61,6 @@ struct RouteParams {
   int* meta;
   Route* routes;           // [M*K]
   int* rpos;               // [M][K] -> position in routes
-  unsigned* cnt;
   unsigned* err;
   int* idx_out;            // optional user outputs
   float* w_out;
@@ -66,88 +69,281 @@ struct RouteParams {
 
 TSM_DEV bool topk_better(float v1, int i1, float v2, int i2) { return v1 > v2 || (v1 == v2 && i1 < i2); }
 
-constexpr int ROUTE_THREADS = 256;
+constexpr int ROUTE_THREADS = 512;
+constexpr int ROUTE_WARPS = ROUTE_THREADS / 32;
+constexpr int RKW = 2048;                 // K elements of x staged per window
+constexpr int RROW = RKW * 2 + 32;        // bytes per staged row (= 32 mod 128: conflict-free B loads)
+constexpr int ROUTE_PRE = 6;              // router units per warp fetched before x is ready
 
-__global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const RouteParams p) {
-  extern __shared__ float rsm[];
-  float* xs = rsm;          // [H] router input x * xscale
-  float* lg = rsm + p.H;    // [E] logits
-  __shared__ float red[ROUTE_THREADS / 32];
-  __shared__ int s_last;
-  __shared__ int s_cnt[MAX_E], s_off[MAX_E], s_idx[MAX_TOK * MAX_K];
+// Shared memory of the route kernel (dynamic).
+struct RouteSmem {
+  uint8_t xw[2][MAX_TOK][RROW];           // staged x window: [hi/lo][token][K]
+  float part[ROUTE_WARPS][16][16];        // per-warp partial logits [row][token]
+  float lg[MAX_TOK][MAX_E];               // logits
+  int shift[MAX_TOK];
+  int cnt[MAX_E], off[MAX_E], idx[MAX_TOK * MAX_K];
+};
+
+// Stages x[t][k0 .. k0+len) (FP32 product with xscale, times 2^shift[t]) as
+// FP16 hi (+ lo when `split`) into the window; also writes xh when `write_xh`.
+TSM_DEV void stage_window(RouteSmem& s, const RouteParams& p, int k0, int len, bool split, bool write_xh) {
+  constexpr int U = 4;  // items (8 elements each) per thread per trip, loads issued together
+  const int per_row = len / 8, total = p.M * per_row;
+  for (int base = threadIdx.x; base < total; base += ROUTE_THREADS * U) {
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * ROUTE_THREADS;
+      raw[u] = make_uint4(0, 0, 0, 0);
+      if (i < total) {
+        const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
+        if (k < p.H) raw[u] = *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * ROUTE_THREADS;
+      if (i >= total) break;
+      const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
+      const float sc = __uint_as_float((uint32_t)(s.shift[t] + 127) << 23);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+      __half hx[8], hh[8], hl[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(b2[q]);
+        hx[2 * q] = __float2half_rn(f.x * sc);
+        hx[2 * q + 1] = __float2half_rn(f.y * sc);
+        if (split) {
+          const bool in = k + 2 * q < p.H;
+          const float xa = f.x * (in ? p.xscale[k + 2 * q] : 1.f) * sc;
+          const float xb = f.y * (in ? p.xscale[k + 2 * q + 1] : 1.f) * sc;
+          hh[2 * q] = __float2half_rn(xa);
+          hh[2 * q + 1] = __float2half_rn(xb);
+          hl[2 * q] = __float2half_rn(xa - __half2float(hh[2 * q]));
+          hl[2 * q + 1] = __float2half_rn(xb - __half2float(hh[2 * q + 1]));
+        }
+      }
+      if (write_xh) *reinterpret_cast<uint4*>(p.xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
+      *reinterpret_cast<uint4*>(&s.xw[0][t][(k - k0) * 2]) = *reinterpret_cast<uint4*>(split ? hh : hx);
+      if (split) *reinterpret_cast<uint4*>(&s.xw[1][t][(k - k0) * 2]) = *reinterpret_cast<uint4*>(hl);
+    }
+  }
+}
+
+// One Q8_0 (tile, chunk) unit against the staged window: acc += W x.
+template <int NT>
+TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const uint8_t* xc, int lane) {
+  const int g = lane >> 2, c = lane & 3;
+  const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&sc));
+  float tmp[NT][4];
+  const uint32_t a0[4] = {u8x2_to_f16x2<0x4140>(q.x), u8x2_to_f16x2<0x4342>(q.x), u8x2_to_f16x2<0x4140>(q.y),
+                          u8x2_to_f16x2<0x4342>(q.y)};
+  const uint32_t a1[4] = {u8x2_to_f16x2<0x4140>(q.z), u8x2_to_f16x2<0x4342>(q.z), u8x2_to_f16x2<0x4140>(q.w),
+                          u8x2_to_f16x2<0x4342>(q.w)};
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const uint2 b0 = *reinterpret_cast<const uint2*>(xc + (nt * 8 + g) * RROW + (4 * c) * 2);
+    const uint2 b1 = *reinterpret_cast<const uint2*>(xc + (nt * 8 + g) * RROW + (16 + 4 * c) * 2);
+    mma_f16_zc(tmp[nt], a0, b0.x, b0.y);
+    mma_f16_acc(tmp[nt], a1, b1.x, b1.y);
+    acc[nt][0] = fmaf(d.x, tmp[nt][0], acc[nt][0]);
+    acc[nt][1] = fmaf(d.x, tmp[nt][1], acc[nt][1]);
+    acc[nt][2] = fmaf(d.y, tmp[nt][2], acc[nt][2]);
+    acc[nt][3] = fmaf(d.y, tmp[nt][3], acc[nt][3]);
+  }
+}
+
+// Router work split: warp w owns tile w / wpt and every wpt-th chunk of it.
+struct RouterSplit {
+  int T, C, wpt, tile, wsub, nunits;
+  TSM_DEV RouterSplit(const MatGeom& g, int warp) {
+    T = g.tiles;
+    C = g.chunks;
+    wpt = ROUTE_WARPS / T;  // warps per tile (T <= 16)
+    tile = warp / wpt;
+    wsub = warp % wpt;
+    nunits = tile < T ? (C - wsub + wpt - 1) / wpt : 0;
+  }
+  TSM_DEV const uint8_t* unit(const RouteParams& p, int k) const {
+    const int ck = wsub + k * wpt;
+    const int grp = tile / p.rg.gs, jt = tile % p.rg.gs, ntg = group_tiles(T, p.rg.gs, grp);
+    return p.rw + group_offset(p.rg.gs, C, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
+  }
+};
+
+// Router GEMV over all tokens from the staged windows; pq/ps hold the warp's
+// first ROUTE_PRE units (fetched at kernel start).
+template <int NT>
+TSM_DEV void router_gemv(RouteSmem& s, const RouteParams& p, bool split, int warp, int lane, const RouterSplit& rs,
+                         const uint4 (&pq)[ROUTE_PRE], const uint32_t (&ps)[ROUTE_PRE]) {
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  const int nwin = (rs.C * 32 + RKW - 1) / RKW;
+  for (int wdw = 0; wdw < nwin; ++wdw) {
+    const int k0 = wdw * RKW, len = min(RKW, p.Hp - k0);
+    if (wdw > 0) {
+      __syncthreads();
+      stage_window(s, p, k0, len, split, false);
+    }
+    __syncthreads();
+    for (int half = 0; half < (split ? 2 : 1); ++half) {
+#pragma unroll
+      for (int k = 0; k < ROUTE_PRE; ++k) {
+        const int ck = rs.wsub + k * rs.wpt;
+        if (k < rs.nunits && ck * 32 >= k0 && ck * 32 < k0 + len)
+          router_unit<NT>(acc, pq[k], ps[k], &s.xw[half][0][(ck * 32 - k0) * 2], lane);
+      }
+      for (int kb = ROUTE_PRE; kb < rs.nunits; kb += 4) {  // the rest, four loads in flight at a time
+        uint4 q[4];
+        uint32_t sc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (kb + k < rs.nunits) {
+            const uint8_t* u = rs.unit(p, kb + k);
+            q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
+            sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
+          }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int ck = rs.wsub + (kb + k) * rs.wpt;
+          if (kb + k < rs.nunits && ck * 32 >= k0 && ck * 32 < k0 + len)
+            router_unit<NT>(acc, q[k], sc[k], &s.xw[half][0][(ck * 32 - k0) * 2], lane);
+        }
+      }
+    }
+  }
+  const int gq = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    s.part[warp][gq][nt * 8 + 2 * c] = acc[nt][0];
+    s.part[warp][gq][nt * 8 + 2 * c + 1] = acc[nt][1];
+    s.part[warp][gq + 8][nt * 8 + 2 * c] = acc[nt][2];
+    s.part[warp][gq + 8][nt * 8 + 2 * c + 1] = acc[nt][3];
+  }
+  __syncthreads();
+  // logits[t][e] = sum over the tile's warps in order, times 2^-shift[t]
+  for (int i = threadIdx.x; i < p.M * p.E; i += ROUTE_THREADS) {
+    const int t = i / p.E, e = i - t * p.E;
+    const int tl = e >> 4, r = e & 15;
+    float v = 0.f;
+    for (int w = 0; w < rs.wpt; ++w) v += s.part[tl * rs.wpt + w][r][t];
+    s.lg[t][e] = v * __uint_as_float((uint32_t)(127 - s.shift[t]) << 23);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RouteParams p) {
+  extern __shared__ __align__(128) uint8_t route_smem_raw[];
+  RouteSmem& s = *reinterpret_cast<RouteSmem*>(route_smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // The router does not depend on the previous kernel: fetch this warp's first units now.
+  const RouterSplit rs(p.rg, warp);
+  uint4 pq[ROUTE_PRE];
+  uint32_t ps[ROUTE_PRE];
+#pragma unroll
+  for (int k = 0; k < ROUTE_PRE; ++k)
+    if (k < rs.nunits) {
+      const uint8_t* u = rs.unit(p, k);
+      pq[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
+      ps[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
+    }
 
   grid_dep_wait();
   grid_dep_launch();
 
-  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const __nv_bfloat16* xr = p.x + (size_t)t * p.H;
-
-  // ---- x: router input, |x| max
-  float amax = 0.f;
-  for (int n = tid; n < p.H; n += ROUTE_THREADS) {
-    float v = __bfloat162float(xr[n]);
-    amax = fmaxf(amax, fabsf(v));
-    xs[n] = p.xscale ? v * p.xscale[n] : v;
-  }
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) red[warp] = amax;
-  __syncthreads();
-  amax = red[0];
-  for (int i = 1; i < ROUTE_THREADS / 32; ++i) amax = fmaxf(amax, red[i]);
-  int sh = 0;
-  if (amax > 0.f && amax <= 3.4e38f) {
-    int e2;
-    frexpf(amax, &e2);  // amax in [2^(e2-1), 2^e2)
-    sh = min(126, max(-126, 14 - e2));
-  }
-  const float xsc = __uint_as_float((uint32_t)(sh + 127) << 23);
-  __half* xhr = p.xh + (size_t)t * p.Hp;
-  for (int n = tid; n < p.Hp; n += ROUTE_THREADS)
-    xhr[n] = n < p.H ? __float2half_rn(__bfloat162float(xr[n]) * xsc) : __ushort_as_half(0);
-  if (tid == 0) p.shift[t] = sh;
-  __syncthreads();
-
-  // ---- router GEMV: warp per expert, lane per 32-block
-  const int nb = p.H / 32;
-  for (int e = warp; e < p.E; e += ROUTE_THREADS / 32) {
-    const int8_t* q = p.rq + (size_t)e * p.H;
-    const float* d = p.rd + (size_t)e * nb;
-    float acc = 0.f;
-    for (int b = lane; b < nb; b += 32) {
-      const int4* qv = reinterpret_cast<const int4*>(q + (size_t)b * 32);
-      int4 qa = qv[0], qb = qv[1];
-      int qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      const float* xb = xs + b * 32;
-      float s = 0.f;
+  // ---- per-token |x| and |x * xscale| max -> power-of-two scale (warp t: token t)
+  if (warp < p.M) {
+    const int t = warp;
+    float m = 0.f;
+    constexpr int U = 4;
+    for (int kb = lane * 8; kb < p.H; kb += 32 * 8 * U) {
+      uint4 raw[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) s = fmaf((float)(int8_t)(qw[i] >> (8 * k)), xb[4 * i + k], s);
+      for (int u = 0; u < U; ++u) {
+        const int k = kb + u * 256;
+        raw[u] = k < p.H ? *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k) : make_uint4(0, 0, 0, 0);
       }
-      acc = fmaf(d[b], s, acc);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int k = kb + u * 256;
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(b2[q]);
+          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          if (p.xscale && k < p.H) {
+            m = fmaxf(m, fabsf(f.x * p.xscale[k + 2 * q]));
+            m = fmaxf(m, fabsf(f.y * p.xscale[k + 2 * q + 1]));
+          }
+        }
+      }
     }
-    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) lg[e] = acc;
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    int sh = 0;
+    if (m > 0.f && m <= 3.4e38f) {
+      int e2;
+      frexpf(m, &e2);  // m in [2^(e2-1), 2^e2)
+      sh = min(126, max(-126, 14 - e2));
+    }
+    if (lane == 0) {
+      s.shift[t] = sh;
+      p.shift[t] = sh;
+    }
   }
   __syncthreads();
+  const bool split = p.xscale != nullptr;
+  // window 0 (and all of xh)
+  stage_window(s, p, 0, min(RKW, p.Hp), split, true);
+  for (int k0 = RKW; k0 < p.Hp; k0 += RKW) {
+    // the rest of xh; windows after the first are restaged inside the GEMV
+    const int len = min(RKW, p.Hp - k0), per_row = len / 8;
+    for (int i = tid; i < p.M * per_row; i += ROUTE_THREADS) {
+      const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
+      const float sc = __uint_as_float((uint32_t)(s.shift[t] + 127) << 23);
+      __half hx[8];
+      if (k < p.H) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(b2[q]);
+          hx[2 * q] = __float2half_rn(f.x * sc);
+          hx[2 * q + 1] = __float2half_rn(f.y * sc);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) hx[q] = __ushort_as_half(0);
+      }
+      *reinterpret_cast<uint4*>(p.xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
+    }
+  }
+  if (p.M > 8)
+    router_gemv<2>(s, p, split, warp, lane, rs, pq, ps);
+  else
+    router_gemv<1>(s, p, split, warp, lane, rs, pq, ps);
 
-  // ---- top-k and weights (warp 0; lane holds experts lane, lane+32, ...)
-  if (warp == 0) {
+  // ---- top-k and weights: warp t handles token t (lane holds experts lane, lane+32, ...)
+  if (warp < p.M) {
+    const int t = warp;
     constexpr int PER = MAX_E / 32;
     float vsel[PER], vsc[PER];
     unsigned taken = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane + 32 * i;
-      float l = e < p.E ? lg[e] : -INFINITY;
-      float ls = (e < p.E && p.bias && p.bias_mode != 0) ? l + p.bias[e] : l;
+      const float l = e < p.E ? s.lg[t][e] : -INFINITY;
+      const float ls = (e < p.E && p.bias && p.bias_mode != 0) ? l + p.bias[e] : l;
       vsel[i] = ls;
       vsc[i] = (p.bias_mode == 1 && p.bias) ? ls : l;
-      if (e < p.E && p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
-      if (e < p.E) p.logits[(size_t)t * p.E + e] = l;
+      if (e < p.E) {
+        p.logits[(size_t)t * p.E + e] = l;
+        if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
+      }
     }
-    int sel[MAX_K];
-    float ssc[MAX_K];
+    int selk = 0;  // lane k holds the k-th selected expert and its score logit
+    float sck = -INFINITY;
     for (int k = 0; k < p.K; ++k) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
@@ -160,8 +356,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const RouteParams 
         }
       }
       for (int o = 16; o; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (topk_better(ov, oi, bv, bi)) {
           bv = ov;
           bi = oi;
@@ -171,105 +367,109 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const RouteParams 
         if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
         bi = 0;
       }
-      sel[k] = bi;
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      // score logit of the chosen expert, from its owner lane
       float mine = 0.f;
 #pragma unroll
       for (int i = 0; i < PER; ++i)
         if (i == (bi >> 5)) mine = vsc[i];
-      ssc[k] = __shfl_sync(0xffffffffu, mine, bi & 31);
-    }
-    float wk[MAX_K];
-    if (p.score == 0) {
-      float m = -INFINITY;
-      for (int k = 0; k < p.K; ++k) m = fmaxf(m, ssc[k]);
-      float den = 0.f;
-      for (int k = 0; k < p.K; ++k) {
-        wk[k] = expf(ssc[k] - m);
-        den += wk[k];
+      const float sc = __shfl_sync(0xffffffffu, mine, bi & 31);
+      if (lane == k) {
+        selk = bi;
+        sck = sc;
       }
-      for (int k = 0; k < p.K; ++k) wk[k] /= den;
-    } else {
-      float m = -INFINITY;
+    }
+    const bool act = lane < p.K;
+    float m = act ? sck : -INFINITY;
+    if (p.score != 0) {
 #pragma unroll
       for (int i = 0; i < PER; ++i)
         if (lane + 32 * i < p.E) m = fmaxf(m, vsc[i]);
-      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float den = 0.f;
+    }
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float den = 0.f;
+    if (p.score == 0) {
+      den = act ? expf(sck - m) : 0.f;
+    } else {
 #pragma unroll
       for (int i = 0; i < PER; ++i)
         if (lane + 32 * i < p.E) den += expf(vsc[i] - m);
-      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-      for (int k = 0; k < p.K; ++k) wk[k] = expf(ssc[k] - m) / den;
     }
-    if (lane == 0) {
-      for (int k = 0; k < p.K; ++k) {
-        const float wv = wk[k] * (p.pes ? p.pes[sel[k]] : 1.f);
-        p.idx[t * p.K + k] = sel[k];
-        p.w[t * p.K + k] = wv;
-        if (p.idx_out) p.idx_out[t * p.K + k] = sel[k];
-        if (p.w_out) p.w_out[t * p.K + k] = wv;
-      }
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (act) {
+      const float wv = expf(sck - m) / den * (p.pes ? p.pes[selk] : 1.f);
+      s.idx[t * p.K + lane] = selk;
+      p.idx[t * p.K + lane] = selk;
+      p.w[t * p.K + lane] = wv;
+      if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
+      if (p.w_out) p.w_out[t * p.K + lane] = wv;
     }
   }
+  for (int e = tid; e < p.E; e += ROUTE_THREADS) s.cnt[e] = 0;
+  __syncthreads();
 
-  // ---- last CTA builds the route list (no waiting: the other CTAs are done)
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(p.cnt, 1u) == (unsigned)(p.M - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  // ---- route list: group the (token, slot) pairs by expert
   const int MK = p.M * p.K;
-  for (int i = tid; i < MK; i += ROUTE_THREADS) s_idx[i] = ld_cg_i(p.idx + i);
-  for (int e = tid; e < p.E; e += ROUTE_THREADS) s_cnt[e] = 0;
+  for (int i = tid; i < MK; i += ROUTE_THREADS) atomicAdd(&s.cnt[s.idx[i]], 1);
   __syncthreads();
-  for (int i = tid; i < MK; i += ROUTE_THREADS) {
-    int e = s_idx[i];
-    if (e < 0 || e >= p.E) {
-      atomicOr(p.err, ERR_BAD_INDEX);
-      e = s_idx[i] = 0;
+  if (warp == 0) {
+    // exclusive scan of the counts and compaction of the touched experts
+    constexpr int PER = MAX_E / 32;
+    int cl[PER], tot = 0, nz = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      cl[i] = e < p.E ? s.cnt[e] : 0;
+      tot += cl[i];
+      nz += cl[i] > 0;
     }
-    atomicAdd(&s_cnt[e], 1);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0, nT = 0;
-    for (int e = 0; e < p.E; ++e) {
-      s_off[e] = run;
-      if (s_cnt[e]) {
-        p.meta[META_EX + nT] = e;
-        p.meta[META_RO + nT] = run;
-        p.meta[META_NC + nT] = s_cnt[e];
-        ++nT;
+    int incl = tot, nzincl = nz;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o), w = __shfl_up_sync(0xffffffffu, nzincl, o);
+      if (lane >= o) {
+        incl += v;
+        nzincl += w;
       }
-      run += s_cnt[e];
     }
-    if (p.has_shared) {
-      p.meta[META_EX + nT] = p.E;
-      p.meta[META_RO + nT] = MK;
-      p.meta[META_NC + nT] = p.M;
+    int run = incl - tot, slot = nzincl - nz;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane * PER + i;
+      if (e < p.E) {
+        s.off[e] = run;
+        if (cl[i]) {
+          p.meta[META_EX + slot] = e;
+          p.meta[META_RO + slot] = run;
+          p.meta[META_NC + slot] = cl[i];
+          ++slot;
+        }
+        run += cl[i];
+      }
     }
-    p.meta[META_M] = p.M;
-    p.meta[META_NT] = nT;
-    p.meta[META_MK] = MK;
-    p.meta[META_HAS_SHARED] = p.has_shared;
-    p.meta[META_NE] = nT + (p.has_shared ? 1 : 0);
-    *p.cnt = 0u;
+    const int nT = __shfl_sync(0xffffffffu, nzincl, 31);
+    if (lane == 0) {
+      if (p.has_shared) {
+        p.meta[META_EX + nT] = p.E;
+        p.meta[META_RO + nT] = MK;
+        p.meta[META_NC + nT] = p.M;
+      }
+      p.meta[META_M] = p.M;
+      p.meta[META_NT] = nT;
+      p.meta[META_MK] = MK;
+      p.meta[META_HAS_SHARED] = p.has_shared;
+      p.meta[META_NE] = nT + (p.has_shared ? 1 : 0);
+    }
   }
   __syncthreads();
   for (int i = tid; i < MK; i += ROUTE_THREADS) {
-    const int e = s_idx[i], tk = i / p.K;
+    const int e = s.idx[i], tk = i / p.K;
     int rank = 0;
-    for (int i2 = 0; i2 < MK; ++i2)
-      if (s_idx[i2] == e && i2 / p.K < tk) ++rank;
-    const int pos = s_off[e] + rank;
+    for (int i2 = 0; i2 < tk * p.K; ++i2) rank += s.idx[i2] == e;
+    const int pos = s.off[e] + rank;
     Route r;
     r.token = tk;
     r.slot = i % p.K;
     r.expert = e;
-    r.w = ld_cg(p.w + i);
+    r.w = p.w[i];
     p.routes[pos] = r;
     p.rpos[i] = pos;
   }

@@ -26,11 +26,11 @@ namespace {
 thread_local std::string g_open_error;
 
 struct LayerDev {
-  int8_t* rq = nullptr;
-  float* rd = nullptr;
+  uint8_t* rw = nullptr;   // router, repacked Q8_0 fragment tiles
   float* bias = nullptr;
   float* pes = nullptr;
   float* xscale = nullptr;
+  bool has_xscale = false; // some router x-scale differs from 1
   uint8_t* wB = nullptr;   // routed gate/up, E matrices
   uint8_t* wC = nullptr;   // routed down
   uint8_t* wBs = nullptr;  // shared gate/up
@@ -47,8 +47,8 @@ struct ts_moe {
   ts_moe_config cfg{};
   int sm_count = 0, nb = 0;
   int Hp = 0, Ip = 0, Sp = 0;
-  MatGeom gB{}, gC{}, gBs{}, gCs{};
-  int ng_max_B = 0, ng_max_C = 0;
+  MatGeom gR{}, gB{}, gC{}, gBs{}, gCs{};
+  int ng_max_B = 0;
   uint8_t* arena = nullptr;
   size_t arena_bytes = 0;
   uint8_t* ws = nullptr;
@@ -67,10 +67,8 @@ struct ts_moe {
   __half* acts_sh = nullptr;
   float* P = nullptr;
   float* partial = nullptr;
-  unsigned* cnt_route = nullptr;
-  unsigned* cnt_gB = nullptr;
-  unsigned* cnt_gC = nullptr;
-  unsigned* cnt_rg = nullptr;
+  unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group) chunk counters
+  unsigned* grid = nullptr;     // down: grid barrier {arrivals, generation}
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
   uint8_t* counters = nullptr;
@@ -173,24 +171,23 @@ ts_moe_status set_smem_attrs(ts_moe* h) {
   TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  const int rbytes = (h->cfg.hidden + h->cfg.num_experts) * 4;
-  if (rbytes > 48 * 1024)
-    TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rbytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)sizeof(RouteSmem)));
   return TS_MOE_OK;
 }
 
 template <int PHASE>
 void launch_repack(int fmt, const uint8_t* a, const uint8_t* b, int row_bytes, int nblocks, const MatGeom& g,
-                   uint8_t* dst, unsigned* bad, cudaStream_t st) {
+                   uint8_t* dst, unsigned* bad, cudaStream_t st, int nrows) {
   const long long units = (long long)g.tiles * g.chunks;
   const int threads = 256;
   const long long blocks = std::min<long long>((units + 7) / 8, 65535LL * 8);
   if (fmt == TS_FMT_MXFP4)
     repack_kernel<1, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
-                                                                                      g.chunks, g.gs, dst, bad);
+                                                                                      g.chunks, g.gs, dst, bad, nrows);
   else
     repack_kernel<0, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
-                                                                                      g.chunks, g.gs, dst, bad);
+                                                                                      g.chunks, g.gs, dst, bad, nrows);
 }
 
 }  // namespace
@@ -223,10 +220,11 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   const int H = c.hidden, I = c.moe_inter, E = c.num_experts, K = c.top_k, S = c.shared_inter, Mx = c.max_tokens;
   const int fmt = c.expert_fmt;
   h->sm_count = prop.multiProcessorCount;
-  h->nb = h->sm_count;
+  h->nb = std::min(h->sm_count, MAX_NB);
   h->Hp = round_up(H, 64);
   h->Ip = round_up(I, 64);
   h->Sp = S ? round_up(S, 64) : 0;
+  h->gR = make_geom((E + 15) / 16, H, TS_FMT_Q8_0);
   h->gB = make_geom(I / 8, H, fmt);
   h->gC = make_geom(H / 16, I, fmt);
   if (S) {
@@ -234,7 +232,6 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
   }
   h->ng_max_B = std::max(h->gB.ngroups, S ? h->gBs.ngroups : 0);
-  h->ng_max_C = std::max(h->gC.ngroups, S ? h->gCs.ngroups : 0);
   h->expert_bytes = 2ull * I * blob_row_bytes(fmt, H) + (uint64_t)H * blob_row_bytes(fmt, I);
   h->router_bytes = (uint64_t)E * blob_row_bytes(TS_FMT_Q8_0, H);
   h->shared_bytes = S ? 2ull * S * blob_row_bytes(TS_FMT_Q8_0, H) + (uint64_t)H * blob_row_bytes(TS_FMT_Q8_0, S) : 0;
@@ -246,8 +243,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
 
   // ---- arena
   size_t per_layer = 0;
-  per_layer += align256((size_t)E * H);            // rq
-  per_layer += align256((size_t)E * (H / 32) * 4); // rd
+  per_layer += align256(h->gR.bytes);             // router
   per_layer += align256((size_t)E * 4) * 2;        // bias, pes
   per_layer += align256((size_t)H * 4);            // xscale
   per_layer += align256(h->gB.bytes * E);
@@ -270,8 +266,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     };
     for (int l = 0; l < c.num_layers; ++l) {
       LayerDev& d = h->layers[l];
-      d.rq = (int8_t*)take((size_t)E * H);
-      d.rd = (float*)take((size_t)E * (H / 32) * 4);
+      d.rw = take(h->gR.bytes);
       d.bias = (float*)take((size_t)E * 4);
       d.pes = (float*)take((size_t)E * 4);
       d.xscale = (float*)take((size_t)H * 4);
@@ -305,7 +300,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
     const size_t o_partial = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = 1 + (size_t)(E + 1) * h->ng_max_B + (size_t)(E + 1) * h->ng_max_C + h->gC.ngroups + 1;
+    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + 2 + 1;
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -329,11 +324,9 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     unsigned* cn = (unsigned*)(h->ws + o_cnt);
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
-    h->cnt_route = cn;
-    h->cnt_gB = cn + 1;
-    h->cnt_gC = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
-    h->cnt_rg = h->cnt_gC + (size_t)(E + 1) * h->ng_max_C;
-    h->err = h->cnt_rg + h->gC.ngroups;
+    h->cnt_gB = cn;
+    h->grid = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
+    h->err = h->grid + 2;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
     if (ce != cudaSuccess) {
@@ -382,8 +375,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     // router + small vectors
     const uint8_t* r = src(w.router, router_b, 0);
     if (ce != cudaSuccess) break;
-    repack_router_kernel<<<std::max<int>(1, (int)std::min<long long>(((long long)E * (H / 32) + 255) / 256, 65535)),
-                           256, 0, st0>>>(r, E, H, d.rq, d.rd, d_bad);
+    launch_repack<1>(TS_FMT_Q8_0, r, nullptr, (int)blob_row_bytes(TS_FMT_Q8_0, H), H / 32, h->gR, d.rw, d_bad, st0, E);
     if (ce == cudaSuccess) ce = cudaDeviceSynchronize();  // the staging buffer is reused next
     if (w.router_bias && ce == cudaSuccess) ce = cudaMemcpy(d.bias, w.router_bias, E * 4, cudaMemcpyHostToDevice);
     if (ce == cudaSuccess)
@@ -392,6 +384,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
       for (int n = 0; n < H; ++n) {
         uint32_t u = (uint32_t)w.router_xscale[n] << 16;
         std::memcpy(&tmp[n], &u, 4);
+        if (tmp[n] != 1.0f) d.has_xscale = true;
       }
     } else {
       std::fill(tmp.begin(), tmp.begin() + H, 1.0f);
@@ -404,14 +397,14 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const int rbH = (int)blob_row_bytes(fmt, H), rbI = (int)blob_row_bytes(fmt, I);
     for (int e = 0; e < E; ++e)
       launch_repack<0>(fmt, gsrc + (size_t)e * I * rbH, usrc + (size_t)e * I * rbH, rbH, H / 32, h->gB,
-                       d.wB + (size_t)e * h->gB.bytes, d_bad, st0);
+                       d.wB + (size_t)e * h->gB.bytes, d_bad, st0, I);
     ce = cudaDeviceSynchronize();
     if (ce != cudaSuccess) break;
     const uint8_t* dsrc = src(w.down, down_bytes, 0);
     if (ce != cudaSuccess) break;
     for (int e = 0; e < E; ++e)
       launch_repack<1>(fmt, dsrc + (size_t)e * H * rbI, nullptr, rbI, I / 32, h->gC, d.wC + (size_t)e * h->gC.bytes,
-                       d_bad, st0);
+                       d_bad, st0, H);
     ce = cudaDeviceSynchronize();
     if (ce != cudaSuccess) break;
     if (S) {
@@ -419,12 +412,12 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
       const uint8_t* sg = src(w.sh_gate, shg, 0);
       const uint8_t* su = src(w.sh_up, shg, shg);
       if (ce != cudaSuccess) break;
-      launch_repack<0>(TS_FMT_Q8_0, sg, su, rbHq, H / 32, h->gBs, d.wBs, d_bad, st0);
+      launch_repack<0>(TS_FMT_Q8_0, sg, su, rbHq, H / 32, h->gBs, d.wBs, d_bad, st0, S);
       ce = cudaDeviceSynchronize();
       if (ce != cudaSuccess) break;
       const uint8_t* sd = src(w.sh_down, shd, 0);
       if (ce != cudaSuccess) break;
-      launch_repack<1>(TS_FMT_Q8_0, sd, nullptr, rbS, S / 32, h->gCs, d.wCs, d_bad, st0);
+      launch_repack<1>(TS_FMT_Q8_0, sd, nullptr, rbS, S / 32, h->gCs, d.wCs, d_bad, st0, H);
       ce = cudaDeviceSynchronize();
     }
   }
@@ -458,9 +451,9 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.Hp = h->Hp;
   rp.E = c.num_experts;
   rp.K = c.top_k;
-  rp.rq = d.rq;
-  rp.rd = d.rd;
-  rp.xscale = d.xscale;
+  rp.rw = d.rw;
+  rp.rg = h->gR;
+  rp.xscale = d.has_xscale ? d.xscale : nullptr;
   rp.bias = c.bias_mode != TS_BIAS_NONE ? d.bias : nullptr;
   rp.pes = d.pes;
   rp.bias_mode = c.bias_mode;
@@ -474,7 +467,6 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.meta = h->meta;
   rp.routes = h->routes;
   rp.rpos = h->rpos;
-  rp.cnt = h->cnt_route;
   rp.err = h->err;
   rp.idx_out = nullptr;
   rp.w_out = nullptr;
@@ -487,12 +479,12 @@ static ts_moe_status check_call(ts_moe* h, int layer, const void* x, int M) {
   if (layer < 0 || layer >= h->cfg.num_layers) return fail(h, TS_MOE_EINVAL, "layer out of range");
   if (M < 0 || M > h->cfg.max_tokens) return fail(h, TS_MOE_EINVAL, "M out of range [0, max_tokens]");
   if (M > 0 && !x) return fail(h, TS_MOE_EINVAL, "x is NULL");
+  if (((uintptr_t)x & 15) != 0) return fail(h, TS_MOE_EINVAL, "x must be 16-byte aligned");
   return TS_MOE_OK;
 }
 
 static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t st) {
-  const size_t smem = (size_t)(h->cfg.hidden + h->cfg.num_experts) * 4;
-  cudaError_t e = launch_pdl(route_kernel, rp.M, ROUTE_THREADS, smem, st, rp);
+  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, sizeof(RouteSmem), st, rp);
   if (e != cudaSuccess) return cuda_fail(h, e, "route_kernel launch");
   return TS_MOE_OK;
 }
@@ -543,7 +535,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   pp.P = h->P;
   pp.y = y;
   pp.resid = (__nv_bfloat16*)resid;
-  pp.cnt_rg = h->cnt_rg;
+  pp.grid_cnt = h->grid;
+  pp.grid_gen = h->grid + 1;
 
   // phase 1: gate/up + activation
   PhaseParams p1 = pp;
@@ -569,8 +562,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   p2.b_routed_ld = h->Ip;
   p2.b_shared = h->acts_sh;
   p2.b_shared_ld = h->Sp;
-  p2.cnt_group = h->cnt_gC;
-  p2.ng_max = h->ng_max_C;
+  p2.cnt_group = nullptr;
+  p2.ng_max = 0;
 
   const size_t smem = sizeof(PhaseSmem);
   cudaError_t e;

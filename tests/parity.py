@@ -6,7 +6,11 @@ Rules (the tolerances the routed-half spec states):
   there the GPU's set must still be a valid top-K within 1e-5 and the outputs
   are compared with the oracle's forced-routing result for the GPU's set;
 * routing weights within 1e-5 absolute (FP32 softmax vs FP64);
-* max |y_gpu - y_ref| <= 1e-2 * RMS(y_ref), and the same for resid + y.
+* max |y_gpu - y_ref| <= 1e-2 * RMS(y_ref) for the FP32 routed(+shared) sum;
+* the BF16 residual output: out_gpu is bit-exactly bf16_rn(resid + y_gpu) in
+  FP32 (the epilogue), and |out_gpu - out_ref| <= 1e-2 * RMS(out_ref) plus half
+  a BF16 ulp of out_ref (the output rounding itself, which alone exceeds
+  1e-2 * RMS wherever |out| >= 4).
 """
 from __future__ import annotations
 
@@ -91,10 +95,17 @@ def compare(shape, Lh: dict, x: torch.Tensor, resid_in: torch.Tensor, idx_gpu: n
     err_y = float(np.max(np.abs(yg - ref.y)))
     og = out_gpu[toks].astype(np.float64)
     rms_o = float(np.sqrt(np.mean(ref.out ** 2)))
+    # epilogue: out = bf16_rn(float(resid) + y) exactly
+    r32 = torch.from_numpy(rb[toks].view(np.int16)).view(torch.bfloat16).float()
+    want = (r32 + torch.from_numpy(y_gpu[toks].astype(np.float32))).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(want, out_gpu[toks].astype(np.float32)), "out != bf16(resid + y)"
+    _, ex = np.frexp(np.abs(ref.out))
+    half_ulp = np.ldexp(1.0, ex - 9)                  # bf16: 8 significant bits
+    slack = np.abs(og - ref.out) - half_ulp
     err_o = float(np.max(np.abs(og - ref.out)))
     rep = ParityReport(err_y, rms_y, err_o, rms_o, ties, idx_equal)
     assert err_y <= REL_TOL * rms_y, f"y: max err {err_y:.3e} > 1e-2 * RMS {rms_y:.3e}"
-    assert err_o <= REL_TOL * rms_o, f"out: max err {err_o:.3e} > 1e-2 * RMS {rms_o:.3e}"
+    assert float(np.max(slack)) <= REL_TOL * rms_o, f"out: max err beyond rounding {np.max(slack):.3e}"
     return rep
 
 

@@ -146,12 +146,13 @@ def test_split_groups_use_distinct_slots(B, chunks, ngroups, NB):
 
 def test_group_sizes_divide_or_cap():
     from quantized_moe_routed_router_b200 import binding as B
-    for tiles in (1, 8, 15, 16, 17, 32, 88, 176, 180, 352, 360, 1792, 97):
+    for tiles in (1, 8, 15, 16, 17, 32, 33, 88, 176, 180, 352, 360, 1792, 97):
         gs = B.lib.ts_moe_debug_group_size(tiles)
-        assert 1 <= gs <= 16
-        if tiles <= 16:
+        assert 1 <= gs <= 30
+        if tiles <= 30:
             assert gs == tiles
-        elif any(tiles % g == 0 for g in range(8, 17)):
-            assert tiles % gs == 0 and gs >= 8
+        elif any(tiles % g == 0 for g in range(15, 31)):
+            assert tiles % gs == 0 and gs >= 15
+            assert not any(tiles % g == 0 for g in range(gs + 1, 31))
         else:
-            assert gs == 16
+            assert gs == 30
