@@ -152,6 +152,38 @@ ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
  * them, so a timed run without hooks is the throughput number. */
 ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4);
 
+/* Router GEMV + top-k for callers that cannot allocate device memory -- no
+ * counterpart in the paper; this is a library convenience.  Some callers
+ * cannot call cudaMalloc at the point where they need routing: code that
+ * runs while a stream is being captured into a CUDA graph (allocation is not
+ * capturable), engines that hand all device memory to their own pool and
+ * forbid other allocations, or plugins that are given only a stream and
+ * buffers.  They cannot use ts_moe_open (which allocates the weight arena
+ * and workspace), so this entry point takes the raw router itself and keeps
+ * all of its scratch in one file-scope device array of
+ * TS_MOE_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
+ * until the process exits.  It performs no allocation of any kind.
+ *
+ * router: device [E][H] Q8_0 blocks (as in ts_moe_layer_weights.router);
+ * router_bias, per_expert_scale: DEVICE [E] float32 or NULL (bias required
+ * iff bias_mode != TS_BIAS_NONE); the router x-scale is taken as ones.
+ * x: device [M][H] BF16, 16-byte aligned; idx: device [M][K] int32; w: device
+ * [M][K] float32; logits: device [M][E] float32 or NULL.  Same semantics and
+ * results as ts_moe_route on a handle opened with this router.
+ * Limits: 1 <= E <= 256, 1 <= K <= min(8, E), H a positive multiple of 32,
+ * 0 <= M <= 16, and the scratch (repacked router + staged x + route state)
+ * must fit in TS_MOE_NOALLOC_SCRATCH_BYTES, else TS_MOE_EINVAL with the
+ * required size in ts_moe_last_error(NULL).
+ * The first call on a device looks up the scratch array's device address and
+ * sets a kernel attribute; make that first call before any stream capture.
+ * Every call shares the one array and leaves its contents behind: calls that
+ * overlap on the GPU (different streams, or graphs replayed concurrently)
+ * race and must be serialised by the caller.  Asynchronous on `stream`. */
+#define TS_MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
+ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias, const float* per_expert_scale,
+                                   int num_experts, int hidden, int top_k, int score, int bias_mode, const void* x,
+                                   int M, int32_t* idx, float* w, float* logits, void* stream);
+
 /* Reason for the last failure on this handle; with h == NULL, the last
  * failure of ts_moe_open on the calling thread.  Never NULL. */
 const char* ts_moe_last_error(const ts_moe* h);

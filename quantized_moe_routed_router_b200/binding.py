@@ -68,8 +68,9 @@ def _load():
     lib.ts_moe_debug_partial_slot.argtypes = [C.c_uint64, i32, i32, C.c_uint64]
     lib.ts_moe_debug_group_size.argtypes = [i32]
     lib.ts_moe_debug_validate.argtypes = [C.POINTER(Config), C.POINTER(LayerWeights)]
+    lib.ts_moe_route_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
     for f in ("ts_moe_open", "ts_moe_route", "ts_moe_forward", "ts_moe_device_status", "ts_moe_get_info",
-              "ts_moe_set_timing_events", "ts_moe_close", "ts_moe_debug_validate"):
+              "ts_moe_set_timing_events", "ts_moe_close", "ts_moe_debug_validate", "ts_moe_route_noalloc"):
         getattr(lib, f).restype = C.c_int
     return lib
 
@@ -183,6 +184,19 @@ class MoE:
             self.close()
         except Exception:
             pass
+
+
+def route_noalloc(router: torch.Tensor, bias: Optional[torch.Tensor], pes: Optional[torch.Tensor], num_experts: int,
+                  hidden: int, top_k: int, score: int, bias_mode: int, x: torch.Tensor, idx: torch.Tensor,
+                  w: torch.Tensor, logits: Optional[torch.Tensor] = None, stream=None):
+    """Router GEMV + top-k without a handle and without any device allocation
+    (scratch lives in the library's static device array).  router: device Q8_0
+    blob [E][H]; bias / pes: device float32 [E] or None; x: device bf16 [M][H]."""
+    M = x.shape[0]
+    st = lib.ts_moe_route_noalloc(_ptr(router), _ptr(bias), _ptr(pes), num_experts, hidden, top_k, score, bias_mode,
+                                  _ptr(x), M, _ptr(idx), _ptr(w), _ptr(logits), _stream(stream))
+    if st != 0:
+        raise TsMoeError(st, lib.ts_moe_last_error(None).decode())
 
 
 def validate(shape: "synth.MoEShape", layers: Sequence["synth.LayerBlobs"], **cfg_over) -> tuple:

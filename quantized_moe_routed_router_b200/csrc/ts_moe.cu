@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -634,6 +635,115 @@ ts_moe_status ts_moe_close(ts_moe* h) {
   if (h->arena) cudaFree(h->arena);
   if (h->ws) cudaFree(h->ws);
   delete h;
+  return TS_MOE_OK;
+}
+
+// ----------------------------------------------------------------------------- routing without allocation
+// Scratch for ts_moe_route_noalloc: a file-scope device array.  Host code must
+// not use the symbol itself as a device pointer (on the host it names a
+// host-side stand-in); the device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[TS_MOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+
+// Once per device, with that device current: the array's device address and
+// the route kernel's shared-memory attribute.
+ts_moe_status noalloc_setup(int dev, uint8_t** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RouteSmem));
+    if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = (uint8_t*)ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TS_MOE_OK;
+}
+}  // namespace
+
+ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias, const float* per_expert_scale, int E,
+                                   int H, int K, int score, int bias_mode, const void* x, int M, int32_t* idx,
+                                   float* w, float* logits, void* stream) {
+  if (E < 1 || E > TS_MOE_MAX_EXPERTS) return fail(nullptr, TS_MOE_EINVAL, "num_experts must be in [1, 256]");
+  if (K < 1 || K > TS_MOE_MAX_TOPK || K > E) return fail(nullptr, TS_MOE_EINVAL, "top_k must be in [1, min(8, E)]");
+  if (H <= 0 || H % 32 || H > 16384) return fail(nullptr, TS_MOE_EINVAL, "hidden must be a positive multiple of 32, <= 16384");
+  if (M < 0 || M > TS_MOE_MAX_TOKENS) return fail(nullptr, TS_MOE_EINVAL, "M must be in [0, 16]");
+  if (score != TS_SCORE_SOFTMAX_SELECTED && score != TS_SCORE_SOFTMAX_ALL_NORENORM) return fail(nullptr, TS_MOE_EINVAL, "unknown score");
+  if (bias_mode < TS_BIAS_NONE || bias_mode > TS_BIAS_SELECT_ONLY) return fail(nullptr, TS_MOE_EINVAL, "unknown bias_mode");
+  if ((bias_mode != TS_BIAS_NONE) != (router_bias != nullptr))
+    return fail(nullptr, TS_MOE_EINVAL, "router_bias must be given iff bias_mode != NONE");
+  if (M == 0) return TS_MOE_OK;
+  if (!router || !x || !idx || !w) return fail(nullptr, TS_MOE_EINVAL, "router, x, idx and w must be non-NULL");
+  if (((uintptr_t)x & 15) != 0) return fail(nullptr, TS_MOE_EINVAL, "x must be 16-byte aligned");
+
+  // scratch layout: repacked router | xh | logits | idx | w | shift | meta | routes | rpos | error word
+  const MatGeom gR = make_geom((E + 15) / 16, H, TS_FMT_Q8_0);
+  const int Hp = round_up(H, 64);
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t r = off;
+    off += align256(n);
+    return r;
+  };
+  const size_t o_rw = take(gR.bytes), o_xh = take((size_t)M * Hp * 2), o_lg = take((size_t)M * E * 4),
+               o_idx = take((size_t)M * K * 4), o_w = take((size_t)M * K * 4), o_sh = take((size_t)M * 4),
+               o_meta = take((size_t)META_INTS * 4), o_rt = take((size_t)M * K * sizeof(Route)),
+               o_rpos = take((size_t)M * K * 4), o_err = take(8);
+  if (off > TS_MOE_NOALLOC_SCRATCH_BYTES)
+    return fail(nullptr, TS_MOE_EINVAL, "routing needs " + std::to_string(off) + " bytes of scratch, more than the " +
+                                            std::to_string(TS_MOE_NOALLOC_SCRATCH_BYTES) + " this entry point has");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return fail(nullptr, TS_MOE_EUNSUPPORTED, "device ordinal >= 64");
+  uint8_t* sc = nullptr;
+  ts_moe_status st = noalloc_setup(dev, &sc);
+  if (st != TS_MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+
+  unsigned* errw = (unsigned*)(sc + o_err);  // the error and repack words must start at zero
+  e = cudaMemsetAsync(errw, 0, 8, s);
+  if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaMemsetAsync: ") + cudaGetErrorString(e));
+  launch_repack<1>(TS_FMT_Q8_0, (const uint8_t*)router, nullptr, (int)blob_row_bytes(TS_FMT_Q8_0, H), H / 32, gR,
+                   sc + o_rw, errw + 1, s, E);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("router repack launch: ") + cudaGetErrorString(e));
+
+  RouteParams rp;
+  std::memset(&rp, 0, sizeof(rp));
+  rp.x = (const __nv_bfloat16*)x;
+  rp.M = M;
+  rp.H = H;
+  rp.Hp = Hp;
+  rp.E = E;
+  rp.K = K;
+  rp.rw = sc + o_rw;
+  rp.rg = gR;
+  rp.xscale = nullptr;
+  rp.bias = bias_mode != TS_BIAS_NONE ? router_bias : nullptr;
+  rp.pes = per_expert_scale;
+  rp.bias_mode = bias_mode;
+  rp.score = score;
+  rp.has_shared = 0;
+  rp.logits = (float*)(sc + o_lg);
+  rp.idx = (int*)(sc + o_idx);
+  rp.w = (float*)(sc + o_w);
+  rp.shift = (int*)(sc + o_sh);
+  rp.xh = (__half*)(sc + o_xh);
+  rp.meta = (int*)(sc + o_meta);
+  rp.routes = (Route*)(sc + o_rt);
+  rp.rpos = (int*)(sc + o_rpos);
+  rp.err = errw;
+  rp.idx_out = idx;
+  rp.w_out = w;
+  rp.logits_out = logits;
+  e = launch_pdl(route_kernel, 1, ROUTE_THREADS, sizeof(RouteSmem), s, rp);
+  if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("route_kernel launch: ") + cudaGetErrorString(e));
   return TS_MOE_OK;
 }
 
