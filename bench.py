@@ -199,10 +199,7 @@ def run_ours(args, rank, world, local):
                 n = len(set(idx.cpu().numpy().ravel().tolist()))
                 n_touched.append(n)
         per_layer = [n * info.expert_bytes + info.router_bytes + info.shared_bytes for n in n_touched]
-        gu_expert = 2 * shape.moe_inter * synth.row_bytes(shape.expert_fmt, H)
-        gu_shared = 2 * shape.shared_inter * synth.row_bytes(synth.FMT_Q8_0, H) if shape.shared_inter else 0
-        gate_up = [n * gu_expert + gu_shared for n in n_touched]
-        return sum(per_layer), n_touched, gate_up
+        return sum(per_layer), n_touched, per_layer
 
     def make_graph(Mx, out):
         g = torch.cuda.CUDAGraph()
@@ -237,14 +234,14 @@ def run_ours(args, rank, world, local):
 
     out = rs.clone()
     g = make_graph(M, out)
-    algo_bytes, n_touched, gate_up_bytes = touched_bytes(M)
+    algo_bytes, n_touched, layer_bytes = touched_bytes(M)
     sampler = ClockSampler(local)
     ms_step, clocks = time_graph(g, args.steps, args.warmup, sampler)
     moe.device_status(stream)
     tok_s = world * M / (ms_step * 1e-3)
     gbs = algo_bytes / (ms_step * 1e-3) / 1e9
 
-    # dominant kernel (gate/up): CUDA events on the launching stream around each launch
+    # the layer kernel (the only kernel of a forward): CUDA events on the launching stream around each launch
     prof_steps = max(3, min(20, args.steps // 10))
     ev_all = []
     with torch.cuda.stream(stream):
@@ -260,19 +257,15 @@ def run_ours(args, rank, world, local):
                 ev_all.append((l, evs))
         moe.set_timing_events(None)
         stream.synchronize()
-    t_gu = [e[0].elapsed_time(e[1]) for _, e in ev_all]
-    t_dn = [e[2].elapsed_time(e[3]) for _, e in ev_all]
-    gu_bytes_per_launch = statistics.mean(gate_up_bytes[l] for l, _ in ev_all)
-    avg_gu_ms = statistics.mean(t_gu)
-    avg_dn_ms = statistics.mean(t_dn)
+    t_layer = [e[0].elapsed_time(e[1]) for _, e in ev_all]
+    bytes_per_launch = statistics.mean(layer_bytes[l] for l, _ in ev_all)
+    avg_ms = statistics.mean(t_layer)
     peak, peak_kind = measured_peaks()
-    achieved = gu_bytes_per_launch / (avg_gu_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "expert_kernel<MXFP4, gate/up>" if shape.expert_fmt else
-                "expert_kernel<Q8_0, gate/up>", "achieved": round(achieved, 1), "peak": peak,
-                "peak_kind": f"{peak_kind} HBM copy bandwidth", "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "traffic": None, "avg_launch_us": round(avg_gu_ms * 1e3, 2),
-                "algorithmic_bytes_per_launch": int(gu_bytes_per_launch),
-                "down_kernel_avg_launch_us": round(avg_dn_ms * 1e3, 2)}
+    achieved = bytes_per_launch / (avg_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": f"layer_kernel<{'MXFP4' if shape.expert_fmt else 'Q8_0'}> (route + gate/up + down + combine)",
+                "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "avg_launch_us": round(avg_ms * 1e3, 2), "algorithmic_bytes_per_launch": int(bytes_per_launch)}
 
     # end to end through host buffers: pinned H2D of x and resid, D2H of the updated resid
     x_h = xs[:, :M].cpu().pin_memory()
@@ -342,7 +335,7 @@ def run_ours(args, rank, world, local):
             "roofline": roofline,
             "e2e": {"value": round(world * M / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-            "gpu_launches": args.steps * NL * 3,
+            "gpu_launches": args.steps * NL,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

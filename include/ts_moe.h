@@ -145,11 +145,11 @@ typedef struct {
 } ts_moe_info;
 ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
 
-/* Optional per-phase timing hooks for profiling: when set, ts_moe_forward
- * records events[0] before the gate/up kernel and events[1] after it, and
- * events[2] / events[3] around the down+combine kernel, on the call's stream
- * (cudaEvent_t values; NULL clears).  Events between the kernels serialise
- * them, so a timed run without hooks is the throughput number. */
+/* Optional timing hooks for profiling: when set, ts_moe_forward records
+ * events[0] before and events[1] after its layer kernel on the call's stream
+ * (cudaEvent_t values; events[2] and events[3] must be valid events and are
+ * reserved; NULL clears).  An event between two forwards separates their
+ * kernels, so a timed run without hooks is the throughput number. */
 ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4);
 
 /* Router GEMV + top-k for callers that cannot allocate device memory -- no

@@ -20,6 +20,7 @@ enum : unsigned {
   ERR_BAD_INDEX = 1u << 4,       // an expert / token index read from the route list was out of range
   ERR_BAD_META = 1u << 5,        // route metadata inconsistent with the launch
   ERR_TIMEOUT_GRID = 1u << 6,    // a CTA gave up waiting at the grid-wide barrier
+  ERR_TIMEOUT_ACTS = 1u << 7,    // a down producer gave up waiting for an expert's acts
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -107,6 +108,10 @@ TSM_DEV void bulk_g2s_hint(void* dst, const void* src, unsigned bytes, uint64_t*
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy) writes to the same bytes.
 TSM_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Orders generic-proxy global memory accesses (made visible to this thread)
+// before later async-proxy (bulk copy) reads of the same global memory.
+TSM_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------- PDL
 TSM_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -1,30 +1,34 @@
-// Grouped expert kernels: phase 1 = gate/up GEMV + activation, phase 2 =
-// down GEMV + weighted combine + shared expert + residual add.
+// The routed MoE half of one layer as ONE persistent kernel per layer
+// (one CTA per SM, all resident):
 //
-// Both phases are the same persistent, stream-K kernel over the route list
-// the route kernel built (gpt-oss state page, `BatchedRoutedScratch`: phase 1
-// writes `batch_acts [M*top_k, moe_inter]` from the route list, the fused
-// phase 2 writes the per-token sum that the residual add reads; deepseek2
-// state page: phase 2 is seeded with the shared expert, "y = shared +
-// sum(w * expert)").
+//   1. route   -- every CTA computes the routing itself (router GEMV on the
+//                 tensor cores, top-k, route list; see route.cuh), so no CTA
+//                 waits for another and no separate launch sits in front;
+//   2. gate/up -- grouped GEMV of the touched experts (+ shared expert) and
+//                 the activation, written as FP16 acts (gpt-oss state page,
+//                 `BatchedRoutedScratch`: phase 1 fills `batch_acts` from the
+//                 route list);
+//   3. down    -- grouped GEMV of the acts; a CTA whose down work needs an
+//                 expert's acts waits (bounded) until every gate/up group of
+//                 that expert is done, prefetching its weights meanwhile;
+//   4. combine -- after a bounded grid-wide barrier each CTA forms 1/NB of
+//                 y[t] = sum_k w[t][k] down_k[t] (+ shared, deepseek2 state
+//                 page: "y = shared + sum(w * expert)") and resid += y.
 //
-// Work: every touched expert (plus the shared expert as one more entry with
-// all M tokens) contributes (group, chunk) units -- a group is up to 30
-// tiles of 16 MMA rows, a chunk 64 (MXFP4) or 32 (Q8_0) elements of K.  The
-// units of the launch are cut into one equal contiguous range per CTA (one
-// CTA per SM), so every SM streams the same number of weight bytes whatever
-// the routing.  A group split between CTAs is finished by the last CTA to
-// add its chunk count to the group's counter: partial sums go to per-CTA
-// slots and are added back in CTA order, so results do not depend on timing.
+// Work split: the (entry, group, chunk) units of each GEMV phase are cut into
+// one equal contiguous range per CTA (stream-K), so every SM streams the same
+// number of weight bytes whatever the routing.  A group split between CTAs is
+// finished from per-CTA partial slots added in CTA order: results do not
+// depend on timing.
 //
 // Per CTA: one producer warp issues 1-D bulk copies (TMA, no multicast) of
-// weight stages (contiguous runs of a group's chunks) into a 4-deep ring,
-// and of activation windows (512 K-elements of each column's FP16 row) into a
+// weight stages (contiguous runs of a group's chunks) into a 4-deep ring, and
+// of activation windows (512 K-elements of each column's FP16 row) into a
 // 2-deep ring, each completing on an mbarrier.  Fifteen consumer warps own two
 // tiles each; per chunk they convert their A fragments in registers (MXFP4:
 // cvt e2m1x2 -> f16x2; Q8_0: byte permute into 1024+u and subtract), run
-// m16n8k16 tensor-core MMAs against the activation columns (tokens or
-// routes, padded to 8 or 16) and fold each 32-block's partial sum into FP32
+// m16n8k16 tensor-core MMAs against the activation columns (tokens or routes,
+// padded to 8 or 16) and fold each 32-block's partial sum into FP32
 // accumulators with the block scale.  Every wait is bounded.
 #pragma once
 #include "common.cuh"
@@ -44,55 +48,52 @@ constexpr int XROW = KW * 2 + 32;          // bytes per window row; 1056 = 32 mo
 constexpr int WSTAGE = GS_MAX * KS * UNIT_BYTES;
 constexpr int XWIN = 16 * XROW;
 constexpr int SLOT_FLOATS = GS_MAX * 16 * 16;
-constexpr int MAX_NB = 1024;               // CTAs per launch (one per SM)
+constexpr int MAX_NB = 512;                // CTAs per launch (one per SM)
 static_assert(GS_MAX == NWC * RW, "a group is one tile per consumer-warp slot");
+static_assert(ROUTE_WARPS <= NWC + 1, "routing uses the first ROUTE_WARPS warps");
 
-struct PhaseParams {
-  const uint8_t* w_routed;  // expert e's matrix at w_routed + e * w_stride
-  uint64_t w_stride;
-  const uint8_t* w_shared;  // shared expert matrix or null
-  MatGeom gr, gsh;          // routed / shared geometry
-  const __half* b_routed;   // B rows: phase 1 x (FP16, scaled) [M][ld]; phase 2 acts [M*K][ld]
-  int b_routed_ld;
-  const __half* b_shared;   // phase 1: x; phase 2: shared acts [M][ld]
-  int b_shared_ld;
-  const int* meta;
-  const Route* routes;
-  const int* shift;         // [M] x scale exponents (phase 1)
-  __half* acts;             // phase 1 out: [M*K][acts_ld]
-  int acts_ld;
-  __half* acts_sh;          // phase 1 out: shared [M][acts_sh_ld]
-  int acts_sh_ld;
-  float* P;                 // phase 2: per-route down outputs [M*K + M][H]
-  const float* wts;         // [M][K] routing weights
-  const int* rpos;          // [M][K] route positions
+struct LayerParams {
+  RouteParams rp;           // routing inputs; its output pointers are written by CTA 0 only
+  __half* xh_cta;           // [NB][Mmax*Hp] per-CTA FP16 x (gate/up B operand)
+  __half* rin_cta;          // [NB][2*Mmax*Hp] per-CTA router input hi/lo (x-scale only) or null
+  int xh_stride, rin_stride;
+  const uint8_t* wB;        // gate/up: expert e at wB + e * wB_stride
+  uint64_t wB_stride;
+  const uint8_t* wBs;       // shared gate/up or null
+  const uint8_t* wC;        // down
+  uint64_t wC_stride;
+  const uint8_t* wCs;       // shared down or null
+  MatGeom gB, gBs, gC, gCs;
+  __half* acts;             // [M*K][Ip]
+  __half* acts_sh;          // [M][Sp]
+  int Ip, Sp;
+  float* P;                 // [M*K + M][H] down outputs of whole segments
+  float* partial0;          // [NB][2][SLOT_FLOATS] gate/up partial slots
+  float* partial1;          // [NB][2][SLOT_FLOATS] down partial slots
+  unsigned* cnt_group;      // [(E+1) * ng_max] gate/up chunk counters
+  int ng_max;
+  unsigned* entry_done;     // [E+1] gate/up groups finished per expert (+ shared)
+  unsigned* grid_cnt;       // grid barrier arrivals
+  unsigned* grid_gen;       // grid barrier generation
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
-  float* partial;           // [NB][2][SLOT_FLOATS]
-  unsigned* cnt_group;      // [(E+1) * ng_max]
-  int ng_max;
-  unsigned* grid_cnt;       // phase 2: grid barrier arrivals
-  unsigned* grid_gen;       // phase 2: grid barrier generation
   unsigned* err;
-  int H, K, E;
   int act;
   float alpha, limit;
 };
 
-struct __align__(128) PhaseSmem {
+struct __align__(128) LayerSmem {
   uint8_t w[NSW][WSTAGE];
   uint8_t x[NSX][XWIN];
   uint64_t wfull[NSW], wempty[NSW], xfull[NSX], xempty[NSX];
-  long long upre[MAX_ENTRIES + 1];  // entry-major: first unit of each entry
-  int cpre[MAX_ENTRIES + 1];        // group-major: first unit of each entry inside a group
-  int ex[MAX_ENTRIES], ro[MAX_ENTRIES], nc[MAX_ENTRIES];
-  int tok[MAX_TOK * MAX_K];
-  int rj[MAX_TOK * MAX_K];          // entry index of each route position
-  unsigned rs[MAX_NB + 1];          // first unit of each CTA's range
-  unsigned gen0;                    // grid barrier generation seen at kernel start
-  int nE, nT, M, MK, has_shared;
+  RouteState r;
+  long long upre0[MAX_ENTRIES + 1];  // gate/up: first unit of each entry (entry-major)
+  int cpre1[MAX_ENTRIES + 1];        // down: first unit of each entry inside a group (group-major)
+  unsigned rs0[MAX_NB + 1];          // first unit of each CTA's range, per phase
+  unsigned rs1[MAX_NB + 1];
   int dead;
   int flag;
+  unsigned gen0;
 };
 
 struct Seg {
@@ -101,36 +102,38 @@ struct Seg {
   int grp, c0, c1;
   int chunks, tiles, gs, ntg;
   int nc, ro;
-  long long g0;   // unit index of the group's first chunk
+  long long g0;   // unit index of the (entry, group)'s first chunk
 };
 
-// Next segment (one entry's group, a run of its chunks) of [u, u1).
-// GM = group-major order (the down phase: every entry has the same groups).
-template <bool GM>
-TSM_DEV bool next_seg(const PhaseSmem& s, const PhaseParams& p, long long& u, long long u1, int& j, Seg& sg) {
+// Next segment (one entry's group, a run of its chunks) of [u, u1) of phase PH
+// (0: entry-major gate/up units, 1: group-major down units).
+template <int PH>
+TSM_DEV bool next_seg(const LayerSmem& s, const LayerParams& p, long long& u, long long u1, int& j, Seg& sg) {
   if (u >= u1) return false;
+  const MatGeom& gr = PH == 0 ? p.gB : p.gC;
+  const MatGeom& gsh = PH == 0 ? p.gBs : p.gCs;
   int grp, c0;
   long long base;
-  if (GM) {
-    const int upg = s.cpre[s.nE];
+  if (PH == 1) {
+    const int upg = s.cpre1[s.r.nE];
     grp = (int)(u / upg);
     const int r = (int)(u - (long long)grp * upg);
     j = 0;
-    while (r >= s.cpre[j + 1]) ++j;
-    c0 = r - s.cpre[j];
-    base = (long long)grp * upg + s.cpre[j];
+    while (r >= s.cpre1[j + 1]) ++j;
+    c0 = r - s.cpre1[j];
+    base = (long long)grp * upg + s.cpre1[j];
   } else {
-    while (u >= s.upre[j + 1]) ++j;
-    const bool sh = s.has_shared && j == s.nT;
-    const int chunks = sh ? p.gsh.chunks : p.gr.chunks;
-    const long long local = u - s.upre[j];
+    while (u >= s.upre0[j + 1]) ++j;
+    const bool sh = p.rp.has_shared && j == s.r.nT;
+    const int chunks = sh ? gsh.chunks : gr.chunks;
+    const long long local = u - s.upre0[j];
     grp = (int)(local / chunks);
     c0 = (int)(local - (long long)grp * chunks);
-    base = s.upre[j] + (long long)grp * chunks;
+    base = s.upre0[j] + (long long)grp * chunks;
   }
   sg.j = j;
-  sg.sh = s.has_shared && j == s.nT;
-  const MatGeom& g = sg.sh ? p.gsh : p.gr;
+  sg.sh = p.rp.has_shared && j == s.r.nT;
+  const MatGeom& g = sg.sh ? gsh : gr;
   sg.chunks = g.chunks;
   sg.tiles = g.tiles;
   sg.gs = g.gs;
@@ -139,19 +142,19 @@ TSM_DEV bool next_seg(const PhaseSmem& s, const PhaseParams& p, long long& u, lo
   const long long rem = u1 - u;
   sg.c1 = (int)((long long)c0 + rem < g.chunks ? c0 + rem : g.chunks);
   sg.ntg = group_tiles(g.tiles, g.gs, grp);
-  sg.nc = s.nc[j];
-  sg.ro = s.ro[j];
+  sg.nc = s.r.nc[j];
+  sg.ro = s.r.ro[j];
   sg.g0 = base;
   u += sg.c1 - sg.c0;
   return true;
 }
 
 // The CTA whose range holds unit u: the largest b with rs[b] <= u.
-TSM_DEV int owner_tab(const PhaseSmem& s, int NB, unsigned u) {
+TSM_DEV int owner_tab(const unsigned* rs, int NB, unsigned u) {
   int lo = 0, hi = NB - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.rs[mid] <= u)
+    if (rs[mid] <= u)
       lo = mid;
     else
       hi = mid - 1;
@@ -233,43 +236,72 @@ TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, i
   }
 }
 
+// First / last CTA that worked on the down segment (entry j, row group grp),
+// packed as bf | bl << 16.
+TSM_DEV unsigned down_owners(const LayerSmem& s, const LayerParams& p, int NB, int grp, int j) {
+  const bool sh = p.rp.has_shared && j == s.r.nT;
+  const unsigned C = (unsigned)(sh ? p.gCs.chunks : p.gC.chunks);
+  const unsigned g0 = (unsigned)grp * (unsigned)s.cpre1[s.r.nE] + (unsigned)s.cpre1[j];
+  return (unsigned)owner_tab(s.rs1, NB, g0) | ((unsigned)owner_tab(s.rs1, NB, g0 + C - 1) << 16);
+}
+
 // Value of the down output of entry j, column n, row h (row group `grp`):
 // written to P when one CTA covered the whole (group, entry) segment, else
 // the sum of the contributing CTAs' partial slots in CTA order.
-TSM_DEV float down_value(const PhaseSmem& s, const PhaseParams& p, int NB, int grp, int gs, int j, int n, int h,
-                         int route) {
-  const bool sh = s.has_shared && j == s.nT;
-  const unsigned C = (unsigned)(sh ? p.gsh.chunks : p.gr.chunks);
-  const unsigned g0 = (unsigned)grp * (unsigned)s.cpre[s.nE] + (unsigned)s.cpre[j];
-  const int bf = owner_tab(s, NB, g0), bl = owner_tab(s, NB, g0 + C - 1);
-  if (bf == bl) return ld_cg(p.P + (size_t)route * p.H + h);
+TSM_DEV float down_value(const LayerSmem& s, const LayerParams& p, unsigned owners, int grp, int gs, int j, int n,
+                         int h, int route) {
+  const int bf = owners & 0xFFFF, bl = owners >> 16;
+  if (bf == bl) return ld_cg(p.P + (size_t)route * p.rp.H + h);
+  const unsigned g0 = (unsigned)grp * (unsigned)s.cpre1[s.r.nE] + (unsigned)s.cpre1[j];
   const int rel = h - grp * gs * 16;
   const int off = ((rel >> 4) * 16 + (rel & 15)) * 16 + n;
   float v = 0.f;
   for (int b2 = bf; b2 <= bl; ++b2) {
-    if (s.rs[b2] == s.rs[b2 + 1]) continue;  // empty range
-    const int slot = s.rs[b2] >= g0 ? 0 : 1;
-    v += ld_cg(p.partial + ((size_t)b2 * 2 + slot) * SLOT_FLOATS + off);
+    if (s.rs1[b2] == s.rs1[b2 + 1]) continue;  // empty range
+    const int slot = s.rs1[b2] >= g0 ? 0 : 1;
+    v += ld_cg(p.partial1 + ((size_t)b2 * 2 + slot) * SLOT_FLOATS + off);
   }
   return v;
 }
 
-// Phase 2 finish, after the grid barrier: this CTA's 1/NB slice of the M x H
-// outputs, y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared) in slot order;
-// resid += y (BF16).
-TSM_DEV void final_combine(const PhaseSmem& s, const PhaseParams& p, int NB, int ctid) {
-  const int M = s.M, K = p.K, H = p.H, gs = p.gr.gs;
+// After the grid barrier: this CTA's 1/NB slice of the M x H outputs,
+// y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared) in slot order; resid += y.
+// The (row group, entry) -> contributing CTAs table goes in the routing
+// scratch (free by now) when it fits.
+TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid) {
+  const int M = p.rp.M, K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = M * K, nE = s.r.nE;
+  unsigned* tab = reinterpret_cast<unsigned*>(&s.r.part[0][0][0]);
+  constexpr int TAB_CAP = (int)(sizeof(s.r.part) / sizeof(unsigned));
+  const bool use_tab = p.gC.ngroups * nE <= TAB_CAP;
+  if (use_tab)
+    for (int i = ctid; i < p.gC.ngroups * nE; i += NWC * 32) tab[i] = down_owners(s, p, NB, i / nE, i % nE);
+  bar_sync(1, NWC * 32);
   const long long MH = (long long)M * H;
   const int lo = (int)(MH * blockIdx.x / NB), hi = (int)(MH * (blockIdx.x + 1) / NB);
   for (int i = lo + ctid; i < hi; i += NWC * 32) {
     const int t = i / H, h = i - t * H, grp = h / (gs * 16);
-    float y = 0.f;
-    for (int k = 0; k < K; ++k) {
-      const int pos = p.rpos[t * K + k];
-      const int j = s.rj[pos];
-      y = fmaf(p.wts[t * K + k], down_value(s, p, NB, grp, gs, j, pos - s.ro[j], h, pos), y);
+    float v[MAX_K + 1];
+#pragma unroll
+    for (int k = 0; k < MAX_K; ++k) {
+      v[k] = 0.f;
+      if (k < K) {
+        const int pos = s.r.rpos[t * K + k];
+        const int j = s.r.rj[pos];
+        const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
+        v[k] = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
+      }
     }
-    if (s.has_shared) y += down_value(s, p, NB, grp, gs, s.nT, t, h, s.MK + t);
+    v[MAX_K] = 0.f;
+    if (p.rp.has_shared) {
+      const int j = s.r.nT;
+      const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
+      v[MAX_K] = down_value(s, p, own, grp, gs, j, t, h, MK + t);
+    }
+    float y = 0.f;
+#pragma unroll
+    for (int k = 0; k < MAX_K; ++k)
+      if (k < K) y = fmaf(s.r.w[t * K + k], v[k], y);
+    y += v[MAX_K];
     if (p.y) p.y[(size_t)t * H + h] = y;
     if (p.resid) {
       __nv_bfloat16* r = p.resid + (size_t)t * H + h;
@@ -281,7 +313,7 @@ TSM_DEV void final_combine(const PhaseSmem& s, const PhaseParams& p, int NB, int
 // Grid-wide barrier among the consumer warps of all CTAs (one CTA per SM, all
 // resident).  Bounded: a CTA that waits longer than WAIT_LIMIT_NS records
 // ERR_TIMEOUT_GRID and goes on.
-TSM_DEV void grid_barrier(const PhaseSmem& s, const PhaseParams& p, int NB, int ctid) {
+TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
   __threadfence();
   bar_sync(1, NWC * 32);
   if (ctid == 0) {
@@ -303,12 +335,19 @@ TSM_DEV void grid_barrier(const PhaseSmem& s, const PhaseParams& p, int NB, int 
   __threadfence();
 }
 
+// A finished gate/up group: every consumer's acts are written; count it for its entry.
+TSM_DEV void entry_group_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int ctid) {
+  __threadfence();
+  bar_sync(1, NWC * 32);
+  if (ctid == 0) atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
+}
+
 // Group epilogue with complete sums in acc.
-template <int PHASE, int NT>
-TSM_DEV void group_epilogue(PhaseSmem& s, const PhaseParams& p, const Seg& sg, float (&acc)[RW][NT][4], int warp,
-                            int lane, int ctid) {
+template <int PH, int NT>
+TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg& sg, float (&acc)[RW][NT][4],
+                            int warp, int lane, int ctid) {
   const int g = lane >> 2, c = lane & 3;
-  if constexpr (PHASE == 0) {
+  if constexpr (PH == 0) {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       const int jt = warp * RW + r;
@@ -320,14 +359,15 @@ TSM_DEV void group_epilogue(PhaseSmem& s, const PhaseParams& p, const Seg& sg, f
         for (int h = 0; h < 2; ++h) {
           const int n = nt * 8 + 2 * c + h;
           if (n < sg.nc) {
-            const int tk = sg.sh ? n : s.tok[sg.ro + n];
-            const float scl = __uint_as_float((uint32_t)(127 - p.shift[tk]) << 23);
+            const int tk = sg.sh ? n : s.r.tok[sg.ro + n];
+            const float scl = __uint_as_float((uint32_t)(127 - s.r.shift[tk]) << 23);
             const float a = act_fn(p.act, p.alpha, p.limit, acc[r][nt][h] * scl, acc[r][nt][2 + h] * scl);
-            __half* dst = sg.sh ? p.acts_sh + (size_t)n * p.acts_sh_ld : p.acts + (size_t)(sg.ro + n) * p.acts_ld;
+            __half* dst = sg.sh ? p.acts_sh + (size_t)n * p.Sp : p.acts + (size_t)(sg.ro + n) * p.Ip;
             dst[arow] = __float2half_rn(a);
           }
         }
     }
+    entry_group_done(p, sg, s, ctid);
   } else {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
@@ -340,8 +380,8 @@ TSM_DEV void group_epilogue(PhaseSmem& s, const PhaseParams& p, const Seg& sg, f
         for (int hh = 0; hh < 2; ++hh) {
           const int n = nt * 8 + 2 * c + hh;
           if (n < sg.nc) {
-            const int route = sg.sh ? s.MK + n : sg.ro + n;
-            float* dst = p.P + (size_t)route * p.H + h0;
+            const int route = sg.sh ? p.rp.M * p.rp.K + n : sg.ro + n;
+            float* dst = p.P + (size_t)route * p.rp.H + h0;
             dst[0] = acc[r][nt][hh];
             dst[8] = acc[r][nt][2 + hh];
           }
@@ -350,9 +390,9 @@ TSM_DEV void group_epilogue(PhaseSmem& s, const PhaseParams& p, const Seg& sg, f
   }
 }
 
-template <int FMT, int PHASE, int NT>
-TSM_DEV void consume_seg(PhaseSmem& s, const PhaseParams& p, const Seg& sg, int& wi, int& wph, int& xi, int& xph,
-                         int warp, int lane, int ctid, long long U, int NB) {
+template <int FMT, int PH, int NT>
+TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int& wi, int& wph, int& xi, int& xph,
+                         int warp, int lane, int ctid, int NB) {
   constexpr int KC = FMT == 1 ? 64 : 32;
   constexpr int KWC = KW / KC;
   float acc[RW][NT][4];
@@ -389,17 +429,18 @@ TSM_DEV void consume_seg(PhaseSmem& s, const PhaseParams& p, const Seg& sg, int&
     ws = we;
   }
 
-  const bool whole = sg.c0 == 0 && sg.c1 == sg.chunks;
-  if (whole) {
-    group_epilogue<PHASE, NT>(s, p, sg, acc, warp, lane, ctid);
+  if (sg.c0 == 0 && sg.c1 == sg.chunks) {
+    group_epilogue<PH, NT>(s, p, sg, acc, warp, lane, ctid);
     return;
   }
   // split group: publish this CTA's partial
   const int b = blockIdx.x;
   const int g = lane >> 2, c = lane & 3;
+  const unsigned* rs = PH == 0 ? s.rs0 : s.rs1;
+  float* slots = PH == 0 ? p.partial0 : p.partial1;
   {
-    const int slot = s.rs[b] >= (unsigned)sg.g0 ? 0 : 1;
-    float* sp = p.partial + ((size_t)b * 2 + slot) * SLOT_FLOATS;
+    const int slot = rs[b] >= (unsigned)sg.g0 ? 0 : 1;
+    float* sp = slots + ((size_t)b * 2 + slot) * SLOT_FLOATS;
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       const int jt = warp * RW + r;
@@ -412,11 +453,11 @@ TSM_DEV void consume_seg(PhaseSmem& s, const PhaseParams& p, const Seg& sg, int&
       }
     }
   }
-  if (PHASE == 1) return;  // phase 2 combines everything after the grid barrier
-  // phase 1: the last contributor of the group finishes it
+  if (PH == 1) return;  // down partials are combined after the grid barrier
+  // gate/up: the last contributor of the group finishes it
   __threadfence();
   bar_sync(1, NWC * 32);
-  const int key = (sg.sh ? p.E : s.ex[sg.j]) * p.ng_max + sg.grp;
+  const int key = (sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp;
   if (ctid == 0) {
     const unsigned inc = (unsigned)(sg.c1 - sg.c0);
     s.flag = (atomicAdd(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks);
@@ -428,12 +469,12 @@ TSM_DEV void consume_seg(PhaseSmem& s, const PhaseParams& p, const Seg& sg, int&
   for (int r = 0; r < RW; ++r)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[r][nt][0] = acc[r][nt][1] = acc[r][nt][2] = acc[r][nt][3] = 0.f;
-  const int bf = owner_tab(s, NB, (unsigned)sg.g0);
-  const int bl = owner_tab(s, NB, (unsigned)(sg.g0 + sg.chunks - 1));
+  const int bf = owner_tab(rs, NB, (unsigned)sg.g0);
+  const int bl = owner_tab(rs, NB, (unsigned)(sg.g0 + sg.chunks - 1));
   for (int b2 = bf; b2 <= bl; ++b2) {
-    if (s.rs[b2] == s.rs[b2 + 1]) continue;  // empty range
-    const int slot = s.rs[b2] >= (unsigned)sg.g0 ? 0 : 1;
-    const float* sp = p.partial + ((size_t)b2 * 2 + slot) * SLOT_FLOATS;
+    if (rs[b2] == rs[b2 + 1]) continue;  // empty range
+    const int slot = rs[b2] >= (unsigned)sg.g0 ? 0 : 1;
+    const float* sp = slots + ((size_t)b2 * 2 + slot) * SLOT_FLOATS;
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       const int jt = warp * RW + r;
@@ -451,18 +492,132 @@ TSM_DEV void consume_seg(PhaseSmem& s, const PhaseParams& p, const Seg& sg, int&
     }
   }
   if (ctid == 0) p.cnt_group[key] = 0u;
-  group_epilogue<PHASE, NT>(s, p, sg, acc, warp, lane, ctid);
+  group_epilogue<PH, NT>(s, p, sg, acc, warp, lane, ctid);
 }
 
-template <int FMT, int PHASE>
-__global__ void __launch_bounds__(NTHREADS, 1) expert_kernel(const PhaseParams p) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  PhaseSmem& s = *reinterpret_cast<PhaseSmem*>(smem_raw);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NB = gridDim.x;
+// Producer: weight stages and activation windows of phase PH in consumer order.
+template <int FMT, int PH>
+TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, long long u1, int& wi, int& wph, int& xi,
+                           int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_mine) {
   constexpr int KC = FMT == 1 ? 64 : 32;
   constexpr int KWC = KW / KC;
+  long long u = u0;
+  int j = 0;
+  Seg sg;
+  bool alive = true;
+  while (alive && next_seg<PH>(s, p, u, u1, j, sg)) {
+    const uint8_t* mat = PH == 0 ? (sg.sh ? p.wBs : p.wB + (uint64_t)s.r.ex[sg.j] * p.wB_stride)
+                                 : (sg.sh ? p.wCs : p.wC + (uint64_t)s.r.ex[sg.j] * p.wC_stride);
+    const uint8_t* gbase = mat + group_offset(sg.gs, sg.chunks, sg.grp);
+    const __half* brow = nullptr;
+    if (lane < sg.nc) {
+      if (PH == 0)
+        brow = xh_mine + (size_t)(sg.sh ? lane : s.r.tok[sg.ro + lane]) * p.rp.Hp;
+      else
+        brow = sg.sh ? p.acts_sh + (size_t)lane * p.Sp : p.acts + (size_t)(sg.ro + lane) * p.Ip;
+    }
+    const unsigned ustride = (unsigned)sg.ntg * UNIT_BYTES;
+    int k_issued = sg.c0;  // first chunk whose weight stage is not yet issued
+    for (int ws = sg.c0; alive && ws < sg.c1;) {
+      const int we = min(sg.c1, (ws / KWC + 1) * KWC);
+      if (PH == 1 && ws == sg.c0) {
+        // down: prefetch weight stages of the first window, then wait until the
+        // expert's acts are complete before fetching them
+        for (int pre = 0; pre < NSW && k_issued < we && alive; ++pre) {
+          const int kk = min(KS, we - k_issued);
+          if (lane == 0) {
+            alive = mbar_wait(&s.wempty[wi], wph ^ 1, &s.dead, p.err, ERR_TIMEOUT_WEMPTY);
+            if (alive) {
+              mbar_arrive_expect_tx(&s.wfull[wi], (unsigned)kk * ustride);
+              bulk_g2s_hint(s.w[wi], gbase + (uint64_t)k_issued * ustride, (unsigned)kk * ustride, &s.wfull[wi], pol);
+            }
+          }
+          alive = __shfl_sync(0xffffffffu, alive, 0);
+          ++wuse[wi];
+          if (++wi == NSW) {
+            wi = 0;
+            wph ^= 1;
+          }
+          k_issued += kk;
+        }
+        if (lane == 0 && alive) {
+          const unsigned need = (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups);
+          const unsigned* done = p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]);
+          const unsigned long long t0 = globaltimer();
+          while (ld_acquire_u32(done) < need) {
+            if (s.dead) break;
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+              s.dead = 1;
+              atomicOr(p.err, ERR_TIMEOUT_ACTS);
+              break;
+            }
+          }
+        }
+        alive = __shfl_sync(0xffffffffu, alive && !s.dead, 0);
+        if (!alive) break;
+        // the acts were written through the generic proxy by other CTAs; the
+        // bulk copies below read them through the async proxy
+        __threadfence();
+        fence_proxy_async_global();
+      }
+      const unsigned xbytes = (unsigned)(we - ws) * KC * 2;
+      if (lane == 0) {
+        alive = mbar_wait(&s.xempty[xi], xph ^ 1, &s.dead, p.err, ERR_TIMEOUT_XEMPTY);
+        if (alive) mbar_arrive_expect_tx(&s.xfull[xi], xbytes * (unsigned)sg.nc);
+      }
+      alive = __shfl_sync(0xffffffffu, alive, 0);
+      if (!alive) break;
+      if (lane < sg.nc) bulk_g2s(s.x[xi] + lane * XROW, brow + (size_t)ws * KC, xbytes, &s.xfull[xi]);
+      ++xuse[xi];
+      if (++xi == NSX) {
+        xi = 0;
+        xph ^= 1;
+      }
+      for (int k = max(ws, k_issued); k < we; k += KS) {
+        const int kk = min(KS, we - k);
+        if (lane == 0) {
+          alive = mbar_wait(&s.wempty[wi], wph ^ 1, &s.dead, p.err, ERR_TIMEOUT_WEMPTY);
+          if (alive) {
+            mbar_arrive_expect_tx(&s.wfull[wi], (unsigned)kk * ustride);
+            bulk_g2s_hint(s.w[wi], gbase + (uint64_t)k * ustride, (unsigned)kk * ustride, &s.wfull[wi], pol);
+          }
+        }
+        alive = __shfl_sync(0xffffffffu, alive, 0);
+        if (!alive) break;
+        ++wuse[wi];
+        if (++wi == NSW) {
+          wi = 0;
+          wph ^= 1;
+        }
+      }
+      k_issued = max(k_issued, we);
+      ws = we;
+    }
+  }
+  return alive;
+}
 
+template <int FMT>
+__global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  LayerSmem& s = *reinterpret_cast<LayerSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NB = gridDim.x, b = blockIdx.x;
+
+  // ---- 1. route (every CTA; identical arithmetic to route_kernel)
+  RouteParams rp = p.rp;
+  if (b != 0) {
+    rp.logits = nullptr;
+    rp.idx = nullptr;
+    rp.w = nullptr;
+    rp.shift = nullptr;
+    rp.meta = nullptr;
+    rp.routes = nullptr;
+    rp.rpos = nullptr;
+  }
+  const RouterSplit rsplit(rp.rg, warp);
+  RoutePrefetch pf;
+  route_prefetch(rp, rsplit, lane, pf);
   if (tid == 0) {
     for (int i = 0; i < NSW; ++i) {
       mbar_init(&s.wfull[i], 1);
@@ -474,133 +629,65 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_kernel(const PhaseParams p
     }
     fence_barrier_init();
     s.dead = 0;
-    if (PHASE == 1) s.gen0 = ld_acquire_u32(p.grid_gen);
   }
   grid_dep_wait();
   grid_dep_launch();
-  if (tid == 0) {
-    s.M = p.meta[META_M];
-    s.nT = p.meta[META_NT];
-    s.MK = p.meta[META_MK];
-    s.has_shared = p.meta[META_HAS_SHARED];
-    s.nE = p.meta[META_NE];
-    if (s.nE < 0 || s.nE > MAX_ENTRIES || s.MK > MAX_TOK * MAX_K || s.nT > MAX_E || s.M > MAX_TOK) {
-      atomicOr(p.err, ERR_BAD_META);
-      s.nE = 0;
-      s.nT = 0;
-    }
-  }
+  if (tid == 0) s.gen0 = ld_acquire_u32(p.grid_gen);
+  __half* xh_mine = p.xh_cta + (size_t)b * p.xh_stride;
+  __half* rin_mine = p.rin_cta ? p.rin_cta + (size_t)b * p.rin_stride : nullptr;
+  route_shift(rp, s.r, warp, lane);
+  __syncthreads();
+  // the router input is staged in the (still idle) weight and window rings when it fits
+  const bool stage = route_stage_bytes(rp.M, rp.Hp, rp.xscale != nullptr) <= sizeof(s.w) + sizeof(s.x);
+  __half* bs = stage ? reinterpret_cast<__half*>(&s.w[0][0]) : nullptr;
+  route_convert(rp, s.r, xh_mine, rin_mine, bs, tid, NTHREADS);
+  fence_proxy_async_global();  // the producer reads xh_mine with bulk copies
   __syncthreads();
   {
-    // entries in parallel; every routed entry has the same geometry, so the
-    // unit prefixes have closed forms
-    const long long units_r = (long long)p.gr.ngroups * p.gr.chunks;
-    for (int j = tid; j < s.nE; j += NTHREADS) {
-      int ex = p.meta[META_EX + j], ro = p.meta[META_RO + j], nc = p.meta[META_NC + j];
-      const bool sh = s.has_shared && j == s.nT;
-      if (nc < 1 || nc > MAX_TOK || ro < 0 || (!sh && (ex < 0 || ex >= p.E || ro + nc > MAX_TOK * MAX_K))) {
-        atomicOr(p.err, ERR_BAD_META);
-        nc = 1;
-        ex = 0;
-        ro = 0;
-      }
-      s.ex[j] = ex;
-      s.ro[j] = ro;
-      s.nc[j] = nc;
-      s.upre[j] = (long long)j * units_r;
-      s.cpre[j] = j * p.gr.chunks;
-      if (!sh)
-        for (int n = 0; n < nc; ++n) s.rj[ro + n] = j;
-    }
-    if (tid == 0) {
-      const bool hs = s.has_shared && s.nE > s.nT;
-      s.upre[s.nE] = (long long)s.nT * units_r + (hs ? (long long)p.gsh.ngroups * p.gsh.chunks : 0);
-      s.cpre[s.nE] = s.nT * p.gr.chunks + (hs ? p.gsh.chunks : 0);
-    }
+    const __half* bsrc = bs ? bs : (rp.xscale ? rin_mine : xh_mine);
+    const int ld = bs ? route_bs_ld(rp.Hp) : rp.Hp;
+    if (rp.M > 8)
+      route_gemv<2>(rp, s.r, rsplit, pf, bsrc, ld, warp, lane, tid, NTHREADS);
+    else
+      route_gemv<1>(rp, s.r, rsplit, pf, bsrc, ld, warp, lane, tid, NTHREADS);
   }
-  for (int i = tid; i < MAX_TOK * MAX_K; i += NTHREADS) {
-    int tk = 0;
-    if (i < s.MK) {
-      tk = p.routes[i].token;
-      if (tk < 0 || tk >= MAX_TOK) {
-        atomicOr(p.err, ERR_BAD_INDEX);
-        tk = 0;
-      }
-    }
-    s.tok[i] = tk;
-  }
+  route_topk(rp, s.r, warp, lane);
   __syncthreads();
+  route_list(rp, s.r, warp, lane, tid, NTHREADS);
+  fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
 
-  const long long U = s.upre[s.nE];
-  if (U == 0) return;
-  for (int b = tid; b <= NB; b += NTHREADS) s.rs[b] = (unsigned)range_start((uint64_t)U, NB, b);
+  // ---- unit prefixes and the per-phase CTA ranges
+  const int nE = s.r.nE, nT = s.r.nT;
+  const bool hs = rp.has_shared != 0;
+  const long long units_b = (long long)p.gB.ngroups * p.gB.chunks;
+  for (int j = tid; j <= nE; j += NTHREADS) {
+    s.upre0[j] = (long long)min(j, nT) * units_b + (j > nT ? (long long)p.gBs.ngroups * p.gBs.chunks : 0);
+    s.cpre1[j] = min(j, nT) * p.gC.chunks + (j > nT ? p.gCs.chunks : 0);
+  }
   __syncthreads();
-  const long long u0 = (long long)range_start((uint64_t)U, NB, blockIdx.x);
-  const long long u1 = (long long)range_start((uint64_t)U, NB, blockIdx.x + 1);
-  if (u0 >= u1 && PHASE == 0) return;
+  const long long U0 = s.upre0[nE];
+  const long long U1 = (long long)p.gC.ngroups * s.cpre1[nE];
+  for (int i = tid; i <= NB; i += NTHREADS) {
+    s.rs0[i] = (unsigned)range_start((uint64_t)U0, NB, i);
+    s.rs1[i] = (unsigned)range_start((uint64_t)U1, NB, i);
+  }
+  __syncthreads();
+  const long long a0 = s.rs0[b], a1 = s.rs0[b + 1], d0 = s.rs1[b], d1 = s.rs1[b + 1];
+  (void)hs;
 
   if (warp == NWC) {
-    // ---------------------------------------------------------------- producer warp
+    // ------------------------------------------------------------ producer warp
     const uint64_t pol = policy_evict_first();
     int wi = 0, wph = 0, xi = 0, xph = 0;
     int wuse[NSW], xuse[NSX];
     for (int i = 0; i < NSW; ++i) wuse[i] = 0;
     for (int i = 0; i < NSX; ++i) xuse[i] = 0;
-    long long u = u0;
-    int j = 0;
-    Seg sg;
-    bool alive = true;
-    while (alive && next_seg<PHASE == 1>(s, p, u, u1, j, sg)) {
-      const uint8_t* mat = sg.sh ? p.w_shared : p.w_routed + (uint64_t)s.ex[sg.j] * p.w_stride;
-      const uint8_t* gbase = mat + group_offset(sg.gs, sg.chunks, sg.grp);
-      const __half* brow = nullptr;
-      if (lane < sg.nc) {
-        if (PHASE == 0)
-          brow = sg.sh ? p.b_shared + (size_t)lane * p.b_shared_ld
-                       : p.b_routed + (size_t)s.tok[sg.ro + lane] * p.b_routed_ld;
-        else
-          brow = sg.sh ? p.b_shared + (size_t)lane * p.b_shared_ld : p.b_routed + (size_t)(sg.ro + lane) * p.b_routed_ld;
-      }
-      const unsigned ustride = (unsigned)sg.ntg * UNIT_BYTES;
-      for (int ws = sg.c0; alive && ws < sg.c1;) {
-        const int we = min(sg.c1, (ws / KWC + 1) * KWC);
-        const unsigned xbytes = (unsigned)(we - ws) * KC * 2;
-        if (lane == 0) {
-          alive = mbar_wait(&s.xempty[xi], xph ^ 1, &s.dead, p.err, ERR_TIMEOUT_XEMPTY);
-          if (alive) mbar_arrive_expect_tx(&s.xfull[xi], xbytes * (unsigned)sg.nc);
-        }
-        alive = __shfl_sync(0xffffffffu, alive, 0);
-        if (!alive) break;
-        if (lane < sg.nc) bulk_g2s(s.x[xi] + lane * XROW, brow + (size_t)ws * KC, xbytes, &s.xfull[xi]);
-        ++xuse[xi];
-        if (++xi == NSX) {
-          xi = 0;
-          xph ^= 1;
-        }
-        for (int k = ws; k < we; k += KS) {
-          const int kk = min(KS, we - k);
-          if (lane == 0) {
-            alive = mbar_wait(&s.wempty[wi], wph ^ 1, &s.dead, p.err, ERR_TIMEOUT_WEMPTY);
-            if (alive) {
-              mbar_arrive_expect_tx(&s.wfull[wi], (unsigned)kk * ustride);
-              bulk_g2s_hint(s.w[wi], gbase + (uint64_t)k * ustride, (unsigned)kk * ustride, &s.wfull[wi], pol);
-            }
-          }
-          alive = __shfl_sync(0xffffffffu, alive, 0);
-          if (!alive) break;
-          ++wuse[wi];
-          if (++wi == NSW) {
-            wi = 0;
-            wph ^= 1;
-          }
-        }
-        ws = we;
-      }
-    }
+    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_mine);
+    if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_mine);
     // Copies still in flight must land before the CTA can exit (only matters
     // when a wait gave up): wait, bounded, for each slot's last issued phase.
     if (lane == 0 && s.dead) {
-      unsigned long long t0 = globaltimer();
+      const unsigned long long t0 = globaltimer();
       for (int i = 0; i < NSW; ++i)
         if (wuse[i])
           while (!mbar_try_wait(&s.wfull[i], (wuse[i] - 1) & 1) && globaltimer() - t0 < WAIT_LIMIT_NS) {
@@ -613,21 +700,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_kernel(const PhaseParams p
     return;
   }
 
-  // ------------------------------------------------------------------ consumer warps
+  // ------------------------------------------------------------ consumer warps
   int wi = 0, wph = 0, xi = 0, xph = 0;
-  long long u = u0;
-  int j = 0;
-  Seg sg;
-  while (next_seg<PHASE == 1>(s, p, u, u1, j, sg)) {
-    if (sg.nc > 8)
-      consume_seg<FMT, PHASE, 2>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, U, NB);
-    else
-      consume_seg<FMT, PHASE, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, U, NB);
+  {
+    long long u = a0;
+    int j = 0;
+    Seg sg;
+    while (next_seg<0>(s, p, u, a1, j, sg)) {
+      if (sg.nc > 8)
+        consume_seg<FMT, 0, 2>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
+      else
+        consume_seg<FMT, 0, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
+    }
   }
-  if (PHASE == 1) {
-    grid_barrier(s, p, NB, tid);
-    final_combine(s, p, NB, tid);
+  {
+    long long u = d0;
+    int j = 0;
+    Seg sg;
+    while (next_seg<1>(s, p, u, d1, j, sg)) {
+      if (sg.nc > 8)
+        consume_seg<FMT, 1, 2>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
+      else
+        consume_seg<FMT, 1, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
+    }
   }
+  grid_barrier(s, p, NB, tid);
+  final_combine(s, p, NB, tid);
+  if (b == 0)
+    for (int e = tid; e <= rp.E; e += NWC * 32) p.entry_done[e] = 0u;  // every readiness wait of this launch is over
 }
 
 }  // namespace tsm

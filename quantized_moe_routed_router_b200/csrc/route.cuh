@@ -53,12 +53,13 @@ struct RouteParams {
   const float* bias;       // [E] or null
   const float* pes;        // [E] or null
   int bias_mode, score, has_shared;
-  float* logits;           // [M][E] workspace
-  int* idx;                // [M][K] workspace
-  float* w;                // [M][K] workspace
-  int* shift;              // [M]
-  __half* xh;              // [M][Hp]
-  int* meta;
+  float* logits;           // [M][E] (optional)
+  int* idx;                // [M][K] (optional)
+  float* w;                // [M][K] (optional)
+  int* shift;              // [M] (optional)
+  __half* xh;              // [M][Hp] x as FP16 * 2^shift
+  __half* rin;             // [2][M][Hp] router input hi/lo (used only with an x-scale)
+  int* meta;               // optional global copies of the route list
   Route* routes;           // [M*K]
   int* rpos;               // [M][K] -> position in routes
   unsigned* err;
@@ -69,42 +70,130 @@ struct RouteParams {
 
 TSM_DEV bool topk_better(float v1, int i1, float v2, int i2) { return v1 > v2 || (v1 == v2 && i1 < i2); }
 
-constexpr int ROUTE_THREADS = 512;
-constexpr int ROUTE_WARPS = ROUTE_THREADS / 32;
-constexpr int RKW = 2048;                 // K elements of x staged per window
-constexpr int RROW = RKW * 2 + 32;        // bytes per staged row (= 32 mod 128: conflict-free B loads)
-constexpr int ROUTE_PRE = 6;              // router units per warp fetched before x is ready
+constexpr int ROUTE_WARPS = 16;           // warps that do the router GEMV (tiles are split over them)
+constexpr int ROUTE_PRE = 4;              // router units per warp fetched before x is ready
 
-// Shared memory of the route kernel (dynamic).
-struct RouteSmem {
-  uint8_t xw[2][MAX_TOK][RROW];           // staged x window: [hi/lo][token][K]
+// Routing results, in the shared memory of the kernel that routes.
+struct RouteState {
   float part[ROUTE_WARPS][16][16];        // per-warp partial logits [row][token]
-  float lg[MAX_TOK][MAX_E];               // logits
-  int shift[MAX_TOK];
-  int cnt[MAX_E], off[MAX_E], idx[MAX_TOK * MAX_K];
+  float lg[MAX_TOK][MAX_E];               // logits (before bias)
+  int shift[MAX_TOK];                     // per-token power-of-two scale of x
+  int idx[MAX_TOK * MAX_K];               // selected experts, slot order
+  float w[MAX_TOK * MAX_K];               // their weights
+  int cnt[MAX_E], off[MAX_E];
+  unsigned tmask[MAX_E];                  // tokens that selected each expert (bit t)
+  int ex[MAX_ENTRIES], ro[MAX_ENTRIES], nc[MAX_ENTRIES];  // touched experts (+ shared entry)
+  int tok[MAX_TOK * MAX_K];               // token of each route position
+  int rpos[MAX_TOK * MAX_K];              // route position of each (token, slot)
+  int rj[MAX_TOK * MAX_K];                // entry index of each route position
+  int nT, nE;
 };
 
-// Stages x[t][k0 .. k0+len) (FP32 product with xscale, times 2^shift[t]) as
-// FP16 hi (+ lo when `split`) into the window; also writes xh when `write_xh`.
-TSM_DEV void stage_window(RouteSmem& s, const RouteParams& p, int k0, int len, bool split, bool write_xh) {
-  constexpr int U = 4;  // items (8 elements each) per thread per trip, loads issued together
-  const int per_row = len / 8, total = p.M * per_row;
-  for (int base = threadIdx.x; base < total; base += ROUTE_THREADS * U) {
+// Router work split: warp w (< ROUTE_WARPS) owns tile w / wpt and every wpt-th chunk of it.
+struct RouterSplit {
+  int T, C, wpt, tile, wsub, nunits;
+  TSM_DEV RouterSplit(const MatGeom& g, int warp) {
+    T = g.tiles;
+    C = g.chunks;
+    wpt = ROUTE_WARPS / T;  // warps per tile (T <= 16)
+    tile = warp / wpt;
+    wsub = warp % wpt;
+    nunits = (warp < ROUTE_WARPS && tile < T) ? (C - wsub + wpt - 1) / wpt : 0;
+  }
+  TSM_DEV const uint8_t* unit(const RouteParams& p, int k) const {
+    const int ck = wsub + k * wpt;
+    const int grp = tile / p.rg.gs, jt = tile % p.rg.gs, ntg = group_tiles(T, p.rg.gs, grp);
+    return p.rw + group_offset(p.rg.gs, C, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
+  }
+};
+
+struct RoutePrefetch {
+  uint4 q[ROUTE_PRE];
+  uint32_t sc[ROUTE_PRE];
+};
+
+// The router does not depend on the previous kernel: its first units can be
+// fetched before griddepcontrol.wait.
+TSM_DEV void route_prefetch(const RouteParams& p, const RouterSplit& rs, int lane, RoutePrefetch& pf) {
+#pragma unroll
+  for (int k = 0; k < ROUTE_PRE; ++k)
+    if (k < rs.nunits) {
+      const uint8_t* u = rs.unit(p, k);
+      pf.q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
+      pf.sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
+    }
+}
+
+// Per-token |x| (and |x * xscale|) max -> power-of-two shift (warp t: token t).
+TSM_DEV void route_shift(const RouteParams& p, RouteState& s, int warp, int lane) {
+  if (warp >= p.M) return;
+  const int t = warp;
+  float m = 0.f;
+  constexpr int U = 4;
+  for (int kb = lane * 8; kb < p.H; kb += 32 * 8 * U) {
     uint4 raw[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int i = base + u * ROUTE_THREADS;
+      const int k = kb + u * 256;
+      raw[u] = k < p.H ? *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = kb + u * 256;
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(b2[q]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        if (p.xscale && k < p.H) {
+          m = fmaxf(m, fabsf(f.x * p.xscale[k + 2 * q]));
+          m = fmaxf(m, fabsf(f.y * p.xscale[k + 2 * q + 1]));
+        }
+      }
+    }
+  }
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  int sh = 0;
+  if (m > 0.f && m <= 3.4e38f) {
+    int e2;
+    frexpf(m, &e2);  // m in [2^(e2-1), 2^e2)
+    sh = min(126, max(-126, 14 - e2));
+  }
+  if (lane == 0) {
+    s.shift[t] = sh;
+    if (p.shift) p.shift[t] = sh;
+  }
+}
+
+// Row stride (halves) of the router input staged in shared memory: 32 bytes
+// past a multiple of 128 keeps the B-fragment loads conflict-free.
+TSM_DEV int route_bs_ld(int Hp) { return Hp + 16; }
+
+// x -> FP16 * 2^shift into xh [M][Hp] (zero padded).  The router input (the
+// same values, or with an x-scale x * xscale * 2^shift as an FP16 hi + lo
+// pair) also goes to `bs` (rows route_bs_ld(Hp) halves apart; hi rows 0..M-1,
+// lo rows M..2M-1) when bs is not null, else to `rin` [2][M][Hp].
+TSM_DEV void route_convert(const RouteParams& p, const RouteState& s, __half* xh, __half* rin, __half* bs, int tid,
+                           int nthr) {
+  constexpr int U = 4;
+  const int per_row = p.Hp / 8, total = p.M * per_row, bld = route_bs_ld(p.Hp);
+  const bool split = p.xscale != nullptr;
+  for (int base = tid; base < total; base += nthr * U) {
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * nthr;
       raw[u] = make_uint4(0, 0, 0, 0);
       if (i < total) {
-        const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
+        const int t = i / per_row, k = (i - t * per_row) * 8;
         if (k < p.H) raw[u] = *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int i = base + u * ROUTE_THREADS;
+      const int i = base + u * nthr;
       if (i >= total) break;
-      const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
+      const int t = i / per_row, k = (i - t * per_row) * 8;
       const float sc = __uint_as_float((uint32_t)(s.shift[t] + 127) << 23);
       const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
       __half hx[8], hh[8], hl[8];
@@ -123,16 +212,22 @@ TSM_DEV void stage_window(RouteSmem& s, const RouteParams& p, int k0, int len, b
           hl[2 * q + 1] = __float2half_rn(xb - __half2float(hh[2 * q + 1]));
         }
       }
-      if (write_xh) *reinterpret_cast<uint4*>(p.xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
-      *reinterpret_cast<uint4*>(&s.xw[0][t][(k - k0) * 2]) = *reinterpret_cast<uint4*>(split ? hh : hx);
-      if (split) *reinterpret_cast<uint4*>(&s.xw[1][t][(k - k0) * 2]) = *reinterpret_cast<uint4*>(hl);
+      *reinterpret_cast<uint4*>(xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
+      if (bs) {
+        *reinterpret_cast<uint4*>(bs + (size_t)t * bld + k) = *reinterpret_cast<uint4*>(split ? hh : hx);
+        if (split) *reinterpret_cast<uint4*>(bs + (size_t)(p.M + t) * bld + k) = *reinterpret_cast<uint4*>(hl);
+      } else if (split) {
+        *reinterpret_cast<uint4*>(rin + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hh);
+        *reinterpret_cast<uint4*>(rin + (size_t)(p.M + t) * p.Hp + k) = *reinterpret_cast<uint4*>(hl);
+      }
     }
   }
 }
 
-// One Q8_0 (tile, chunk) unit against the staged window: acc += W x.
+// One Q8_0 (tile, chunk) unit of the router against x rows in global memory
+// (b points at column 32 * chunk of row 0, rows `ld` halves apart): acc += W x.
 template <int NT>
-TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const uint8_t* xc, int lane) {
+TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const __half* b, int ld, int M, int lane) {
   const int g = lane >> 2, c = lane & 3;
   const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&sc));
   float tmp[NT][4];
@@ -142,8 +237,10 @@ TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const uint8_
                           u8x2_to_f16x2<0x4342>(q.w)};
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const uint2 b0 = *reinterpret_cast<const uint2*>(xc + (nt * 8 + g) * RROW + (4 * c) * 2);
-    const uint2 b1 = *reinterpret_cast<const uint2*>(xc + (nt * 8 + g) * RROW + (16 + 4 * c) * 2);
+    const int row = min(nt * 8 + g, M - 1);  // columns past M repeat the last token; their outputs are unused
+    const __half* br = b + (size_t)row * ld;
+    const uint2 b0 = *reinterpret_cast<const uint2*>(br + 4 * c);
+    const uint2 b1 = *reinterpret_cast<const uint2*>(br + 16 + 4 * c);
     mma_f16_zc(tmp[nt], a0, b0.x, b0.y);
     mma_f16_acc(tmp[nt], a1, b1.x, b1.y);
     acc[nt][0] = fmaf(d.x, tmp[nt][0], acc[nt][0]);
@@ -153,77 +250,56 @@ TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const uint8_
   }
 }
 
-// Router work split: warp w owns tile w / wpt and every wpt-th chunk of it.
-struct RouterSplit {
-  int T, C, wpt, tile, wsub, nunits;
-  TSM_DEV RouterSplit(const MatGeom& g, int warp) {
-    T = g.tiles;
-    C = g.chunks;
-    wpt = ROUTE_WARPS / T;  // warps per tile (T <= 16)
-    tile = warp / wpt;
-    wsub = warp % wpt;
-    nunits = tile < T ? (C - wsub + wpt - 1) / wpt : 0;
-  }
-  TSM_DEV const uint8_t* unit(const RouteParams& p, int k) const {
-    const int ck = wsub + k * wpt;
-    const int grp = tile / p.rg.gs, jt = tile % p.rg.gs, ntg = group_tiles(T, p.rg.gs, grp);
-    return p.rw + group_offset(p.rg.gs, C, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
-  }
-};
-
-// Router GEMV over all tokens from the staged windows; pq/ps hold the warp's
-// first ROUTE_PRE units (fetched at kernel start).
+// Router GEMV of all tokens -> s.lg (bias not applied).  bsrc: router input
+// rows `ld` halves apart (lo rows follow the M hi rows with an x-scale), in
+// shared or global memory.  Needs a barrier of the whole CTA after
+// route_convert; ends with one.
 template <int NT>
-TSM_DEV void router_gemv(RouteSmem& s, const RouteParams& p, bool split, int warp, int lane, const RouterSplit& rs,
-                         const uint4 (&pq)[ROUTE_PRE], const uint32_t (&ps)[ROUTE_PRE]) {
+TSM_DEV void route_gemv(const RouteParams& p, RouteState& s, const RouterSplit& rs, const RoutePrefetch& pf,
+                        const __half* bsrc, int ld, int warp, int lane, int tid, int nthr) {
   float acc[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const int nwin = (rs.C * 32 + RKW - 1) / RKW;
-  for (int wdw = 0; wdw < nwin; ++wdw) {
-    const int k0 = wdw * RKW, len = min(RKW, p.Hp - k0);
-    if (wdw > 0) {
-      __syncthreads();
-      stage_window(s, p, k0, len, split, false);
-    }
-    __syncthreads();
-    for (int half = 0; half < (split ? 2 : 1); ++half) {
+  const bool split = p.xscale != nullptr;
+  // units past the prefetched ones: ROUTE_PRE at a time, the next batch in flight while one is used
+  RoutePrefetch nb;
+  auto fetch = [&](RoutePrefetch& f, int k0) {
 #pragma unroll
-      for (int k = 0; k < ROUTE_PRE; ++k) {
-        const int ck = rs.wsub + k * rs.wpt;
-        if (k < rs.nunits && ck * 32 >= k0 && ck * 32 < k0 + len)
-          router_unit<NT>(acc, pq[k], ps[k], &s.xw[half][0][(ck * 32 - k0) * 2], lane);
+    for (int k = 0; k < ROUTE_PRE; ++k)
+      if (k0 + k < rs.nunits) {
+        const uint8_t* u = rs.unit(p, k0 + k);
+        f.q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
+        f.sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
       }
-      for (int kb = ROUTE_PRE; kb < rs.nunits; kb += 4) {  // the rest, four loads in flight at a time
-        uint4 q[4];
-        uint32_t sc[4];
+  };
+  for (int half = 0; half < (split ? 2 : 1); ++half) {
+    const __half* b = bsrc + (size_t)half * p.M * ld;
+    if (ROUTE_PRE < rs.nunits) fetch(nb, ROUTE_PRE);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (kb + k < rs.nunits) {
-            const uint8_t* u = rs.unit(p, kb + k);
-            q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
-            sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
-          }
+    for (int k = 0; k < ROUTE_PRE; ++k)
+      if (k < rs.nunits) router_unit<NT>(acc, pf.q[k], pf.sc[k], b + (rs.wsub + k * rs.wpt) * 32, ld, p.M, lane);
+    for (int kb = ROUTE_PRE; kb < rs.nunits; kb += ROUTE_PRE) {
+      RoutePrefetch cur = nb;
+      if (kb + ROUTE_PRE < rs.nunits) fetch(nb, kb + ROUTE_PRE);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int ck = rs.wsub + (kb + k) * rs.wpt;
-          if (kb + k < rs.nunits && ck * 32 >= k0 && ck * 32 < k0 + len)
-            router_unit<NT>(acc, q[k], sc[k], &s.xw[half][0][(ck * 32 - k0) * 2], lane);
-        }
-      }
+      for (int k = 0; k < ROUTE_PRE; ++k)
+        if (kb + k < rs.nunits)
+          router_unit<NT>(acc, cur.q[k], cur.sc[k], b + (rs.wsub + (kb + k) * rs.wpt) * 32, ld, p.M, lane);
     }
   }
-  const int gq = lane >> 2, c = lane & 3;
+  if (warp < ROUTE_WARPS) {
+    const int gq = lane >> 2, c = lane & 3;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    s.part[warp][gq][nt * 8 + 2 * c] = acc[nt][0];
-    s.part[warp][gq][nt * 8 + 2 * c + 1] = acc[nt][1];
-    s.part[warp][gq + 8][nt * 8 + 2 * c] = acc[nt][2];
-    s.part[warp][gq + 8][nt * 8 + 2 * c + 1] = acc[nt][3];
+    for (int nt = 0; nt < NT; ++nt) {
+      s.part[warp][gq][nt * 8 + 2 * c] = acc[nt][0];
+      s.part[warp][gq][nt * 8 + 2 * c + 1] = acc[nt][1];
+      s.part[warp][gq + 8][nt * 8 + 2 * c] = acc[nt][2];
+      s.part[warp][gq + 8][nt * 8 + 2 * c + 1] = acc[nt][3];
+    }
   }
   __syncthreads();
   // logits[t][e] = sum over the tile's warps in order, times 2^-shift[t]
-  for (int i = threadIdx.x; i < p.M * p.E; i += ROUTE_THREADS) {
+  for (int i = tid; i < p.M * p.E; i += nthr) {
     const int t = i / p.E, e = i - t * p.E;
     const int tl = e >> 4, r = e & 15;
     float v = 0.f;
@@ -233,186 +309,105 @@ TSM_DEV void router_gemv(RouteSmem& s, const RouteParams& p, bool split, int war
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RouteParams p) {
-  extern __shared__ __align__(128) uint8_t route_smem_raw[];
-  RouteSmem& s = *reinterpret_cast<RouteSmem*>(route_smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  // The router does not depend on the previous kernel: fetch this warp's first units now.
-  const RouterSplit rs(p.rg, warp);
-  uint4 pq[ROUTE_PRE];
-  uint32_t ps[ROUTE_PRE];
+// Top-k and weights: warp t handles token t (lane holds experts lane, lane+32, ...).
+TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane) {
+  if (warp >= p.M) return;
+  const int t = warp;
+  constexpr int PER = MAX_E / 32;
+  float vsel[PER], vsc[PER];
+  unsigned taken = 0;
 #pragma unroll
-  for (int k = 0; k < ROUTE_PRE; ++k)
-    if (k < rs.nunits) {
-      const uint8_t* u = rs.unit(p, k);
-      pq[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
-      ps[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
-    }
-
-  grid_dep_wait();
-  grid_dep_launch();
-
-  // ---- per-token |x| and |x * xscale| max -> power-of-two scale (warp t: token t)
-  if (warp < p.M) {
-    const int t = warp;
-    float m = 0.f;
-    constexpr int U = 4;
-    for (int kb = lane * 8; kb < p.H; kb += 32 * 8 * U) {
-      uint4 raw[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int k = kb + u * 256;
-        raw[u] = k < p.H ? *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int k = kb + u * 256;
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(b2[q]);
-          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-          if (p.xscale && k < p.H) {
-            m = fmaxf(m, fabsf(f.x * p.xscale[k + 2 * q]));
-            m = fmaxf(m, fabsf(f.y * p.xscale[k + 2 * q + 1]));
-          }
-        }
-      }
-    }
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    int sh = 0;
-    if (m > 0.f && m <= 3.4e38f) {
-      int e2;
-      frexpf(m, &e2);  // m in [2^(e2-1), 2^e2)
-      sh = min(126, max(-126, 14 - e2));
-    }
-    if (lane == 0) {
-      s.shift[t] = sh;
-      p.shift[t] = sh;
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    const float l = e < p.E ? s.lg[t][e] : -INFINITY;
+    const float ls = (e < p.E && p.bias && p.bias_mode != 0) ? l + p.bias[e] : l;
+    vsel[i] = ls;
+    vsc[i] = (p.bias_mode == 1 && p.bias) ? ls : l;
+    if (e < p.E) {
+      if (p.logits) p.logits[(size_t)t * p.E + e] = l;
+      if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
     }
   }
-  __syncthreads();
-  const bool split = p.xscale != nullptr;
-  // window 0 (and all of xh)
-  stage_window(s, p, 0, min(RKW, p.Hp), split, true);
-  for (int k0 = RKW; k0 < p.Hp; k0 += RKW) {
-    // the rest of xh; windows after the first are restaged inside the GEMV
-    const int len = min(RKW, p.Hp - k0), per_row = len / 8;
-    for (int i = tid; i < p.M * per_row; i += ROUTE_THREADS) {
-      const int t = i / per_row, k = k0 + (i - t * per_row) * 8;
-      const float sc = __uint_as_float((uint32_t)(s.shift[t] + 127) << 23);
-      __half hx[8];
-      if (k < p.H) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(b2[q]);
-          hx[2 * q] = __float2half_rn(f.x * sc);
-          hx[2 * q + 1] = __float2half_rn(f.y * sc);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) hx[q] = __ushort_as_half(0);
-      }
-      *reinterpret_cast<uint4*>(p.xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
-    }
-  }
-  if (p.M > 8)
-    router_gemv<2>(s, p, split, warp, lane, rs, pq, ps);
-  else
-    router_gemv<1>(s, p, split, warp, lane, rs, pq, ps);
-
-  // ---- top-k and weights: warp t handles token t (lane holds experts lane, lane+32, ...)
-  if (warp < p.M) {
-    const int t = warp;
-    constexpr int PER = MAX_E / 32;
-    float vsel[PER], vsc[PER];
-    unsigned taken = 0;
+  int selk = 0;  // lane k holds the k-th selected expert and its score logit
+  float sck = -INFINITY;
+  for (int k = 0; k < p.K; ++k) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane + 32 * i;
-      const float l = e < p.E ? s.lg[t][e] : -INFINITY;
-      const float ls = (e < p.E && p.bias && p.bias_mode != 0) ? l + p.bias[e] : l;
-      vsel[i] = ls;
-      vsc[i] = (p.bias_mode == 1 && p.bias) ? ls : l;
-      if (e < p.E) {
-        p.logits[(size_t)t * p.E + e] = l;
-        if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
+      if (e < p.E && !((taken >> i) & 1u) && topk_better(vsel[i], e, bv, bi)) {
+        bv = vsel[i];
+        bi = e;
       }
     }
-    int selk = 0;  // lane k holds the k-th selected expert and its score logit
-    float sck = -INFINITY;
-    for (int k = 0; k < p.K; ++k) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const int e = lane + 32 * i;
-        if (e < p.E && !((taken >> i) & 1u) && topk_better(vsel[i], e, bv, bi)) {
-          bv = vsel[i];
-          bi = e;
-        }
-      }
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (topk_better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (bi < 0 || bi >= p.E) {  // only with NaN logits
-        if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
-        bi = 0;
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      float mine = 0.f;
-#pragma unroll
-      for (int i = 0; i < PER; ++i)
-        if (i == (bi >> 5)) mine = vsc[i];
-      const float sc = __shfl_sync(0xffffffffu, mine, bi & 31);
-      if (lane == k) {
-        selk = bi;
-        sck = sc;
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (topk_better(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
       }
     }
-    const bool act = lane < p.K;
-    float m = act ? sck : -INFINITY;
-    if (p.score != 0) {
-#pragma unroll
-      for (int i = 0; i < PER; ++i)
-        if (lane + 32 * i < p.E) m = fmaxf(m, vsc[i]);
+    if (bi < 0 || bi >= p.E) {  // only with NaN logits
+      if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
+      bi = 0;
     }
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float den = 0.f;
-    if (p.score == 0) {
-      den = act ? expf(sck - m) : 0.f;
-    } else {
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    float mine = 0.f;
 #pragma unroll
-      for (int i = 0; i < PER; ++i)
-        if (lane + 32 * i < p.E) den += expf(vsc[i] - m);
-    }
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (act) {
-      const float wv = expf(sck - m) / den * (p.pes ? p.pes[selk] : 1.f);
-      s.idx[t * p.K + lane] = selk;
-      p.idx[t * p.K + lane] = selk;
-      p.w[t * p.K + lane] = wv;
-      if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
-      if (p.w_out) p.w_out[t * p.K + lane] = wv;
+    for (int i = 0; i < PER; ++i)
+      if (i == (bi >> 5)) mine = vsc[i];
+    const float sc = __shfl_sync(0xffffffffu, mine, bi & 31);
+    if (lane == k) {
+      selk = bi;
+      sck = sc;
     }
   }
-  for (int e = tid; e < p.E; e += ROUTE_THREADS) s.cnt[e] = 0;
-  __syncthreads();
+  const bool act = lane < p.K;
+  float m = act ? sck : -INFINITY;
+  if (p.score != 0) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (lane + 32 * i < p.E) m = fmaxf(m, vsc[i]);
+  }
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float den = 0.f;
+  if (p.score == 0) {
+    den = act ? expf(sck - m) : 0.f;
+  } else {
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (lane + 32 * i < p.E) den += expf(vsc[i] - m);
+  }
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (act) {
+    const float wv = expf(sck - m) / den * (p.pes ? p.pes[selk] : 1.f);
+    s.idx[t * p.K + lane] = selk;
+    s.w[t * p.K + lane] = wv;
+    if (p.idx) p.idx[t * p.K + lane] = selk;
+    if (p.w) p.w[t * p.K + lane] = wv;
+    if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
+    if (p.w_out) p.w_out[t * p.K + lane] = wv;
+  }
+}
 
-  // ---- route list: group the (token, slot) pairs by expert
+// Route list: the (token, slot) pairs grouped by expert (touched experts in
+// ascending order, tokens ascending), plus the shared expert as the last
+// entry with all M tokens.  Needs a CTA barrier after route_topk; ends with one.
+TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
+  for (int e = tid; e < p.E; e += nthr) {
+    s.cnt[e] = 0;
+    s.tmask[e] = 0u;
+  }
+  __syncthreads();
   const int MK = p.M * p.K;
-  for (int i = tid; i < MK; i += ROUTE_THREADS) atomicAdd(&s.cnt[s.idx[i]], 1);
+  for (int i = tid; i < MK; i += nthr) {
+    atomicAdd(&s.cnt[s.idx[i]], 1);
+    atomicOr(&s.tmask[s.idx[i]], 1u << (i / p.K));
+  }
   __syncthreads();
   if (warp == 0) {
-    // exclusive scan of the counts and compaction of the touched experts
     constexpr int PER = MAX_E / 32;
     int cl[PER], tot = 0, nz = 0;
 #pragma unroll
@@ -437,9 +432,14 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
       if (e < p.E) {
         s.off[e] = run;
         if (cl[i]) {
-          p.meta[META_EX + slot] = e;
-          p.meta[META_RO + slot] = run;
-          p.meta[META_NC + slot] = cl[i];
+          s.ex[slot] = e;
+          s.ro[slot] = run;
+          s.nc[slot] = cl[i];
+          if (p.meta) {
+            p.meta[META_EX + slot] = e;
+            p.meta[META_RO + slot] = run;
+            p.meta[META_NC + slot] = cl[i];
+          }
           ++slot;
         }
         run += cl[i];
@@ -447,32 +447,81 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
     }
     const int nT = __shfl_sync(0xffffffffu, nzincl, 31);
     if (lane == 0) {
+      s.nT = nT;
+      s.nE = nT + (p.has_shared ? 1 : 0);
       if (p.has_shared) {
-        p.meta[META_EX + nT] = p.E;
-        p.meta[META_RO + nT] = MK;
-        p.meta[META_NC + nT] = p.M;
+        s.ex[nT] = p.E;
+        s.ro[nT] = MK;
+        s.nc[nT] = p.M;
       }
-      p.meta[META_M] = p.M;
-      p.meta[META_NT] = nT;
-      p.meta[META_MK] = MK;
-      p.meta[META_HAS_SHARED] = p.has_shared;
-      p.meta[META_NE] = nT + (p.has_shared ? 1 : 0);
+      if (p.meta) {
+        if (p.has_shared) {
+          p.meta[META_EX + nT] = p.E;
+          p.meta[META_RO + nT] = MK;
+          p.meta[META_NC + nT] = p.M;
+        }
+        p.meta[META_M] = p.M;
+        p.meta[META_NT] = nT;
+        p.meta[META_MK] = MK;
+        p.meta[META_HAS_SHARED] = p.has_shared;
+        p.meta[META_NE] = s.nE;
+      }
     }
   }
   __syncthreads();
-  for (int i = tid; i < MK; i += ROUTE_THREADS) {
+  for (int i = tid; i < MK; i += nthr) {
     const int e = s.idx[i], tk = i / p.K;
-    int rank = 0;
-    for (int i2 = 0; i2 < tk * p.K; ++i2) rank += s.idx[i2] == e;
-    const int pos = s.off[e] + rank;
-    Route r;
-    r.token = tk;
-    r.slot = i % p.K;
-    r.expert = e;
-    r.w = p.w[i];
-    p.routes[pos] = r;
-    p.rpos[i] = pos;
+    const int pos = s.off[e] + __popc(s.tmask[e] & ((1u << tk) - 1u));  // tokens before tk that chose e
+    s.tok[pos] = tk;
+    s.rpos[i] = pos;
+    if (p.routes) {
+      Route r;
+      r.token = tk;
+      r.slot = i % p.K;
+      r.expert = e;
+      r.w = s.w[i];
+      p.routes[pos] = r;
+    }
+    if (p.rpos) p.rpos[i] = pos;
   }
+  __syncthreads();
+  // entry index of each route position
+  for (int j = tid; j < s.nT; j += nthr)
+    for (int n = 0; n < s.nc[j]; ++n) s.rj[s.ro[j] + n] = j;
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------- standalone route kernel
+constexpr int ROUTE_THREADS = ROUTE_WARPS * 32;
+
+// Shared memory of route_kernel: RouteState, then the staged router input
+// (2 * M rows of route_bs_ld(Hp) halves) when it fits.
+TSM_HD size_t route_stage_bytes(int M, int Hp, bool split) { return (size_t)(split ? 2 : 1) * M * (Hp + 16) * 2; }
+
+__global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RouteParams p, int stage_in_smem) {
+  extern __shared__ __align__(128) uint8_t route_smem_raw[];
+  RouteState& s = *reinterpret_cast<RouteState*>(route_smem_raw);
+  __half* bs = stage_in_smem ? reinterpret_cast<__half*>(route_smem_raw + ((sizeof(RouteState) + 127) & ~(size_t)127))
+                             : nullptr;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const RouterSplit rs(p.rg, warp);
+  RoutePrefetch pf;
+  route_prefetch(p, rs, lane, pf);
+  grid_dep_wait();
+  grid_dep_launch();
+  route_shift(p, s, warp, lane);
+  __syncthreads();
+  route_convert(p, s, p.xh, p.rin, bs, tid, ROUTE_THREADS);
+  __syncthreads();
+  const __half* bsrc = bs ? bs : (p.xscale ? p.rin : p.xh);
+  const int ld = bs ? route_bs_ld(p.Hp) : p.Hp;
+  if (p.M > 8)
+    route_gemv<2>(p, s, rs, pf, bsrc, ld, warp, lane, tid, ROUTE_THREADS);
+  else
+    route_gemv<1>(p, s, rs, pf, bsrc, ld, warp, lane, tid, ROUTE_THREADS);
+  route_topk(p, s, warp, lane);
+  __syncthreads();
+  route_list(p, s, warp, lane, tid, ROUTE_THREADS);
 }
 
 }  // namespace tsm

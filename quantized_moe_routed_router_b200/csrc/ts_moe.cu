@@ -50,6 +50,7 @@ struct ts_moe {
   int Hp = 0, Ip = 0, Sp = 0;
   MatGeom gR{}, gB{}, gC{}, gBs{}, gCs{};
   int ng_max_B = 0;
+  bool any_xscale = false;
   uint8_t* arena = nullptr;
   size_t arena_bytes = 0;
   uint8_t* ws = nullptr;
@@ -64,10 +65,16 @@ struct ts_moe {
   int* meta = nullptr;
   Route* routes = nullptr;
   __half* xh = nullptr;
+  __half* rin = nullptr;        // route kernel: router input hi/lo (x-scale)
+  __half* xh_cta = nullptr;     // layer kernel: per-CTA x
+  __half* rin_cta = nullptr;
+  size_t xh_stride = 0, rin_stride = 0;
   __half* acts = nullptr;
   __half* acts_sh = nullptr;
   float* P = nullptr;
-  float* partial = nullptr;
+  float* partial0 = nullptr;
+  float* partial1 = nullptr;
+  unsigned* entry_done = nullptr;
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group) chunk counters
   unsigned* grid = nullptr;     // down: grid barrier {arrivals, generation}
   unsigned* err = nullptr;
@@ -151,6 +158,16 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
   return TS_MOE_OK;
 }
 
+// Dynamic shared memory of route_kernel: RouteState, then the staged router
+// input when it fits under ROUTE_SMEM_MAX.
+constexpr int ROUTE_SMEM_MAX = 220 * 1024;
+size_t route_smem(int M, int Hp, bool split, int* stage) {
+  const size_t base = (sizeof(RouteState) + 127) & ~(size_t)127;
+  const size_t want = base + route_stage_bytes(M, Hp, split);
+  *stage = want <= (size_t)ROUTE_SMEM_MAX;
+  return *stage ? want : base;
+}
+
 template <typename... Args>
 cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t lc = {};
@@ -167,13 +184,10 @@ cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cud
 }
 
 ts_moe_status set_smem_attrs(ts_moe* h) {
-  const int bytes = (int)sizeof(PhaseSmem);
-  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(expert_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)sizeof(RouteSmem)));
+  const int bytes = (int)sizeof(LayerSmem);
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX));
   return TS_MOE_OK;
 }
 
@@ -233,6 +247,13 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
   }
   h->ng_max_B = std::max(h->gB.ngroups, S ? h->gBs.ngroups : 0);
+  for (int l = 0; l < c.num_layers && !h->any_xscale; ++l)
+    if (layers[l].router_xscale)
+      for (int n = 0; n < H; ++n)
+        if (layers[l].router_xscale[n] != 0x3F80u) {
+          h->any_xscale = true;
+          break;
+        }
   h->expert_bytes = 2ull * I * blob_row_bytes(fmt, H) + (uint64_t)H * blob_row_bytes(fmt, I);
   h->router_bytes = (uint64_t)E * blob_row_bytes(TS_FMT_Q8_0, H);
   h->shared_bytes = S ? 2ull * S * blob_row_bytes(TS_FMT_Q8_0, H) + (uint64_t)H * blob_row_bytes(TS_FMT_Q8_0, S) : 0;
@@ -296,12 +317,18 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_meta = slot((size_t)META_INTS * 4);
     const size_t o_routes = slot((size_t)Mx * K * sizeof(Route));
     const size_t o_xh = slot((size_t)Mx * h->Hp * 2);
+    const size_t o_rin = slot(h->any_xscale ? (size_t)2 * Mx * h->Hp * 2 : 16);
+    h->xh_stride = (size_t)Mx * h->Hp;
+    h->rin_stride = h->any_xscale ? (size_t)2 * Mx * h->Hp : 0;
+    const size_t o_xhc = slot((size_t)h->nb * h->xh_stride * 2);
+    const size_t o_rinc = slot(h->any_xscale ? (size_t)h->nb * h->rin_stride * 2 : 16);
     const size_t o_acts = slot((size_t)Mx * K * h->Ip * 2);
     const size_t o_acts_sh = slot((size_t)Mx * std::max(h->Sp, 64) * 2);
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
-    const size_t o_partial = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
+    const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
+    const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + 2 + 1;
+    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + (E + 1) + 2 + 1;
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -318,15 +345,20 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->meta = (int*)(h->ws + o_meta);
     h->routes = (Route*)(h->ws + o_routes);
     h->xh = (__half*)(h->ws + o_xh);
+    h->rin = h->any_xscale ? (__half*)(h->ws + o_rin) : nullptr;
+    h->xh_cta = (__half*)(h->ws + o_xhc);
+    h->rin_cta = h->any_xscale ? (__half*)(h->ws + o_rinc) : nullptr;
     h->acts = (__half*)(h->ws + o_acts);
     h->acts_sh = (__half*)(h->ws + o_acts_sh);
     h->P = (float*)(h->ws + o_P);
-    h->partial = (float*)(h->ws + o_partial);
+    h->partial0 = (float*)(h->ws + o_part0);
+    h->partial1 = (float*)(h->ws + o_part1);
     unsigned* cn = (unsigned*)(h->ws + o_cnt);
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
     h->cnt_gB = cn;
-    h->grid = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
+    h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
+    h->grid = h->entry_done + (E + 1);
     h->err = h->grid + 2;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
@@ -446,6 +478,7 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   const ts_moe_config& c = h->cfg;
   const LayerDev& d = h->layers[layer];
   RouteParams rp;
+  std::memset(&rp, 0, sizeof(rp));
   rp.x = (const __nv_bfloat16*)x;
   rp.M = M;
   rp.H = c.hidden;
@@ -465,13 +498,11 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.w = h->w;
   rp.shift = h->shift;
   rp.xh = h->xh;
+  rp.rin = h->rin;
   rp.meta = h->meta;
   rp.routes = h->routes;
   rp.rpos = h->rpos;
   rp.err = h->err;
-  rp.idx_out = nullptr;
-  rp.w_out = nullptr;
-  rp.logits_out = nullptr;
   return rp;
 }
 
@@ -485,7 +516,9 @@ static ts_moe_status check_call(ts_moe* h, int layer, const void* x, int M) {
 }
 
 static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t st) {
-  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, sizeof(RouteSmem), st, rp);
+  int stage = 0;
+  const size_t smem = route_smem(rp.M, rp.Hp, rp.xscale != nullptr, &stage);
+  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, smem, st, rp, stage);
   if (e != cudaSuccess) return cuda_fail(h, e, "route_kernel launch");
   return TS_MOE_OK;
 }
@@ -511,79 +544,51 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   cudaStream_t st = (cudaStream_t)stream;
   const ts_moe_config& c = h->cfg;
   const LayerDev& d = h->layers[layer];
-  RouteParams rp = route_params(h, layer, x, M);
-  if ((s = launch_route(h, rp, st)) != TS_MOE_OK) return s;
+  LayerParams lp;
+  std::memset(&lp, 0, sizeof(lp));
+  lp.rp = route_params(h, layer, x, M);
+  lp.xh_cta = h->xh_cta;
+  lp.rin_cta = lp.rp.xscale ? h->rin_cta : nullptr;
+  lp.xh_stride = (int)h->xh_stride;
+  lp.rin_stride = (int)h->rin_stride;
+  lp.wB = d.wB;
+  lp.wB_stride = h->gB.bytes;
+  lp.wBs = d.wBs;
+  lp.wC = d.wC;
+  lp.wC_stride = h->gC.bytes;
+  lp.wCs = d.wCs;
+  lp.gB = h->gB;
+  lp.gBs = h->gBs;
+  lp.gC = h->gC;
+  lp.gCs = h->gCs;
+  lp.acts = h->acts;
+  lp.acts_sh = h->acts_sh;
+  lp.Ip = h->Ip;
+  lp.Sp = h->Sp;
+  lp.P = h->P;
+  lp.partial0 = h->partial0;
+  lp.partial1 = h->partial1;
+  lp.cnt_group = h->cnt_gB;
+  lp.ng_max = h->ng_max_B;
+  lp.entry_done = h->entry_done;
+  lp.grid_cnt = h->grid;
+  lp.grid_gen = h->grid + 1;
+  lp.y = y;
+  lp.resid = (__nv_bfloat16*)resid;
+  lp.err = h->err;
+  lp.act = c.act;
+  lp.alpha = c.act_alpha;
+  lp.limit = c.act_limit;
 
-  PhaseParams pp;
-  std::memset(&pp, 0, sizeof(pp));
-  pp.meta = h->meta;
-  pp.routes = h->routes;
-  pp.shift = h->shift;
-  pp.wts = h->w;
-  pp.rpos = h->rpos;
-  pp.partial = h->partial;
-  pp.err = h->err;
-  pp.H = c.hidden;
-  pp.K = c.top_k;
-  pp.E = c.num_experts;
-  pp.act = c.act;
-  pp.alpha = c.act_alpha;
-  pp.limit = c.act_limit;
-  pp.acts = h->acts;
-  pp.acts_ld = h->Ip;
-  pp.acts_sh = h->acts_sh;
-  pp.acts_sh_ld = h->Sp;
-  pp.P = h->P;
-  pp.y = y;
-  pp.resid = (__nv_bfloat16*)resid;
-  pp.grid_cnt = h->grid;
-  pp.grid_gen = h->grid + 1;
-
-  // phase 1: gate/up + activation
-  PhaseParams p1 = pp;
-  p1.w_routed = d.wB;
-  p1.w_stride = h->gB.bytes;
-  p1.w_shared = d.wBs;
-  p1.gr = h->gB;
-  p1.gsh = h->gBs;
-  p1.b_routed = h->xh;
-  p1.b_routed_ld = h->Hp;
-  p1.b_shared = h->xh;
-  p1.b_shared_ld = h->Hp;
-  p1.cnt_group = h->cnt_gB;
-  p1.ng_max = h->ng_max_B;
-  // phase 2: down + combine
-  PhaseParams p2 = pp;
-  p2.w_routed = d.wC;
-  p2.w_stride = h->gC.bytes;
-  p2.w_shared = d.wCs;
-  p2.gr = h->gC;
-  p2.gsh = h->gCs;
-  p2.b_routed = h->acts;
-  p2.b_routed_ld = h->Ip;
-  p2.b_shared = h->acts_sh;
-  p2.b_shared_ld = h->Sp;
-  p2.cnt_group = nullptr;
-  p2.ng_max = 0;
-
-  const size_t smem = sizeof(PhaseSmem);
+  const size_t smem = sizeof(LayerSmem);
   cudaError_t e;
   if (h->timing) cudaEventRecord(h->ev[0], st);
   if (c.expert_fmt == TS_FMT_MXFP4)
-    e = launch_pdl(expert_kernel<1, 0>, h->nb, NTHREADS, smem, st, p1);
+    e = launch_pdl(layer_kernel<1>, h->nb, NTHREADS, smem, st, lp);
   else
-    e = launch_pdl(expert_kernel<0, 0>, h->nb, NTHREADS, smem, st, p1);
-  if (e != cudaSuccess) return cuda_fail(h, e, "gate/up kernel launch");
-  if (h->timing) {
-    cudaEventRecord(h->ev[1], st);
-    cudaEventRecord(h->ev[2], st);
-  }
-  if (c.expert_fmt == TS_FMT_MXFP4)
-    e = launch_pdl(expert_kernel<1, 1>, h->nb, NTHREADS, smem, st, p2);
-  else
-    e = launch_pdl(expert_kernel<0, 1>, h->nb, NTHREADS, smem, st, p2);
-  if (e != cudaSuccess) return cuda_fail(h, e, "down kernel launch");
-  if (h->timing) cudaEventRecord(h->ev[3], st);
+    e = launch_pdl(layer_kernel<0>, h->nb, NTHREADS, smem, st, lp);
+  if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
+  if (h->timing) cudaEventRecord(h->ev[1], st);
   return TS_MOE_OK;
 }
 
@@ -657,7 +662,7 @@ ts_moe_status noalloc_setup(int dev, uint8_t** out) {
     void* ptr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(RouteSmem));
+    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX);
     if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
     g_noalloc_ptr[dev] = (uint8_t*)ptr;
   }
@@ -742,7 +747,9 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   rp.idx_out = idx;
   rp.w_out = w;
   rp.logits_out = logits;
-  e = launch_pdl(route_kernel, 1, ROUTE_THREADS, sizeof(RouteSmem), s, rp);
+  int stage = 0;
+  const size_t rsm = route_smem(M, Hp, false, &stage);
+  e = launch_pdl(route_kernel, 1, ROUTE_THREADS, rsm, s, rp, stage);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("route_kernel launch: ") + cudaGetErrorString(e));
   return TS_MOE_OK;
 }
