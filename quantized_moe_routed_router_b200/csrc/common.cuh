@@ -21,6 +21,9 @@ enum : unsigned {
   ERR_BAD_META = 1u << 5,        // route metadata inconsistent with the launch
   ERR_TIMEOUT_GRID = 1u << 6,    // a CTA gave up waiting at the grid-wide barrier
   ERR_TIMEOUT_ACTS = 1u << 7,    // a down producer gave up waiting for an expert's acts
+  ERR_TIMEOUT_XSTAGE = 1u << 8,  // the routing gave up waiting for the bulk copy of x
+  ERR_TIMEOUT_XH = 1u << 9,      // a producer gave up waiting for the shared FP16 x
+  ERR_TIMEOUT_ROUTE = 1u << 10,  // a CTA gave up waiting for the published router logits
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -135,6 +138,9 @@ TSM_DEV unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+TSM_DEV void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 TSM_DEV int ld_cg_i(const int* p) {
   int v;

@@ -54,9 +54,11 @@ static_assert(ROUTE_WARPS <= NWC + 1, "routing uses the first ROUTE_WARPS warps"
 
 struct LayerParams {
   RouteParams rp;           // routing inputs; its output pointers are written by CTA 0 only
-  __half* xh_cta;           // [NB][Mmax*Hp] per-CTA FP16 x (gate/up B operand)
-  __half* rin_cta;          // [NB][2*Mmax*Hp] per-CTA router input hi/lo (x-scale only) or null
-  int xh_stride, rin_stride;
+  __half* xh;               // [Mmax][Hp] FP16 x (the gate/up B operand), slice c written by CTA c
+  unsigned* xh_cnt;         // slices of xh written (reset at the end of each launch)
+  float* part_pub;          // [S][M][E] router items (tile j's 16 experts of slice c by CTA j * S + c)
+  float* max_pub;           // [S][M] |x| max of each slice
+  unsigned* route_cnt;      // router items published (reset at the end of each launch)
   const uint8_t* wB;        // gate/up: expert e at wB + e * wB_stride
   uint64_t wB_stride;
   const uint8_t* wBs;       // shared gate/up or null
@@ -73,8 +75,8 @@ struct LayerParams {
   unsigned* cnt_group;      // [(E+1) * ng_max] gate/up chunk counters
   int ng_max;
   unsigned* entry_done;     // [E+1] gate/up groups finished per expert (+ shared)
-  unsigned* grid_cnt;       // grid barrier arrivals
-  unsigned* grid_gen;       // grid barrier generation
+  unsigned* grid_cnt;       // grid barrier arrivals, never reset: NB per launch
+  unsigned* grid_gen;       // launches completed (the last arriver of each grid barrier adds 1)
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
   unsigned* err;
@@ -264,20 +266,38 @@ TSM_DEV float down_value(const LayerSmem& s, const LayerParams& p, unsigned owne
   return v;
 }
 
-// After the grid barrier: this CTA's 1/NB slice of the M x H outputs,
-// y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared) in slot order; resid += y.
-// The (row group, entry) -> contributing CTAs table goes in the routing
-// scratch (free by now) when it fits.
-TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid) {
-  const int M = p.rp.M, K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = M * K, nE = s.r.nE;
+// This CTA's 1/NB slice [lo, hi) of the M x H outputs.
+TSM_DEV void combine_range(const LayerParams& p, int NB, int& lo, int& hi) {
+  const long long MH = (long long)p.rp.M * p.rp.H;
+  lo = (int)(MH * blockIdx.x / NB);
+  hi = (int)(MH * (blockIdx.x + 1) / NB);
+}
+
+// Before the grid barrier (nothing here depends on other CTAs' down work):
+// the (row group, entry) -> contributing CTAs table, in the routing scratch
+// when it fits (returns whether it does), and the residual of this thread's
+// first output of the combine.
+TSM_DEV bool combine_prepare(LayerSmem& s, const LayerParams& p, int NB, int ctid, float& r0) {
+  const int nE = s.r.nE;
   unsigned* tab = reinterpret_cast<unsigned*>(&s.r.part[0][0][0]);
   constexpr int TAB_CAP = (int)(sizeof(s.r.part) / sizeof(unsigned));
   const bool use_tab = p.gC.ngroups * nE <= TAB_CAP;
   if (use_tab)
     for (int i = ctid; i < p.gC.ngroups * nE; i += NWC * 32) tab[i] = down_owners(s, p, NB, i / nE, i % nE);
-  bar_sync(1, NWC * 32);
-  const long long MH = (long long)M * H;
-  const int lo = (int)(MH * blockIdx.x / NB), hi = (int)(MH * (blockIdx.x + 1) / NB);
+  int lo, hi;
+  combine_range(p, NB, lo, hi);
+  r0 = (p.resid && lo + ctid < hi) ? __bfloat162float(p.resid[lo + ctid]) : 0.f;
+  return use_tab;
+}
+
+// After the grid barrier: y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared)
+// in slot order over this CTA's slice; resid += y.  The barrier orders the
+// owner table written by combine_prepare before its reads here.
+TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid, bool use_tab, float r0) {
+  const int K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = p.rp.M * K, nE = s.r.nE;
+  const unsigned* tab = reinterpret_cast<const unsigned*>(&s.r.part[0][0][0]);
+  int lo, hi;
+  combine_range(p, NB, lo, hi);
   for (int i = lo + ctid; i < hi; i += NWC * 32) {
     const int t = i / H, h = i - t * H, grp = h / (gs * 16);
     float v[MAX_K + 1];
@@ -305,25 +325,27 @@ TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid)
     if (p.y) p.y[(size_t)t * H + h] = y;
     if (p.resid) {
       __nv_bfloat16* r = p.resid + (size_t)t * H + h;
-      *r = __float2bfloat16_rn(__bfloat162float(*r) + y);
+      *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
     }
   }
 }
 
 // Grid-wide barrier among the consumer warps of all CTAs (one CTA per SM, all
-// resident).  Bounded: a CTA that waits longer than WAIT_LIMIT_NS records
-// ERR_TIMEOUT_GRID and goes on.
+// resident).  The arrival counter is never reset: launch number gen0 (read at
+// the start, before any CTA of this launch can arrive) is complete when it
+// reaches (gen0 + 1) * NB, which every CTA polls directly; the last arriver
+// also advances the launch counter for the next launch.  Bounded: a CTA that
+// waits longer than WAIT_LIMIT_NS records ERR_TIMEOUT_GRID and goes on.
 TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
   __threadfence();
   bar_sync(1, NWC * 32);
   if (ctid == 0) {
-    if (atomicAdd(p.grid_cnt, 1u) == (unsigned)NB - 1) {
-      *p.grid_cnt = 0u;
-      __threadfence();
+    const unsigned target = (s.gen0 + 1u) * (unsigned)NB;
+    if (atomicAdd(p.grid_cnt, 1u) + 1u == target) {
       atomicAdd(p.grid_gen, 1u);
     } else {
       const unsigned long long t0 = globaltimer();
-      while (ld_acquire_u32(p.grid_gen) == s.gen0) {
+      while ((int)(ld_acquire_u32(p.grid_cnt) - target) < 0) {
         if (globaltimer() - t0 > WAIT_LIMIT_NS) {
           atomicOr(p.err, ERR_TIMEOUT_GRID);
           break;
@@ -496,9 +518,13 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
 }
 
 // Producer: weight stages and activation windows of phase PH in consumer order.
+// Before the first activation window whose data another CTA writes (down:
+// every segment's acts; gate/up: the shared FP16 x when xh_wait) it issues
+// up to NSW weight stages, then waits (bounded) for the data to be published.
 template <int FMT, int PH>
 TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, long long u1, int& wi, int& wph, int& xi,
-                           int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_mine) {
+                           int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_src,
+                           bool xh_wait) {
   constexpr int KC = FMT == 1 ? 64 : 32;
   constexpr int KWC = KW / KC;
   long long u = u0;
@@ -512,7 +538,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
     const __half* brow = nullptr;
     if (lane < sg.nc) {
       if (PH == 0)
-        brow = xh_mine + (size_t)(sg.sh ? lane : s.r.tok[sg.ro + lane]) * p.rp.Hp;
+        brow = xh_src + (size_t)(sg.sh ? lane : s.r.tok[sg.ro + lane]) * p.rp.Hp;
       else
         brow = sg.sh ? p.acts_sh + (size_t)lane * p.Sp : p.acts + (size_t)(sg.ro + lane) * p.Ip;
     }
@@ -520,9 +546,9 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
     int k_issued = sg.c0;  // first chunk whose weight stage is not yet issued
     for (int ws = sg.c0; alive && ws < sg.c1;) {
       const int we = min(sg.c1, (ws / KWC + 1) * KWC);
-      if (PH == 1 && ws == sg.c0) {
-        // down: prefetch weight stages of the first window, then wait until the
-        // expert's acts are complete before fetching them
+      if (PH == 1 ? ws == sg.c0 : xh_wait) {
+        // prefetch weight stages of the first window, then wait until the
+        // expert's acts (down) or the shared x (gate/up) are published
         for (int pre = 0; pre < NSW && k_issued < we && alive; ++pre) {
           const int kk = min(KS, we - k_issued);
           if (lane == 0) {
@@ -541,21 +567,22 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
           k_issued += kk;
         }
         if (lane == 0 && alive) {
-          const unsigned need = (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups);
-          const unsigned* done = p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]);
+          const unsigned need = PH == 1 ? (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups) : (unsigned)p.rp.S;
+          const unsigned* flag = PH == 1 ? p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]) : p.xh_cnt;
           const unsigned long long t0 = globaltimer();
-          while (ld_acquire_u32(done) < need) {
+          while (ld_acquire_u32(flag) < need) {
             if (s.dead) break;
             if (globaltimer() - t0 > WAIT_LIMIT_NS) {
               s.dead = 1;
-              atomicOr(p.err, ERR_TIMEOUT_ACTS);
+              atomicOr(p.err, PH == 1 ? ERR_TIMEOUT_ACTS : ERR_TIMEOUT_XH);
               break;
             }
           }
         }
+        xh_wait = false;
         alive = __shfl_sync(0xffffffffu, alive && !s.dead, 0);
         if (!alive) break;
-        // the acts were written through the generic proxy by other CTAs; the
+        // the data were written through the generic proxy by other CTAs; the
         // bulk copies below read them through the async proxy
         __threadfence();
         fence_proxy_async_global();
@@ -604,10 +631,14 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NB = gridDim.x, b = blockIdx.x;
 
-  // ---- 1. route (every CTA; identical arithmetic to route_kernel)
+  // ---- 1. route.  CTA b < T * S computes router item (tile b / S, slice
+  // b % S) exactly as route_kernel does and publishes it with the slice's |x|
+  // max; every CTA then adds the items in slice order, forms the top-k and the
+  // route list itself.  The CTAs of tile 0 (b < S) also write their slice of
+  // the FP16 x that the gate/up phase reads.
   RouteParams rp = p.rp;
+  rp.logits = nullptr;  // written below by CTA 0 from the summed items
   if (b != 0) {
-    rp.logits = nullptr;
     rp.idx = nullptr;
     rp.w = nullptr;
     rp.shift = nullptr;
@@ -615,9 +646,16 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.routes = nullptr;
     rp.rpos = nullptr;
   }
-  const RouterSplit rsplit(rp.rg, warp);
-  RoutePrefetch pf;
-  route_prefetch(rp, rsplit, lane, pf);
+  const int S = rp.S, nR = rp.rg.tiles * S;
+  const bool rcta = b < nR;
+  const int rj = rcta ? b / S : 0, rcs = rcta ? b % S : 0;
+  // the item's buffers sit in the still idle weight and window rings
+  const SliceSmem L(rp.M, rp.CS, rp.xscale != nullptr);
+  uint8_t* ring = &s.w[0][0];
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring + L.xs);
+  __half* xin = reinterpret_cast<__half*>(ring + L.xin);
+  uint8_t* rt = ring + L.rt;
+  const RouteConst rc = route_const_load(rp, tid);
   if (tid == 0) {
     for (int i = 0; i < NSW; ++i) {
       mbar_init(&s.wfull[i], 1);
@@ -627,32 +665,74 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
       mbar_init(&s.xfull[i], 1);
       mbar_init(&s.xempty[i], NWC);
     }
+    mbar_init(&s.r.xbar, 1);
+    mbar_init(&s.r.rbar, 1);
     fence_barrier_init();
     s.dead = 0;
+    if (rcta) slice_issue_router(rp, s.r, rj, rcs, rt);
   }
   grid_dep_wait();
   grid_dep_launch();
-  if (tid == 0) s.gen0 = ld_acquire_u32(p.grid_gen);
-  __half* xh_mine = p.xh_cta + (size_t)b * p.xh_stride;
-  __half* rin_mine = p.rin_cta ? p.rin_cta + (size_t)b * p.rin_stride : nullptr;
-  route_shift(rp, s.r, warp, lane);
+  if (tid == 0) {
+    if (rcta) slice_issue_x(rp, s.r, rcs, xs);
+    s.gen0 = ld_acquire_u32(p.grid_gen);
+  }
+  route_init_smem(s.r, rc, tid);
   __syncthreads();
-  // the router input is staged in the (still idle) weight and window rings when it fits
-  const bool stage = route_stage_bytes(rp.M, rp.Hp, rp.xscale != nullptr) <= sizeof(s.w) + sizeof(s.x);
-  __half* bs = stage ? reinterpret_cast<__half*>(&s.w[0][0]) : nullptr;
-  route_convert(rp, s.r, xh_mine, rin_mine, bs, tid, NTHREADS);
-  fence_proxy_async_global();  // the producer reads xh_mine with bulk copies
-  __syncthreads();
-  {
-    const __half* bsrc = bs ? bs : (rp.xscale ? rin_mine : xh_mine);
-    const int ld = bs ? route_bs_ld(rp.Hp) : rp.Hp;
+  if (rcta) {
+    mbar_wait(&s.r.xbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+    slice_max(rp, s.r, rcs, xs, warp, lane);
+    __syncthreads();
+    slice_input(rp, s.r, rcs, xs, xin, tid, NTHREADS);
+    __syncthreads();
+    mbar_wait(&s.r.rbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+    float* pub = p.part_pub + (size_t)rcs * rp.M * rp.E;
     if (rp.M > 8)
-      route_gemv<2>(rp, s.r, rsplit, pf, bsrc, ld, warp, lane, tid, NTHREADS);
+      slice_gemv<2>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
     else
-      route_gemv<1>(rp, s.r, rsplit, pf, bsrc, ld, warp, lane, tid, NTHREADS);
+      slice_gemv<1>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
+    if (rj == 0 && tid < rp.M) p.max_pub[rcs * rp.M + tid] = s.r.smax[tid];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) atomicAdd(p.route_cnt, 1u);
+  }
+  // every item published (bounded)
+  if (tid == 0) {
+    const unsigned long long t0 = globaltimer();
+    while (ld_acquire_u32(p.route_cnt) < (unsigned)nR) {
+      if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+        s.dead = 1;
+        atomicOr(p.err, ERR_TIMEOUT_ROUTE);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  // logits: the items added in slice order; shift from the max of the slice maxima
+  for (int i = tid; i < rp.M * rp.E; i += NTHREADS) {
+    float v = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < S; ++c) v += ld_cg(p.part_pub + (size_t)c * rp.M * rp.E + i);
+    s.r.lg[i / rp.E][i % rp.E] = v;
+    if (b == 0 && p.rp.logits) p.rp.logits[i] = v;
+  }
+  if (tid < rp.M) {
+    float m = 0.f;
+    for (int c = 0; c < S; ++c) m = fmaxf(m, ld_cg(p.max_pub + c * rp.M + tid));
+    s.r.shift[tid] = shift_of_max(m);
+    if (rp.shift) rp.shift[tid] = s.r.shift[tid];
+  }
+  __syncthreads();
+  // gate/up B operand: this CTA's slice of x as FP16, published with the count of slices written
+  __half* xh_src = p.xh;
+  const bool xwriter = rcta && rj == 0;
+  if (xwriter) {
+    slice_xh(rp, s.r, rcs, xs, xh_src, tid, NTHREADS);
+    __threadfence();
   }
   route_topk(rp, s.r, warp, lane);
   __syncthreads();
+  if (xwriter && tid == 0) atomicAdd(p.xh_cnt, 1u);
   route_list(rp, s.r, warp, lane, tid, NTHREADS);
   fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
 
@@ -682,8 +762,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     int wuse[NSW], xuse[NSX];
     for (int i = 0; i < NSW; ++i) wuse[i] = 0;
     for (int i = 0; i < NSX; ++i) xuse[i] = 0;
-    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_mine);
-    if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_mine);
+    // gate/up reads x written by the slice CTAs: wait for all S slices
+    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, true);
+    if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, false);
     // Copies still in flight must land before the CTA can exit (only matters
     // when a wait gave up): wait, bounded, for each slot's last issued phase.
     if (lane == 0 && s.dead) {
@@ -724,10 +805,17 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
         consume_seg<FMT, 1, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
     }
   }
+  float r0;
+  const bool use_tab = combine_prepare(s, p, NB, tid, r0);
   grid_barrier(s, p, NB, tid);
-  final_combine(s, p, NB, tid);
-  if (b == 0)
-    for (int e = tid; e <= rp.E; e += NWC * 32) p.entry_done[e] = 0u;  // every readiness wait of this launch is over
+  final_combine(s, p, NB, tid, use_tab, r0);
+  if (b == 0) {  // every readiness wait of this launch is over
+    for (int e = tid; e <= rp.E; e += NWC * 32) p.entry_done[e] = 0u;
+    if (tid == 0) {
+      *p.route_cnt = 0u;
+      *p.xh_cnt = 0u;
+    }
+  }
 }
 
 }  // namespace tsm

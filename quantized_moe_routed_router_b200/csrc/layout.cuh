@@ -63,6 +63,15 @@ inline MatGeom make_geom(int rows_tiles, int kdim, int fmt) {
   return m;
 }
 
+// The router: one tile per group, i.e. tile-major [tile][chunk][544 B], so
+// each 16-expert tile is one contiguous range (one bulk copy).
+inline MatGeom make_router_geom(int num_experts, int kdim) {
+  MatGeom m = make_geom((num_experts + 15) / 16, kdim, 0);
+  m.gs = 1;
+  m.ngroups = m.tiles;
+  return m;
+}
+
 TSM_HD uint64_t group_offset(int gs, int chunks, int grp) { return (uint64_t)grp * gs * chunks * UNIT_BYTES; }
 TSM_HD int group_tiles(int tiles, int gs, int grp) {
   int t = tiles - grp * gs;

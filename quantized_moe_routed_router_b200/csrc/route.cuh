@@ -1,32 +1,43 @@
-// Route kernel: router GEMV -> (bias) -> top-k + weights -> route list.
+// Routing: router GEMV -> (bias) -> top-k + weights -> route list.
 //
-// One CTA does the whole micro-batch.  The router GEMV runs on the tensor
-// cores: the Q8_0 router is repacked at open into the same 16-row MMA
-// fragment layout as the experts (rows past E are zero), x * router_xscale is
-// staged in shared memory as FP16 scaled by a per-token power of two (|x| max
-// lands in [2^13, 2^14); with a non-trivial xscale the product is split into
-// an FP16 hi + lo pair so it stays exact), and the FP32 logits come out of
+// The router GEMV runs on the tensor cores: the Q8_0 router is repacked at
+// open into the 16-row MMA fragment layout of the experts, one 16-expert tile
+// after another (rows past E are zero), and the FP32 logits come out of
 // m16n8k16 MMAs with the block scale folded in per 32-block (llama state page,
 // `router_ones`: the INT8 router kernel scales x[n] per element;
-// `router_logits_f32`: one FP32 row of logits per token).  One warp per token
-// then selects the top K by (selection logit desc, index asc), where the
-// selection logit is l + b when a router bias is present (gpt-oss state page,
-// `router_bias`: added BEFORE the top-k), and forms the weights:
-//   softmax over the selected ("selection reduces to softmax over the
-//   selected", `per_expert_ones`), or the full softmax over all experts taken
-//   at the selected indices without renormalisation (deepseek2 layer sketch),
+// `router_logits_f32`: one FP32 row of logits per token).
+//
+// The GEMV is cut into items (tile j, slice c): slice c is the K range of
+// chunks [c CS, (c + 1) CS) (32 K per chunk).  An item needs only its slice of
+// x and CS units of the router, so in the fused layer kernel the T * S items
+// go to T * S CTAs, each loading a few KB (one SM takes in roughly 50 GB/s, so
+// the whole x and router in one CTA would cost several microseconds).  Within
+// an item, x * router_xscale is staged in shared memory as FP16 scaled by a
+// power of two per (token, slice) -- the slice's |x| max lands in
+// [2^13, 2^14); with a non-trivial xscale the product is an FP16 hi + lo pair
+// so it stays exact -- and the item's 16 warps' partial sums are added in
+// warp order and unscaled exactly.  A logit is the sum of its S item values
+// in slice order.  route_kernel runs the same items one after another in one
+// CTA, so both kernels produce the same bits.
+//
+// One warp per token then selects the top K by (selection logit desc, index
+// asc), where the selection logit is l + b when a router bias is present
+// (gpt-oss state page, `router_bias`: added BEFORE the top-k), and forms the
+// weights: softmax over the selected ("selection reduces to softmax over the
+// selected", `per_expert_ones`), or the full softmax over all experts taken at
+// the selected indices without renormalisation (deepseek2 layer sketch),
 // times the per-expert scale.  The reference does this part on the host after
 // reading the logits back; here it never leaves the device.
 //
-// The same CTA then groups the M*K (token, slot) pairs by expert into the
-// route list the expert kernels walk: per touched expert its first route and
-// count, routes sorted by (expert, token) -- each expert's weights are then
-// streamed once per micro-batch.  The pages' route list is a host-written
-// 16-byte record per route (gpt-oss state page, `batch_routes`); ours is
-// built on the device.
+// The (token, slot) pairs are then grouped by expert into the route list the
+// expert phases walk: per touched expert its first route and count, routes
+// sorted by (expert, token) -- each expert's weights are then streamed once
+// per micro-batch.  The pages' route list is a host-written 16-byte record
+// per route (gpt-oss state page, `batch_routes`); ours is built on the device.
 //
-// It also writes x as FP16 with the same per-token scale (no xscale), the B
-// operand of the gate/up MMA; that kernel undoes the shift exactly.
+// The gate/up B operand is x as FP16 scaled by a per-token power of two taken
+// from the |x| max over the whole row (the max of the slice maxima); the
+// gate/up epilogue undoes it exactly.
 #pragma once
 #include "common.cuh"
 #include "layout.cuh"
@@ -44,10 +55,14 @@ struct Route {
 enum { META_M = 0, META_NT = 1, META_MK = 2, META_HAS_SHARED = 3, META_NE = 4, META_EX = 8,
        META_RO = META_EX + MAX_ENTRIES, META_NC = META_RO + MAX_ENTRIES, META_INTS = META_NC + MAX_ENTRIES };
 
+constexpr int ROUTE_WARPS = 16;  // warps of a routing CTA; an item's chunks are split over them
+constexpr int MAX_SLICES = 64;   // router slices along K
+
 struct RouteParams {
   const __nv_bfloat16* x;  // [M][H]
   int M, H, Hp, E, K;
-  const uint8_t* rw;       // router, repacked Q8_0 fragment tiles (rows padded to 16)
+  int S, CS;               // router slices: S slices of CS chunks (32 K each), the last may be shorter
+  const uint8_t* rw;       // router, repacked Q8_0 fragment tiles, tile-major (rows padded to 16)
   MatGeom rg;              // its geometry
   const float* xscale;     // [H] or null (null = ones)
   const float* bias;       // [E] or null
@@ -57,8 +72,6 @@ struct RouteParams {
   int* idx;                // [M][K] (optional)
   float* w;                // [M][K] (optional)
   int* shift;              // [M] (optional)
-  __half* xh;              // [M][Hp] x as FP16 * 2^shift
-  __half* rin;             // [2][M][Hp] router input hi/lo (used only with an x-scale)
   int* meta;               // optional global copies of the route list
   Route* routes;           // [M*K]
   int* rpos;               // [M][K] -> position in routes
@@ -68,164 +81,193 @@ struct RouteParams {
   float* logits_out;
 };
 
-TSM_DEV bool topk_better(float v1, int i1, float v2, int i2) { return v1 > v2 || (v1 == v2 && i1 < i2); }
-
-constexpr int ROUTE_WARPS = 16;           // warps that do the router GEMV (tiles are split over them)
-constexpr int ROUTE_PRE = 4;              // router units per warp fetched before x is ready
-
 // Routing results, in the shared memory of the kernel that routes.
 struct RouteState {
   float part[ROUTE_WARPS][16][16];        // per-warp partial logits [row][token]
   float lg[MAX_TOK][MAX_E];               // logits (before bias)
-  int shift[MAX_TOK];                     // per-token power-of-two scale of x
+  int shift[MAX_TOK];                     // per-token power-of-two scale of x (whole row)
+  float smax[MAX_TOK];                    // |x| max of the current slice
+  int sshift[MAX_TOK];                    // its power-of-two scale
+  float gmax[MAX_TOK];                    // running |x| max over the slices (route_kernel)
   int idx[MAX_TOK * MAX_K];               // selected experts, slot order
   float w[MAX_TOK * MAX_K];               // their weights
-  int cnt[MAX_E], off[MAX_E];
+  int off[MAX_E];                         // first route position of each expert
+  int eslot[MAX_E];                       // entry index of each touched expert
   unsigned tmask[MAX_E];                  // tokens that selected each expert (bit t)
+  float bias[MAX_E], pes[MAX_E];          // router bias and per-expert scale (read before the dependency wait)
   int ex[MAX_ENTRIES], ro[MAX_ENTRIES], nc[MAX_ENTRIES];  // touched experts (+ shared entry)
   int tok[MAX_TOK * MAX_K];               // token of each route position
   int rpos[MAX_TOK * MAX_K];              // route position of each (token, slot)
   int rj[MAX_TOK * MAX_K];                // entry index of each route position
   int nT, nE;
+  uint64_t xbar;                          // completion of the bulk copy of an x slice
+  uint64_t rbar;                          // completion of the bulk copy of an item's router units
+  int xdead;                              // set when a wait of the routing gave up
 };
 
-// Router work split: warp w (< ROUTE_WARPS) owns tile w / wpt and every wpt-th chunk of it.
-struct RouterSplit {
-  int T, C, wpt, tile, wsub, nunits;
-  TSM_DEV RouterSplit(const MatGeom& g, int warp) {
-    T = g.tiles;
-    C = g.chunks;
-    wpt = ROUTE_WARPS / T;  // warps per tile (T <= 16)
-    tile = warp / wpt;
-    wsub = warp % wpt;
-    nunits = (warp < ROUTE_WARPS && tile < T) ? (C - wsub + wpt - 1) / wpt : 0;
+// ---------------------------------------------------------------------------- slices
+TSM_HD int slice_lo(int CS, int c) { return c * CS; }
+TSM_HD int slice_hi(int CS, int C, int c) { return (c + 1) * CS < C ? (c + 1) * CS : C; }
+// Row stride (halves) of the FP16 router input: 32 bytes past a multiple of
+// 128 keeps the B-fragment loads conflict-free.
+TSM_HD int slice_ld(int CS) { return round_up(CS * 32, 64) + 16; }
+TSM_HD size_t align128(size_t n) { return (n + 127) & ~(size_t)127; }
+
+// Shared-memory buffers of one item: x slice (BF16, [M][CS*32]), router input
+// (FP16, hi rows then lo rows with an x-scale, slice_ld apart) and the item's
+// CS router units.
+struct SliceSmem {
+  size_t xs, xin, rt, total;
+  TSM_HD SliceSmem(int M, int CS, bool split) {
+    xs = 0;
+    xin = align128((size_t)M * CS * 64);
+    rt = xin + align128((size_t)(split ? 2 : 1) * M * slice_ld(CS) * 2);
+    total = rt + align128((size_t)CS * UNIT_BYTES);
   }
-  TSM_DEV const uint8_t* unit(const RouteParams& p, int k) const {
-    const int ck = wsub + k * wpt;
-    const int grp = tile / p.rg.gs, jt = tile % p.rg.gs, ntg = group_tiles(T, p.rg.gs, grp);
-    return p.rw + group_offset(p.rg.gs, C, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
+};
+
+// Router bias and per-expert scale of expert `tid` (0 and 1 where absent).
+// They are weights, so they are read before the dependency wait.
+struct RouteConst {
+  float b, s;
+};
+TSM_DEV RouteConst route_const_load(const RouteParams& p, int tid) {
+  RouteConst c{0.f, 1.f};
+  if (tid < p.E) {
+    if (p.bias) c.b = p.bias[tid];
+    if (p.pes) c.s = p.pes[tid];
   }
-};
-
-struct RoutePrefetch {
-  uint4 q[ROUTE_PRE];
-  uint32_t sc[ROUTE_PRE];
-};
-
-// The router does not depend on the previous kernel: its first units can be
-// fetched before griddepcontrol.wait.
-TSM_DEV void route_prefetch(const RouteParams& p, const RouterSplit& rs, int lane, RoutePrefetch& pf) {
-#pragma unroll
-  for (int k = 0; k < ROUTE_PRE; ++k)
-    if (k < rs.nunits) {
-      const uint8_t* u = rs.unit(p, k);
-      pf.q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
-      pf.sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
-    }
+  return c;
 }
 
-// Per-token |x| (and |x * xscale|) max -> power-of-two shift (warp t: token t).
-TSM_DEV void route_shift(const RouteParams& p, RouteState& s, int warp, int lane) {
-  if (warp >= p.M) return;
-  const int t = warp;
-  float m = 0.f;
-  constexpr int U = 4;
-  for (int kb = lane * 8; kb < p.H; kb += 32 * 8 * U) {
-    uint4 raw[U];
+// Shared-memory state that must be set before the first CTA barrier: the
+// prefetched constants and the cleared per-expert token masks.
+TSM_DEV void route_init_smem(RouteState& s, const RouteConst& c, int tid) {
+  if (tid < MAX_E) {
+    s.bias[tid] = c.b;
+    s.pes[tid] = c.s;
+    s.tmask[tid] = 0u;
+  }
+}
+
+// Running max of |x| (and |x * xscale|) over the 8 BF16 values of `raw` at column k.
+TSM_DEV float absmax8(const RouteParams& p, const uint4& raw, int k, float m) {
+  const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = kb + u * 256;
-      raw[u] = k < p.H ? *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = kb + u * 256;
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(b2[q]);
-        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-        if (p.xscale && k < p.H) {
-          m = fmaxf(m, fabsf(f.x * p.xscale[k + 2 * q]));
-          m = fmaxf(m, fabsf(f.y * p.xscale[k + 2 * q + 1]));
-        }
-      }
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(b2[q]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    if (p.xscale && k < p.H) {
+      m = fmaxf(m, fabsf(f.x * p.xscale[k + 2 * q]));
+      m = fmaxf(m, fabsf(f.y * p.xscale[k + 2 * q + 1]));
     }
   }
-  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
+// 8 BF16 values of x at column k (zero past H) -> FP16 * 2^shift (hx) and,
+// with an x-scale, x * xscale * 2^shift as an FP16 hi + lo pair (hh, hl).
+TSM_DEV void convert8(const RouteParams& p, const uint4& raw, int k, float sc, bool split, uint4& hx, uint4& hh,
+                      uint4& hl) {
+  const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  __half2* ox = reinterpret_cast<__half2*>(&hx);
+  __half* oh = reinterpret_cast<__half*>(&hh);
+  __half* ol = reinterpret_cast<__half*>(&hl);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(b2[q]);
+    ox[q] = __floats2half2_rn(f.x * sc, f.y * sc);  // each half rounded to nearest, as one conversion each
+    if (split) {
+      const bool in = k + 2 * q < p.H;
+      const float xa = f.x * (in ? p.xscale[k + 2 * q] : 1.f) * sc;
+      const float xb = f.y * (in ? p.xscale[k + 2 * q + 1] : 1.f) * sc;
+      oh[2 * q] = __float2half_rn(xa);
+      oh[2 * q + 1] = __float2half_rn(xb);
+      ol[2 * q] = __float2half_rn(xa - __half2float(oh[2 * q]));
+      ol[2 * q + 1] = __float2half_rn(xb - __half2float(oh[2 * q + 1]));
+    }
+  }
+}
+
+// One thread: bulk copies of the M rows of x slice c into xs ([M][CS*32]
+// BF16), completing on s.xbar.  x is 16-byte aligned and H a multiple of 32,
+// so every source starts on a 64-byte boundary.
+TSM_DEV void slice_issue_x(const RouteParams& p, RouteState& s, int c, __nv_bfloat16* xs) {
+  const int lo = slice_lo(p.CS, c), hi = slice_hi(p.CS, p.rg.chunks, c);
+  const unsigned row = (unsigned)(hi - lo) * 64u;
+  mbar_arrive_expect_tx(&s.xbar, row * (unsigned)p.M);
+  for (int t = 0; t < p.M; ++t)
+    bulk_g2s(xs + (size_t)t * p.CS * 32, p.x + (size_t)t * p.H + lo * 32, row, &s.xbar);
+}
+
+// One thread: bulk copy of item (j, c)'s router units (contiguous: the router
+// is tile-major) into rt, completing on s.rbar.  The router is constant, so
+// this may be issued before the dependency wait.
+TSM_DEV void slice_issue_router(const RouteParams& p, RouteState& s, int j, int c, uint8_t* rt) {
+  const int lo = slice_lo(p.CS, c), hi = slice_hi(p.CS, p.rg.chunks, c);
+  const unsigned bytes = (unsigned)(hi - lo) * UNIT_BYTES;
+  mbar_arrive_expect_tx(&s.rbar, bytes);
+  bulk_g2s(rt, p.rw + ((size_t)j * p.rg.chunks + lo) * UNIT_BYTES, bytes, &s.rbar);
+}
+
+// Power-of-two scale that puts |x| max m in [2^13, 2^14) (0 for m = 0 or not finite).
+TSM_DEV int shift_of_max(float m) {
   int sh = 0;
   if (m > 0.f && m <= 3.4e38f) {
     int e2;
     frexpf(m, &e2);  // m in [2^(e2-1), 2^e2)
     sh = min(126, max(-126, 14 - e2));
   }
+  return sh;
+}
+
+TSM_DEV float pow2f(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// Per-token |x| max of slice c (warp t: token t) -> s.smax, s.sshift.
+TSM_DEV void slice_max(const RouteParams& p, RouteState& s, int c, const __nv_bfloat16* xs, int warp, int lane) {
+  if (warp >= p.M) return;
+  const int t = warp, lo = slice_lo(p.CS, c), n = (slice_hi(p.CS, p.rg.chunks, c) - lo) * 32;
+  const __nv_bfloat16* row = xs + (size_t)t * p.CS * 32;
+  float m = 0.f;
+  for (int k = lane * 8; k < n; k += 256) m = absmax8(p, *reinterpret_cast<const uint4*>(row + k), lo * 32 + k, m);
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) {
-    s.shift[t] = sh;
-    if (p.shift) p.shift[t] = sh;
+    s.smax[t] = m;
+    s.sshift[t] = shift_of_max(m);
   }
 }
 
-// Row stride (halves) of the router input staged in shared memory: 32 bytes
-// past a multiple of 128 keeps the B-fragment loads conflict-free.
-TSM_DEV int route_bs_ld(int Hp) { return Hp + 16; }
-
-// x -> FP16 * 2^shift into xh [M][Hp] (zero padded).  The router input (the
-// same values, or with an x-scale x * xscale * 2^shift as an FP16 hi + lo
-// pair) also goes to `bs` (rows route_bs_ld(Hp) halves apart; hi rows 0..M-1,
-// lo rows M..2M-1) when bs is not null, else to `rin` [2][M][Hp].
-TSM_DEV void route_convert(const RouteParams& p, const RouteState& s, __half* xh, __half* rin, __half* bs, int tid,
-                           int nthr) {
-  constexpr int U = 4;
-  const int per_row = p.Hp / 8, total = p.M * per_row, bld = route_bs_ld(p.Hp);
+// Router input of slice c: x (* xscale) * 2^sshift[t] as FP16 (hi, and lo in
+// rows M..2M-1 with an x-scale), rows slice_ld(CS) halves apart.
+TSM_DEV void slice_input(const RouteParams& p, const RouteState& s, int c, const __nv_bfloat16* xs, __half* xin,
+                         int tid, int nthr) {
+  const int lo = slice_lo(p.CS, c), per_row = (slice_hi(p.CS, p.rg.chunks, c) - lo) * 4, ld = slice_ld(p.CS);
   const bool split = p.xscale != nullptr;
-  for (int base = tid; base < total; base += nthr * U) {
-    uint4 raw[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + u * nthr;
-      raw[u] = make_uint4(0, 0, 0, 0);
-      if (i < total) {
-        const int t = i / per_row, k = (i - t * per_row) * 8;
-        if (k < p.H) raw[u] = *reinterpret_cast<const uint4*>(p.x + (size_t)t * p.H + k);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + u * nthr;
-      if (i >= total) break;
-      const int t = i / per_row, k = (i - t * per_row) * 8;
-      const float sc = __uint_as_float((uint32_t)(s.shift[t] + 127) << 23);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
-      __half hx[8], hh[8], hl[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(b2[q]);
-        hx[2 * q] = __float2half_rn(f.x * sc);
-        hx[2 * q + 1] = __float2half_rn(f.y * sc);
-        if (split) {
-          const bool in = k + 2 * q < p.H;
-          const float xa = f.x * (in ? p.xscale[k + 2 * q] : 1.f) * sc;
-          const float xb = f.y * (in ? p.xscale[k + 2 * q + 1] : 1.f) * sc;
-          hh[2 * q] = __float2half_rn(xa);
-          hh[2 * q + 1] = __float2half_rn(xb);
-          hl[2 * q] = __float2half_rn(xa - __half2float(hh[2 * q]));
-          hl[2 * q + 1] = __float2half_rn(xb - __half2float(hh[2 * q + 1]));
-        }
-      }
-      *reinterpret_cast<uint4*>(xh + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hx);
-      if (bs) {
-        *reinterpret_cast<uint4*>(bs + (size_t)t * bld + k) = *reinterpret_cast<uint4*>(split ? hh : hx);
-        if (split) *reinterpret_cast<uint4*>(bs + (size_t)(p.M + t) * bld + k) = *reinterpret_cast<uint4*>(hl);
-      } else if (split) {
-        *reinterpret_cast<uint4*>(rin + (size_t)t * p.Hp + k) = *reinterpret_cast<uint4*>(hh);
-        *reinterpret_cast<uint4*>(rin + (size_t)(p.M + t) * p.Hp + k) = *reinterpret_cast<uint4*>(hl);
-      }
-    }
+  for (int i = tid; i < p.M * per_row; i += nthr) {
+    const int t = i / per_row, k = (i - t * per_row) * 8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(xs + (size_t)t * p.CS * 32 + k);
+    uint4 hx, hh, hl;
+    convert8(p, raw, lo * 32 + k, pow2f(s.sshift[t]), split, hx, hh, hl);
+    *reinterpret_cast<uint4*>(xin + (size_t)t * ld + k) = split ? hh : hx;
+    if (split) *reinterpret_cast<uint4*>(xin + (size_t)(p.M + t) * ld + k) = hl;
   }
 }
 
-// One Q8_0 (tile, chunk) unit of the router against x rows in global memory
-// (b points at column 32 * chunk of row 0, rows `ld` halves apart): acc += W x.
+// x slice c -> FP16 * 2^shift[t] (whole-row scale) into xh [M][Hp].
+TSM_DEV void slice_xh(const RouteParams& p, const RouteState& s, int c, const __nv_bfloat16* xs, __half* xh,
+                      int tid, int nthr) {
+  const int lo = slice_lo(p.CS, c), per_row = (slice_hi(p.CS, p.rg.chunks, c) - lo) * 4;
+  for (int i = tid; i < p.M * per_row; i += nthr) {
+    const int t = i / per_row, k = (i - t * per_row) * 8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(xs + (size_t)t * p.CS * 32 + k);
+    uint4 hx, hh, hl;
+    convert8(p, raw, lo * 32 + k, pow2f(s.shift[t]), false, hx, hh, hl);
+    *reinterpret_cast<uint4*>(xh + (size_t)t * p.Hp + lo * 32 + k) = hx;
+  }
+}
+
+// One Q8_0 (tile, chunk) unit of the router against the FP16 router input
+// (b points at the chunk's column 0 of row 0, rows `ld` halves apart): acc += W x.
 template <int NT>
 TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const __half* b, int ld, int M, int lane) {
   const int g = lane >> 2, c = lane & 3;
@@ -250,128 +292,124 @@ TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const __half
   }
 }
 
-// Router GEMV of all tokens -> s.lg (bias not applied).  bsrc: router input
-// rows `ld` halves apart (lo rows follow the M hi rows with an x-scale), in
-// shared or global memory.  Needs a barrier of the whole CTA after
-// route_convert; ends with one.
+// Item (tile j, slice c): the slice's router units (at `units`, shared or
+// global memory: unit of local chunk q at units + q * UNIT_BYTES) against the
+// router input xin.  Warp w takes local chunks w, w + ROUTE_WARPS, ...; the
+// warps' partial sums are added in warp order and multiplied by
+// 2^-sshift[t].  The value of (token t, expert e = 16 j + r) goes to
+// pub[t * E + e] when pub is not null, else is added to s.lg[t][e].  Needs a
+// CTA barrier after slice_input; ends with one.
 template <int NT>
-TSM_DEV void route_gemv(const RouteParams& p, RouteState& s, const RouterSplit& rs, const RoutePrefetch& pf,
-                        const __half* bsrc, int ld, int warp, int lane, int tid, int nthr) {
+TSM_DEV void slice_gemv(const RouteParams& p, RouteState& s, int j, int c, const __half* xin, const uint8_t* units,
+                        int warp, int lane, int tid, int nthr, float* pub) {
   float acc[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const bool split = p.xscale != nullptr;
-  // units past the prefetched ones: ROUTE_PRE at a time, the next batch in flight while one is used
-  RoutePrefetch nb;
-  auto fetch = [&](RoutePrefetch& f, int k0) {
-#pragma unroll
-    for (int k = 0; k < ROUTE_PRE; ++k)
-      if (k0 + k < rs.nunits) {
-        const uint8_t* u = rs.unit(p, k0 + k);
-        f.q[k] = *reinterpret_cast<const uint4*>(u + lane * 16);
-        f.sc[k] = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
-      }
-  };
-  for (int half = 0; half < (split ? 2 : 1); ++half) {
-    const __half* b = bsrc + (size_t)half * p.M * ld;
-    if (ROUTE_PRE < rs.nunits) fetch(nb, ROUTE_PRE);
-#pragma unroll
-    for (int k = 0; k < ROUTE_PRE; ++k)
-      if (k < rs.nunits) router_unit<NT>(acc, pf.q[k], pf.sc[k], b + (rs.wsub + k * rs.wpt) * 32, ld, p.M, lane);
-    for (int kb = ROUTE_PRE; kb < rs.nunits; kb += ROUTE_PRE) {
-      RoutePrefetch cur = nb;
-      if (kb + ROUTE_PRE < rs.nunits) fetch(nb, kb + ROUTE_PRE);
-#pragma unroll
-      for (int k = 0; k < ROUTE_PRE; ++k)
-        if (kb + k < rs.nunits)
-          router_unit<NT>(acc, cur.q[k], cur.sc[k], b + (rs.wsub + (kb + k) * rs.wpt) * 32, ld, p.M, lane);
-    }
-  }
+  const int nck = slice_hi(p.CS, p.rg.chunks, c) - slice_lo(p.CS, c), ld = slice_ld(p.CS);
+  const int halves = p.xscale ? 2 : 1;
   if (warp < ROUTE_WARPS) {
-    const int gq = lane >> 2, c = lane & 3;
+#pragma unroll 2
+    for (int q = warp; q < nck; q += ROUTE_WARPS) {
+      const uint8_t* u = units + (size_t)q * UNIT_BYTES;
+      const uint4 qw = *reinterpret_cast<const uint4*>(u + lane * 16);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(u + QUANT_BYTES + (lane >> 2) * 4);
+      for (int h = 0; h < halves; ++h)
+        router_unit<NT>(acc, qw, sc, xin + (size_t)h * p.M * ld + q * 32, ld, p.M, lane);
+    }
+    const int gq = lane >> 2, cq = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      s.part[warp][gq][nt * 8 + 2 * c] = acc[nt][0];
-      s.part[warp][gq][nt * 8 + 2 * c + 1] = acc[nt][1];
-      s.part[warp][gq + 8][nt * 8 + 2 * c] = acc[nt][2];
-      s.part[warp][gq + 8][nt * 8 + 2 * c + 1] = acc[nt][3];
+      s.part[warp][gq][nt * 8 + 2 * cq] = acc[nt][0];
+      s.part[warp][gq][nt * 8 + 2 * cq + 1] = acc[nt][1];
+      s.part[warp][gq + 8][nt * 8 + 2 * cq] = acc[nt][2];
+      s.part[warp][gq + 8][nt * 8 + 2 * cq + 1] = acc[nt][3];
     }
   }
   __syncthreads();
-  // logits[t][e] = sum over the tile's warps in order, times 2^-shift[t]
-  for (int i = tid; i < p.M * p.E; i += nthr) {
-    const int t = i / p.E, e = i - t * p.E;
-    const int tl = e >> 4, r = e & 15;
+  for (int i = tid; i < p.M * 16; i += nthr) {
+    const int t = i >> 4, r = i & 15, e = j * 16 + r;
+    if (e >= p.E) continue;
     float v = 0.f;
-    for (int w = 0; w < rs.wpt; ++w) v += s.part[tl * rs.wpt + w][r][t];
-    s.lg[t][e] = v * __uint_as_float((uint32_t)(127 - s.shift[t]) << 23);
+#pragma unroll
+    for (int w = 0; w < ROUTE_WARPS; ++w) v += s.part[w][r][t];
+    v *= pow2f(-s.sshift[t]);
+    if (pub)
+      pub[(size_t)t * p.E + e] = v;
+    else
+      s.lg[t][e] += v;
   }
   __syncthreads();
 }
 
-// Top-k and weights: warp t handles token t (lane holds experts lane, lane+32, ...).
-TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane) {
+// Order-preserving map of an FP32 value to an unsigned key (larger value,
+// larger key; -0 and +0 share a key); NaN maps to 0, below every number.
+TSM_DEV unsigned order_key(float f) {
+  if (f != f) return 0u;
+  const unsigned u = __float_as_uint(f + 0.f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+TSM_DEV float key_value(unsigned k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k); }
+
+// Top-k and weights: warp t handles token t (lane holds experts lane,
+// lane + 32, ...; PER = ceil(E / 32)).  The selection order is (selection
+// logit desc, expert index asc): each step takes the largest key over the
+// warp, then the smallest index holding it.  Each selected (token, expert)
+// also sets the token's bit in the expert's token mask.
+template <int PER>
+TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lane) {
   if (warp >= p.M) return;
   const int t = warp;
-  constexpr int PER = MAX_E / 32;
-  float vsel[PER], vsc[PER];
-  unsigned taken = 0;
+  const bool biased = p.bias && p.bias_mode != 0;
+  const bool score_biased = p.bias && p.bias_mode == 1;
+  unsigned key[PER];
+  float vsc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     const float l = e < p.E ? s.lg[t][e] : -INFINITY;
-    const float ls = (e < p.E && p.bias && p.bias_mode != 0) ? l + p.bias[e] : l;
-    vsel[i] = ls;
-    vsc[i] = (p.bias_mode == 1 && p.bias) ? ls : l;
+    const float ls = (e < p.E && biased) ? l + s.bias[e] : l;
+    key[i] = e < p.E ? order_key(ls) : 0u;
+    vsc[i] = score_biased ? ls : l;
     if (e < p.E) {
       if (p.logits) p.logits[(size_t)t * p.E + e] = l;
       if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
     }
   }
-  int selk = 0;  // lane k holds the k-th selected expert and its score logit
-  float sck = -INFINITY;
+  int selk = 0;  // lane k: the k-th selected expert
   for (int k = 0; k < p.K; ++k) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    unsigned bk = 0u;
+    int be = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = lane + 32 * i;
-      if (e < p.E && !((taken >> i) & 1u) && topk_better(vsel[i], e, bv, bi)) {
-        bv = vsel[i];
-        bi = e;
+    for (int i = 0; i < PER; ++i)
+      if (key[i] > bk) {  // strict: the lowest index wins among this lane's equal keys
+        bk = key[i];
+        be = lane + 32 * i;
       }
-    }
-    for (int o = 16; o; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (topk_better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi < 0 || bi >= p.E) {  // only with NaN logits
+    const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
+    int bi = (int)__reduce_min_sync(0xffffffffu, bk == kmax && kmax != 0u ? (unsigned)be : 0x7fffffffu);
+    if (kmax == 0u || bi >= p.E) {  // no candidate left: only with NaN logits
       if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
       bi = 0;
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    float mine = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i)
-      if (i == (bi >> 5)) mine = vsc[i];
-    const float sc = __shfl_sync(0xffffffffu, mine, bi & 31);
-    if (lane == k) {
-      selk = bi;
-      sck = sc;
-    }
+      if (lane + 32 * i == bi) key[i] = 0u;
+    if (lane == k) selk = bi;
   }
   const bool act = lane < p.K;
-  float m = act ? sck : -INFINITY;
+  // score logit of the selected expert, recomputed exactly as above
+  float sck = -INFINITY;
+  if (act) {
+    const float l = s.lg[t][selk];
+    sck = score_biased ? l + s.bias[selk] : l;
+  }
+  unsigned mk = act ? order_key(sck) : 0u;
   if (p.score != 0) {
 #pragma unroll
     for (int i = 0; i < PER; ++i)
-      if (lane + 32 * i < p.E) m = fmaxf(m, vsc[i]);
+      if (lane + 32 * i < p.E) mk = max(mk, order_key(vsc[i]));
   }
-  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float m = key_value(__reduce_max_sync(0xffffffffu, mk));
   float den = 0.f;
   if (p.score == 0) {
     den = act ? expf(sck - m) : 0.f;
@@ -382,9 +420,10 @@ TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane)
   }
   for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   if (act) {
-    const float wv = expf(sck - m) / den * (p.pes ? p.pes[selk] : 1.f);
+    const float wv = expf(sck - m) / den * s.pes[selk];
     s.idx[t * p.K + lane] = selk;
     s.w[t * p.K + lane] = wv;
+    atomicOr(&s.tmask[selk], 1u << t);
     if (p.idx) p.idx[t * p.K + lane] = selk;
     if (p.w) p.w[t * p.K + lane] = wv;
     if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
@@ -392,28 +431,33 @@ TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane)
   }
 }
 
+TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane) {
+  if (p.E <= 32)
+    route_topk_t<1>(p, s, warp, lane);
+  else if (p.E <= 64)
+    route_topk_t<2>(p, s, warp, lane);
+  else if (p.E <= 128)
+    route_topk_t<4>(p, s, warp, lane);
+  else
+    route_topk_t<8>(p, s, warp, lane);
+}
+
 // Route list: the (token, slot) pairs grouped by expert (touched experts in
 // ascending order, tokens ascending), plus the shared expert as the last
-// entry with all M tokens.  Needs a CTA barrier after route_topk; ends with one.
+// entry with all M tokens.  A token selects an expert at most once, so the
+// expert's route count is the popcount of its token mask (set by
+// route_topk) and a token's rank among them the popcount of the mask's lower
+// bits.  Needs s.tmask cleared (route_init_smem) and a CTA barrier after
+// route_topk; ends with one.
 TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
-  for (int e = tid; e < p.E; e += nthr) {
-    s.cnt[e] = 0;
-    s.tmask[e] = 0u;
-  }
-  __syncthreads();
   const int MK = p.M * p.K;
-  for (int i = tid; i < MK; i += nthr) {
-    atomicAdd(&s.cnt[s.idx[i]], 1);
-    atomicOr(&s.tmask[s.idx[i]], 1u << (i / p.K));
-  }
-  __syncthreads();
   if (warp == 0) {
     constexpr int PER = MAX_E / 32;
     int cl[PER], tot = 0, nz = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane * PER + i;
-      cl[i] = e < p.E ? s.cnt[e] : 0;
+      cl[i] = e < p.E ? __popc(s.tmask[e]) : 0;
       tot += cl[i];
       nz += cl[i] > 0;
     }
@@ -432,6 +476,7 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
       if (e < p.E) {
         s.off[e] = run;
         if (cl[i]) {
+          s.eslot[e] = slot;
           s.ex[slot] = e;
           s.ro[slot] = run;
           s.nc[slot] = cl[i];
@@ -474,6 +519,7 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
     const int pos = s.off[e] + __popc(s.tmask[e] & ((1u << tk) - 1u));  // tokens before tk that chose e
     s.tok[pos] = tk;
     s.rpos[i] = pos;
+    s.rj[pos] = s.eslot[e];
     if (p.routes) {
       Route r;
       r.token = tk;
@@ -485,40 +531,57 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
     if (p.rpos) p.rpos[i] = pos;
   }
   __syncthreads();
-  // entry index of each route position
-  for (int j = tid; j < s.nT; j += nthr)
-    for (int n = 0; n < s.nc[j]; ++n) s.rj[s.ro[j] + n] = j;
-  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------- standalone route kernel
 constexpr int ROUTE_THREADS = ROUTE_WARPS * 32;
 
-// Shared memory of route_kernel: RouteState, then the staged router input
-// (2 * M rows of route_bs_ld(Hp) halves) when it fits.
-TSM_HD size_t route_stage_bytes(int M, int Hp, bool split) { return (size_t)(split ? 2 : 1) * M * (Hp + 16) * 2; }
-
-__global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RouteParams p, int stage_in_smem) {
+// One CTA: the items (j, c) in slice order, each slice's x staged by bulk copy,
+// router units read from global memory; logits accumulated in slice order.
+// Dynamic shared memory: RouteState, then the slice buffers (SliceSmem).
+__global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RouteParams p) {
   extern __shared__ __align__(128) uint8_t route_smem_raw[];
   RouteState& s = *reinterpret_cast<RouteState*>(route_smem_raw);
-  __half* bs = stage_in_smem ? reinterpret_cast<__half*>(route_smem_raw + ((sizeof(RouteState) + 127) & ~(size_t)127))
-                             : nullptr;
+  uint8_t* sbuf = route_smem_raw + align128(sizeof(RouteState));
+  const SliceSmem L(p.M, p.CS, p.xscale != nullptr);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sbuf + L.xs);
+  __half* xin = reinterpret_cast<__half*>(sbuf + L.xin);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const RouterSplit rs(p.rg, warp);
-  RoutePrefetch pf;
-  route_prefetch(p, rs, lane, pf);
+  const RouteConst rc = route_const_load(p, tid);
+  if (tid == 0) {
+    mbar_init(&s.xbar, 1);
+    fence_barrier_init();
+    s.xdead = 0;
+  }
   grid_dep_wait();
   grid_dep_launch();
-  route_shift(p, s, warp, lane);
+  if (tid == 0) slice_issue_x(p, s, 0, xs);
+  route_init_smem(s, rc, tid);
+  for (int i = tid; i < p.M * MAX_E; i += ROUTE_THREADS) s.lg[i / MAX_E][i % MAX_E] = 0.f;
+  if (tid < MAX_TOK) s.gmax[tid] = 0.f;
   __syncthreads();
-  route_convert(p, s, p.xh, p.rin, bs, tid, ROUTE_THREADS);
+  for (int c = 0; c < p.S; ++c) {
+    mbar_wait(&s.xbar, c & 1, &s.xdead, p.err, ERR_TIMEOUT_XSTAGE);
+    slice_max(p, s, c, xs, warp, lane);
+    __syncthreads();
+    slice_input(p, s, c, xs, xin, tid, ROUTE_THREADS);
+    if (tid < p.M) s.gmax[tid] = fmaxf(s.gmax[tid], s.smax[tid]);
+    fence_proxy_async_smem();  // xs is rewritten by the next slice's bulk copies
+    __syncthreads();
+    if (tid == 0 && c + 1 < p.S) slice_issue_x(p, s, c + 1, xs);
+    for (int j = 0; j < p.rg.tiles; ++j) {
+      const uint8_t* units = p.rw + ((size_t)j * p.rg.chunks + slice_lo(p.CS, c)) * UNIT_BYTES;
+      if (p.M > 8)
+        slice_gemv<2>(p, s, j, c, xin, units, warp, lane, tid, ROUTE_THREADS, nullptr);
+      else
+        slice_gemv<1>(p, s, j, c, xin, units, warp, lane, tid, ROUTE_THREADS, nullptr);
+    }
+  }
+  if (tid < p.M) {
+    s.shift[tid] = shift_of_max(s.gmax[tid]);
+    if (p.shift) p.shift[tid] = s.shift[tid];
+  }
   __syncthreads();
-  const __half* bsrc = bs ? bs : (p.xscale ? p.rin : p.xh);
-  const int ld = bs ? route_bs_ld(p.Hp) : p.Hp;
-  if (p.M > 8)
-    route_gemv<2>(p, s, rs, pf, bsrc, ld, warp, lane, tid, ROUTE_THREADS);
-  else
-    route_gemv<1>(p, s, rs, pf, bsrc, ld, warp, lane, tid, ROUTE_THREADS);
   route_topk(p, s, warp, lane);
   __syncthreads();
   route_list(p, s, warp, lane, tid, ROUTE_THREADS);

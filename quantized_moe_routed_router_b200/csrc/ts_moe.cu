@@ -47,6 +47,7 @@ size_t blob_row_bytes(int fmt, int cols) { return (size_t)(cols / 32) * (fmt == 
 struct ts_moe {
   ts_moe_config cfg{};
   int sm_count = 0, nb = 0;
+  int slices[MAX_TOK + 1] = {};  // router slices per token count
   int Hp = 0, Ip = 0, Sp = 0;
   MatGeom gR{}, gB{}, gC{}, gBs{}, gCs{};
   int ng_max_B = 0;
@@ -64,11 +65,9 @@ struct ts_moe {
   int* shift = nullptr;
   int* meta = nullptr;
   Route* routes = nullptr;
-  __half* xh = nullptr;
-  __half* rin = nullptr;        // route kernel: router input hi/lo (x-scale)
-  __half* xh_cta = nullptr;     // layer kernel: per-CTA x
-  __half* rin_cta = nullptr;
-  size_t xh_stride = 0, rin_stride = 0;
+  __half* xh = nullptr;         // layer kernel: FP16 x, the gate/up B operand
+  float* part_pub = nullptr;    // layer kernel: router items [MAX_SLICES][Mmax][E]
+  float* max_pub = nullptr;     // layer kernel: slice |x| maxima [MAX_SLICES][Mmax]
   __half* acts = nullptr;
   __half* acts_sh = nullptr;
   float* P = nullptr;
@@ -76,7 +75,7 @@ struct ts_moe {
   float* partial1 = nullptr;
   unsigned* entry_done = nullptr;
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group) chunk counters
-  unsigned* grid = nullptr;     // down: grid barrier {arrivals, generation}
+  unsigned* grid = nullptr;     // {grid barrier arrivals, launches, x slices written, router items published}
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
   uint8_t* counters = nullptr;
@@ -158,14 +157,35 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
   return TS_MOE_OK;
 }
 
-// Dynamic shared memory of route_kernel: RouteState, then the staged router
-// input when it fits under ROUTE_SMEM_MAX.
+// Dynamic shared memory of route_kernel: RouteState, then one item's slice buffers.
 constexpr int ROUTE_SMEM_MAX = 220 * 1024;
-size_t route_smem(int M, int Hp, bool split, int* stage) {
-  const size_t base = (sizeof(RouteState) + 127) & ~(size_t)127;
-  const size_t want = base + route_stage_bytes(M, Hp, split);
-  *stage = want <= (size_t)ROUTE_SMEM_MAX;
-  return *stage ? want : base;
+size_t route_smem(const RouteParams& rp) {
+  return align128(sizeof(RouteState)) + SliceSmem(rp.M, rp.CS, rp.xscale != nullptr).total;
+}
+
+// Router slices for M tokens: the count S (CS = ceil(C / S) chunks each) that
+// balances the bytes a routing CTA loads (its x slice and CS router units)
+// against the bytes every CTA reads back (S items of M x E logits), with the
+// T * S routing CTAs within the grid and one item's buffers within the
+// layer kernel's weight and window rings.  Returns 0 when no S fits.
+constexpr size_t RING_BYTES = sizeof(LayerSmem::w) + sizeof(LayerSmem::x);
+int choose_slices(int M, int C, int T, int E, int nb, bool split) {
+  int best = 0;
+  double best_cost = 0.0;
+  const int smax = std::min({C, MAX_SLICES, nb / std::max(T, 1)});
+  for (int S = 1; S <= smax; ++S) {
+    const int CS = (C + S - 1) / S;
+    if ((C + CS - 1) / CS != S) continue;  // S must be the slice count CS gives
+    if (SliceSmem(M, CS, split).total > RING_BYTES) continue;
+    const double load = (double)M * CS * 64 + (double)CS * UNIT_BYTES;
+    const double read = (double)S * M * (E + 1) * 4;
+    const double cost = std::max(load, read);
+    if (best == 0 || cost < best_cost) {
+      best = S;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 template <typename... Args>
@@ -239,7 +259,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   h->Hp = round_up(H, 64);
   h->Ip = round_up(I, 64);
   h->Sp = S ? round_up(S, 64) : 0;
-  h->gR = make_geom((E + 15) / 16, H, TS_FMT_Q8_0);
+  h->gR = make_router_geom(E, H);
   h->gB = make_geom(I / 8, H, fmt);
   h->gC = make_geom(H / 16, I, fmt);
   if (S) {
@@ -254,6 +274,14 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
           h->any_xscale = true;
           break;
         }
+  for (int m = 1; m <= Mx; ++m) {
+    h->slices[m] = choose_slices(m, h->gR.chunks, h->gR.tiles, E, h->nb, h->any_xscale);
+    if (h->slices[m] == 0) {
+      g_open_error = "no router slicing fits these sizes (too many experts for the SM count, or hidden too large)";
+      ts_moe_close(h);
+      return TS_MOE_EUNSUPPORTED;
+    }
+  }
   h->expert_bytes = 2ull * I * blob_row_bytes(fmt, H) + (uint64_t)H * blob_row_bytes(fmt, I);
   h->router_bytes = (uint64_t)E * blob_row_bytes(TS_FMT_Q8_0, H);
   h->shared_bytes = S ? 2ull * S * blob_row_bytes(TS_FMT_Q8_0, H) + (uint64_t)H * blob_row_bytes(TS_FMT_Q8_0, S) : 0;
@@ -317,18 +345,15 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_meta = slot((size_t)META_INTS * 4);
     const size_t o_routes = slot((size_t)Mx * K * sizeof(Route));
     const size_t o_xh = slot((size_t)Mx * h->Hp * 2);
-    const size_t o_rin = slot(h->any_xscale ? (size_t)2 * Mx * h->Hp * 2 : 16);
-    h->xh_stride = (size_t)Mx * h->Hp;
-    h->rin_stride = h->any_xscale ? (size_t)2 * Mx * h->Hp : 0;
-    const size_t o_xhc = slot((size_t)h->nb * h->xh_stride * 2);
-    const size_t o_rinc = slot(h->any_xscale ? (size_t)h->nb * h->rin_stride * 2 : 16);
+    const size_t o_part = slot((size_t)MAX_SLICES * Mx * E * 4);
+    const size_t o_max = slot((size_t)MAX_SLICES * Mx * 4);
     const size_t o_acts = slot((size_t)Mx * K * h->Ip * 2);
     const size_t o_acts_sh = slot((size_t)Mx * std::max(h->Sp, 64) * 2);
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + (E + 1) + 2 + 1;
+    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + (E + 1) + 4 + 1;  // + grid[4] + error word
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -345,9 +370,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->meta = (int*)(h->ws + o_meta);
     h->routes = (Route*)(h->ws + o_routes);
     h->xh = (__half*)(h->ws + o_xh);
-    h->rin = h->any_xscale ? (__half*)(h->ws + o_rin) : nullptr;
-    h->xh_cta = (__half*)(h->ws + o_xhc);
-    h->rin_cta = h->any_xscale ? (__half*)(h->ws + o_rinc) : nullptr;
+    h->part_pub = (float*)(h->ws + o_part);
+    h->max_pub = (float*)(h->ws + o_max);
     h->acts = (__half*)(h->ws + o_acts);
     h->acts_sh = (__half*)(h->ws + o_acts_sh);
     h->P = (float*)(h->ws + o_P);
@@ -358,8 +382,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->counters_bytes = n_cnt * 4;
     h->cnt_gB = cn;
     h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
-    h->grid = h->entry_done + (E + 1);
-    h->err = h->grid + 2;
+    h->grid = h->entry_done + (E + 1);  // grid barrier arrivals, launches, x slices written, router items published
+    h->err = h->grid + 4;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
     if (ce != cudaSuccess) {
@@ -497,8 +521,8 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.idx = h->idx;
   rp.w = h->w;
   rp.shift = h->shift;
-  rp.xh = h->xh;
-  rp.rin = h->rin;
+  rp.CS = (h->gR.chunks + h->slices[M] - 1) / h->slices[M];
+  rp.S = (h->gR.chunks + rp.CS - 1) / rp.CS;
   rp.meta = h->meta;
   rp.routes = h->routes;
   rp.rpos = h->rpos;
@@ -516,9 +540,7 @@ static ts_moe_status check_call(ts_moe* h, int layer, const void* x, int M) {
 }
 
 static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t st) {
-  int stage = 0;
-  const size_t smem = route_smem(rp.M, rp.Hp, rp.xscale != nullptr, &stage);
-  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, smem, st, rp, stage);
+  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, route_smem(rp), st, rp);
   if (e != cudaSuccess) return cuda_fail(h, e, "route_kernel launch");
   return TS_MOE_OK;
 }
@@ -547,10 +569,9 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   LayerParams lp;
   std::memset(&lp, 0, sizeof(lp));
   lp.rp = route_params(h, layer, x, M);
-  lp.xh_cta = h->xh_cta;
-  lp.rin_cta = lp.rp.xscale ? h->rin_cta : nullptr;
-  lp.xh_stride = (int)h->xh_stride;
-  lp.rin_stride = (int)h->rin_stride;
+  lp.xh = h->xh;
+  lp.part_pub = h->part_pub;
+  lp.max_pub = h->max_pub;
   lp.wB = d.wB;
   lp.wB_stride = h->gB.bytes;
   lp.wBs = d.wBs;
@@ -573,6 +594,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   lp.entry_done = h->entry_done;
   lp.grid_cnt = h->grid;
   lp.grid_gen = h->grid + 1;
+  lp.xh_cnt = h->grid + 2;
+  lp.route_cnt = h->grid + 3;
   lp.y = y;
   lp.resid = (__nv_bfloat16*)resid;
   lp.err = h->err;
@@ -600,9 +623,11 @@ ts_moe_status ts_moe_device_status(ts_moe* h, void* stream) {
   TSM_CUDA(h, cudaMemcpy(&err, h->err, 4, cudaMemcpyDeviceToHost));
   if (!err) return TS_MOE_OK;
   TSM_CUDA(h, cudaMemset(h->counters, 0, h->counters_bytes));
-  char buf[160];
+  char buf[384];
   std::snprintf(buf, sizeof buf, "device error word 0x%x (bit0/1: weight-stage wait gave up, bit2/3: activation-window "
-                "wait gave up, bit4: bad index, bit5: bad route metadata)", err);
+                "wait gave up, bit4: bad index, bit5: bad route metadata, bit6: grid barrier wait gave up, bit7: "
+                "wait for an expert's activations gave up, bit8: wait for the staged x gave up, bit9: wait for the "
+                "shared FP16 x gave up, bit10: wait for the router logits gave up)", err);
   return fail(h, TS_MOE_EDEVICE, buf);
 }
 
@@ -686,8 +711,8 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   if (!router || !x || !idx || !w) return fail(nullptr, TS_MOE_EINVAL, "router, x, idx and w must be non-NULL");
   if (((uintptr_t)x & 15) != 0) return fail(nullptr, TS_MOE_EINVAL, "x must be 16-byte aligned");
 
-  // scratch layout: repacked router | xh | logits | idx | w | shift | meta | routes | rpos | error word
-  const MatGeom gR = make_geom((E + 15) / 16, H, TS_FMT_Q8_0);
+  // scratch layout: repacked router | logits | idx | w | shift | meta | routes | rpos | error word
+  const MatGeom gR = make_router_geom(E, H);
   const int Hp = round_up(H, 64);
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -695,7 +720,7 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
     off += align256(n);
     return r;
   };
-  const size_t o_rw = take(gR.bytes), o_xh = take((size_t)M * Hp * 2), o_lg = take((size_t)M * E * 4),
+  const size_t o_rw = take(gR.bytes), o_lg = take((size_t)M * E * 4),
                o_idx = take((size_t)M * K * 4), o_w = take((size_t)M * K * 4), o_sh = take((size_t)M * 4),
                o_meta = take((size_t)META_INTS * 4), o_rt = take((size_t)M * K * sizeof(Route)),
                o_rpos = take((size_t)M * K * 4), o_err = take(8);
@@ -739,7 +764,6 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   rp.idx = (int*)(sc + o_idx);
   rp.w = (float*)(sc + o_w);
   rp.shift = (int*)(sc + o_sh);
-  rp.xh = (__half*)(sc + o_xh);
   rp.meta = (int*)(sc + o_meta);
   rp.routes = (Route*)(sc + o_rt);
   rp.rpos = (int*)(sc + o_rpos);
@@ -747,9 +771,14 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   rp.idx_out = idx;
   rp.w_out = w;
   rp.logits_out = logits;
-  int stage = 0;
-  const size_t rsm = route_smem(M, Hp, false, &stage);
-  e = launch_pdl(route_kernel, 1, ROUTE_THREADS, rsm, s, rp, stage);
+  int nsm = 0;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
+  const int S = choose_slices(M, gR.chunks, gR.tiles, E, std::min(nsm, MAX_NB), false);
+  if (S == 0) return fail(nullptr, TS_MOE_EUNSUPPORTED, "no router slicing fits these sizes");
+  rp.CS = (gR.chunks + S - 1) / S;
+  rp.S = (gR.chunks + rp.CS - 1) / rp.CS;
+  e = launch_pdl(route_kernel, 1, ROUTE_THREADS, route_smem(rp), s, rp);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("route_kernel launch: ") + cudaGetErrorString(e));
   return TS_MOE_OK;
 }
