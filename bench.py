@@ -127,6 +127,33 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+KERNEL_SOURCES = os.path.join(ROOT, "quantized_moe_routed_router_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_kernel_traffic.json")
+
+
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources the layer kernel is built from (csrc/*.cu, *.cuh)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNEL_SOURCES)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            h.update(open(os.path.join(KERNEL_SOURCES, name), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(algo_bytes_per_launch: float):
+    """DRAM bytes (read + write) per layer-kernel launch from the committed ncu
+    capture, scaled from the captured launch to this run's launches by their
+    algorithmic bytes; None when the kernel sources changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    if d.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return round(d["dram_bytes_per_launch"] * algo_bytes_per_launch / d["algorithmic_bytes_per_launch"])
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -264,7 +291,7 @@ def run_ours(args, rank, world, local):
     achieved = bytes_per_launch / (avg_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": f"layer_kernel<{'MXFP4' if shape.expert_fmt else 'Q8_0'}> (route + gate/up + down + combine)",
                 "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(bytes_per_launch),
                 "avg_launch_us": round(avg_ms * 1e3, 2), "algorithmic_bytes_per_launch": int(bytes_per_launch)}
 
     # end to end through host buffers: pinned H2D of x and resid, D2H of the updated resid

@@ -100,7 +100,9 @@ typedef struct {
 typedef struct ts_moe ts_moe;
 
 /* Validates cfg and layers[0 .. num_layers-1] (shapes, enums, finiteness of
- * the bias, E8M0 = 255 and non-finite Q8_0 scales are refused), then on
+ * the bias, E8M0 = 255 and non-finite Q8_0 scales are refused with
+ * TS_MOE_EINVAL; sizes for which the router GEMV cannot be cut into per-CTA
+ * items that fit the SM count and shared memory with TS_MOE_EUNSUPPORTED), then on
  * cfg->device allocates the repacked weight arena and the per-call workspace
  * (sized once for max_tokens) and repacks every layer.  All refusals happen
  * before any device memory exists (deepseek2 state page: errors at open, "not
@@ -133,7 +135,7 @@ ts_moe_status ts_moe_device_status(ts_moe* h, void* stream);
 
 /* Sizes the caller may need: arena bytes, per-expert algorithmic bytes in the
  * input format (gate + up + down), router bytes per layer, shared expert bytes
- * per layer, number of CTAs the expert kernels launch. */
+ * per layer, number of CTAs the layer kernel launches (one per SM). */
 typedef struct {
   uint64_t arena_bytes;
   uint64_t workspace_bytes;

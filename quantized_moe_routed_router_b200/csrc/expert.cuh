@@ -56,8 +56,8 @@ struct LayerParams {
   RouteParams rp;           // routing inputs; its output pointers are written by CTA 0 only
   __half* xh;               // [Mmax][Hp] FP16 x (the gate/up B operand), slice c written by CTA c
   unsigned* xh_cnt;         // slices of xh written (reset at the end of each launch)
-  float* part_pub;          // [S][M][E] router items (tile j's 16 experts of slice c by CTA j * S + c)
-  float* max_pub;           // [S][M] |x| max of each slice
+  float* part_pub;          // [S][M][item_ld(E)] router items (tile j's 16 experts of slice c by CTA j * S + c)
+  float* max_pub;           // [S][MAX_TOK] |x| max of each slice
   unsigned* route_cnt;      // router items published (reset at the end of each launch)
   const uint8_t* wB;        // gate/up: expert e at wB + e * wB_stride
   uint64_t wB_stride;
@@ -173,7 +173,9 @@ TSM_DEV float act_fn(int act, float alpha, float limit, float g, float u) {
 
 // One chunk of K for this warp's tiles: A from the weight stage, B from the
 // activation window (column c of the n8 tile nt is window row nt*8 + c).
-template <int FMT, int NT>
+// FULL: the group has all GS_MAX tiles, so no tile of the warp is skipped and
+// the compiler may interleave the tiles' work freely.
+template <int FMT, int NT, bool FULL = false>
 TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, int warp, const uint8_t* xc,
                        int lane) {
   constexpr int STEPS = FMT == 1 ? 4 : 2;
@@ -190,7 +192,7 @@ TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, i
 #pragma unroll
   for (int r = 0; r < RW; ++r) {
     const int jt = warp * RW + r;
-    if (jt >= ntg) break;
+    if (!FULL && jt >= ntg) break;
     const uint8_t* t = chunk + jt * UNIT_BYTES;
     const uint4 q = *reinterpret_cast<const uint4*>(t + lane * 16);
     const uint32_t sc = *reinterpret_cast<const uint32_t*>(t + QUANT_BYTES + g * 4);
@@ -431,10 +433,16 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
       const int kk = min(KS, we - k);
       mbar_wait(&s.wfull[wi], wph, &s.dead, p.err, ERR_TIMEOUT_WFULL);
       const uint8_t* st = s.w[wi];
+      if (kk == KS && sg.ntg == GS_MAX) {  // whole stage of a whole group: no guards
 #pragma unroll
-      for (int q = 0; q < KS; ++q)
-        if (q < kk)
-          mma_chunk<FMT, NT>(acc, st + q * sg.ntg * UNIT_BYTES, sg.ntg, warp, xw + (k + q - ws) * KC * 2, lane);
+        for (int q = 0; q < KS; ++q)
+          mma_chunk<FMT, NT, true>(acc, st + q * GS_MAX * UNIT_BYTES, GS_MAX, warp, xw + (k + q - ws) * KC * 2, lane);
+      } else {
+#pragma unroll
+        for (int q = 0; q < KS; ++q)
+          if (q < kk)
+            mma_chunk<FMT, NT>(acc, st + q * sg.ntg * UNIT_BYTES, sg.ntg, warp, xw + (k + q - ws) * KC * 2, lane);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.wempty[wi]);
       if (++wi == NSW) {
@@ -520,7 +528,8 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
 // Producer: weight stages and activation windows of phase PH in consumer order.
 // Before the first activation window whose data another CTA writes (down:
 // every segment's acts; gate/up: the shared FP16 x when xh_wait) it issues
-// up to NSW weight stages, then waits (bounded) for the data to be published.
+// weight stages (down: up to NSW, as the acts may take long; gate/up: one, as
+// x is soon ready), then waits (bounded) for the data to be published.
 template <int FMT, int PH>
 TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, long long u1, int& wi, int& wph, int& xi,
                            int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_src,
@@ -549,7 +558,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
       if (PH == 1 ? ws == sg.c0 : xh_wait) {
         // prefetch weight stages of the first window, then wait until the
         // expert's acts (down) or the shared x (gate/up) are published
-        for (int pre = 0; pre < NSW && k_issued < we && alive; ++pre) {
+        for (int pre = 0; pre < (PH == 1 ? NSW : 1) && k_issued < we && alive; ++pre) {
           const int kk = min(KS, we - k_issued);
           if (lane == 0) {
             alive = mbar_wait(&s.wempty[wi], wph ^ 1, &s.dead, p.err, ERR_TIMEOUT_WEMPTY);
@@ -652,6 +661,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // the item's buffers sit in the still idle weight and window rings
   const SliceSmem L(rp.M, rp.CS, rp.xscale != nullptr);
   uint8_t* ring = &s.w[0][0];
+  constexpr size_t ring_bytes = sizeof(s.w) + sizeof(s.x);  // w and x are adjacent
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring + L.xs);
   __half* xin = reinterpret_cast<__half*>(ring + L.xin);
   uint8_t* rt = ring + L.rt;
@@ -667,6 +677,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     }
     mbar_init(&s.r.xbar, 1);
     mbar_init(&s.r.rbar, 1);
+    mbar_init(&s.r.pbar, 1);
     fence_barrier_init();
     s.dead = 0;
     if (rcta) slice_issue_router(rp, s.r, rj, rcs, rt);
@@ -686,17 +697,24 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     slice_input(rp, s.r, rcs, xs, xin, tid, NTHREADS);
     __syncthreads();
     mbar_wait(&s.r.rbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
-    float* pub = p.part_pub + (size_t)rcs * rp.M * rp.E;
+    float* pub = p.part_pub + (size_t)rcs * rp.M * item_ld(rp.E);
     if (rp.M > 8)
       slice_gemv<2>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
     else
       slice_gemv<1>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
-    if (rj == 0 && tid < rp.M) p.max_pub[rcs * rp.M + tid] = s.r.smax[tid];
+    if (rj == 0 && tid < rp.M) p.max_pub[rcs * MAX_TOK + tid] = s.r.smax[tid];
     __threadfence();
     __syncthreads();
     if (tid == 0) atomicAdd(p.route_cnt, 1u);
   }
-  // every item published (bounded)
+  // every item published (bounded); then the S items and slice maxima are
+  // brought in by two bulk copies when they fit past the item buffers
+  const int ild = item_ld(rp.E);
+  const unsigned ibytes = (unsigned)((size_t)S * rp.M * ild * 4), mbytes = (unsigned)S * MAX_TOK * 4;
+  const size_t pst = align128(L.total);
+  const bool bulk_items = pst + ibytes + mbytes <= ring_bytes;
+  const float* items = bulk_items ? reinterpret_cast<const float*>(ring + pst) : p.part_pub;
+  const float* maxes = bulk_items ? reinterpret_cast<const float*>(ring + pst + ibytes) : p.max_pub;
   if (tid == 0) {
     const unsigned long long t0 = globaltimer();
     while (ld_acquire_u32(p.route_cnt) < (unsigned)nR) {
@@ -706,19 +724,33 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
         break;
       }
     }
+    if (bulk_items && !s.dead) {  // (no copy left in flight when the wait gave up)
+      fence_proxy_async_global();  // written by other CTAs' generic stores, read by bulk copies
+      mbar_arrive_expect_tx(&s.r.pbar, ibytes + mbytes);
+      bulk_g2s(ring + pst, p.part_pub, ibytes, &s.r.pbar);
+      bulk_g2s(ring + pst + ibytes, p.max_pub, mbytes, &s.r.pbar);
+    }
   }
   __syncthreads();
+  if (bulk_items) mbar_wait(&s.r.pbar, 0, &s.dead, p.err, ERR_TIMEOUT_ROUTE);
   // logits: the items added in slice order; shift from the max of the slice maxima
   for (int i = tid; i < rp.M * rp.E; i += NTHREADS) {
+    const int t = i / rp.E, e = i - t * rp.E;
     float v = 0.f;
 #pragma unroll 8
-    for (int c = 0; c < S; ++c) v += ld_cg(p.part_pub + (size_t)c * rp.M * rp.E + i);
-    s.r.lg[i / rp.E][i % rp.E] = v;
+    for (int c = 0; c < S; ++c) {
+      const float* src = items + ((size_t)c * rp.M + t) * ild + e;
+      v += bulk_items ? *src : ld_cg(src);
+    }
+    s.r.lg[t][e] = v;
     if (b == 0 && p.rp.logits) p.rp.logits[i] = v;
   }
   if (tid < rp.M) {
     float m = 0.f;
-    for (int c = 0; c < S; ++c) m = fmaxf(m, ld_cg(p.max_pub + c * rp.M + tid));
+    for (int c = 0; c < S; ++c) {
+      const float* src = maxes + c * MAX_TOK + tid;
+      m = fmaxf(m, bulk_items ? *src : ld_cg(src));
+    }
     s.r.shift[tid] = shift_of_max(m);
     if (rp.shift) rp.shift[tid] = s.r.shift[tid];
   }

@@ -102,6 +102,7 @@ struct RouteState {
   int nT, nE;
   uint64_t xbar;                          // completion of the bulk copy of an x slice
   uint64_t rbar;                          // completion of the bulk copy of an item's router units
+  uint64_t pbar;                          // completion of the bulk copy of the published items
   int xdead;                              // set when a wait of the routing gave up
 };
 
@@ -112,6 +113,9 @@ TSM_HD int slice_hi(int CS, int C, int c) { return (c + 1) * CS < C ? (c + 1) * 
 // 128 keeps the B-fragment loads conflict-free.
 TSM_HD int slice_ld(int CS) { return round_up(CS * 32, 64) + 16; }
 TSM_HD size_t align128(size_t n) { return (n + 127) & ~(size_t)127; }
+// Row stride (floats) of a published item [M][.]: a multiple of 4, so an
+// item block is whole 16-byte units (one bulk copy).
+TSM_HD int item_ld(int E) { return (E + 3) & ~3; }
 
 // Shared-memory buffers of one item: x slice (BF16, [M][CS*32]), router input
 // (FP16, hi rows then lo rows with an x-scale, slice_ld apart) and the item's
@@ -297,8 +301,8 @@ TSM_DEV void router_unit(float (&acc)[NT][4], uint4 q, uint32_t sc, const __half
 // router input xin.  Warp w takes local chunks w, w + ROUTE_WARPS, ...; the
 // warps' partial sums are added in warp order and multiplied by
 // 2^-sshift[t].  The value of (token t, expert e = 16 j + r) goes to
-// pub[t * E + e] when pub is not null, else is added to s.lg[t][e].  Needs a
-// CTA barrier after slice_input; ends with one.
+// pub[t * item_ld(E) + e] when pub is not null, else is added to s.lg[t][e].
+// Needs a CTA barrier after slice_input; ends with one.
 template <int NT>
 TSM_DEV void slice_gemv(const RouteParams& p, RouteState& s, int j, int c, const __half* xin, const uint8_t* units,
                         int warp, int lane, int tid, int nthr, float* pub) {
@@ -334,7 +338,7 @@ TSM_DEV void slice_gemv(const RouteParams& p, RouteState& s, int j, int c, const
     for (int w = 0; w < ROUTE_WARPS; ++w) v += s.part[w][r][t];
     v *= pow2f(-s.sshift[t]);
     if (pub)
-      pub[(size_t)t * p.E + e] = v;
+      pub[(size_t)t * item_ld(p.E) + e] = v;
     else
       s.lg[t][e] += v;
   }

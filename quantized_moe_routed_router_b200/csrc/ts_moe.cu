@@ -66,8 +66,8 @@ struct ts_moe {
   int* meta = nullptr;
   Route* routes = nullptr;
   __half* xh = nullptr;         // layer kernel: FP16 x, the gate/up B operand
-  float* part_pub = nullptr;    // layer kernel: router items [MAX_SLICES][Mmax][E]
-  float* max_pub = nullptr;     // layer kernel: slice |x| maxima [MAX_SLICES][Mmax]
+  float* part_pub = nullptr;    // layer kernel: router items [MAX_SLICES][Mmax][item_ld(E)]
+  float* max_pub = nullptr;     // layer kernel: slice |x| maxima [MAX_SLICES][MAX_TOK]
   __half* acts = nullptr;
   __half* acts_sh = nullptr;
   float* P = nullptr;
@@ -178,7 +178,7 @@ int choose_slices(int M, int C, int T, int E, int nb, bool split) {
     if ((C + CS - 1) / CS != S) continue;  // S must be the slice count CS gives
     if (SliceSmem(M, CS, split).total > RING_BYTES) continue;
     const double load = (double)M * CS * 64 + (double)CS * UNIT_BYTES;
-    const double read = (double)S * M * (E + 1) * 4;
+    const double read = (double)S * (M * item_ld(E) + MAX_TOK) * 4;
     const double cost = std::max(load, read);
     if (best == 0 || cost < best_cost) {
       best = S;
@@ -345,8 +345,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_meta = slot((size_t)META_INTS * 4);
     const size_t o_routes = slot((size_t)Mx * K * sizeof(Route));
     const size_t o_xh = slot((size_t)Mx * h->Hp * 2);
-    const size_t o_part = slot((size_t)MAX_SLICES * Mx * E * 4);
-    const size_t o_max = slot((size_t)MAX_SLICES * Mx * 4);
+    const size_t o_part = slot((size_t)MAX_SLICES * Mx * item_ld(E) * 4);
+    const size_t o_max = slot((size_t)MAX_SLICES * MAX_TOK * 4);
     const size_t o_acts = slot((size_t)Mx * K * h->Ip * 2);
     const size_t o_acts_sh = slot((size_t)Mx * std::max(h->Sp, 64) * 2);
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
