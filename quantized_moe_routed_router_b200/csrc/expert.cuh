@@ -339,9 +339,9 @@ TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid,
 // also advances the launch counter for the next launch.  Bounded: a CTA that
 // waits longer than WAIT_LIMIT_NS records ERR_TIMEOUT_GRID and goes on.
 TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
-  __threadfence();
-  bar_sync(1, NWC * 32);
+  bar_sync(1, NWC * 32);  // orders every consumer's stores before thread 0's gpu-scope fence
   if (ctid == 0) {
+    __threadfence();
     const unsigned target = (s.gen0 + 1u) * (unsigned)NB;
     if (atomicAdd(p.grid_cnt, 1u) + 1u == target) {
       atomicAdd(p.grid_gen, 1u);
@@ -359,11 +359,16 @@ TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int 
   __threadfence();
 }
 
-// A finished gate/up group: every consumer's acts are written; count it for its entry.
-TSM_DEV void entry_group_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int ctid) {
-  __threadfence();
+// A finished gate/up group: count it for its entry once every consumer's
+// acts are written.  The CTA-wide barrier orders all consumers' stores before
+// one thread's gpu-scope fence (cumulative) and increment; that thread's warp
+// rotates with the group so no warp always pays for the fence.
+TSM_DEV void entry_group_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int warp, int lane) {
   bar_sync(1, NWC * 32);
-  if (ctid == 0) atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
+  if (warp == (sg.j * 7 + sg.grp) % NWC && lane == 0) {
+    __threadfence();
+    atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
+  }
 }
 
 // Group epilogue with complete sums in acc.
@@ -391,7 +396,7 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
           }
         }
     }
-    entry_group_done(p, sg, s, ctid);
+    entry_group_done(p, sg, s, warp, lane);
   } else {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
@@ -484,11 +489,12 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
     }
   }
   if (PH == 1) return;  // down partials are combined after the grid barrier
-  // gate/up: the last contributor of the group finishes it
-  __threadfence();
+  // gate/up: the last contributor of the group finishes it.  The barrier
+  // orders every consumer's partial stores before thread 0's gpu-scope fence.
   bar_sync(1, NWC * 32);
   const int key = (sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp;
   if (ctid == 0) {
+    __threadfence();
     const unsigned inc = (unsigned)(sg.c1 - sg.c0);
     s.flag = (atomicAdd(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks);
   }
