@@ -72,9 +72,9 @@ struct LayerParams {
   float* P;                 // [M*K + M][H] down outputs of whole segments
   float* partial0;          // [NB][2][SLOT_FLOATS] gate/up partial slots
   float* partial1;          // [NB][2][SLOT_FLOATS] down partial slots
-  unsigned* cnt_group;      // [(E+1) * ng_max] gate/up chunk counters
+  unsigned* cnt_group;      // [(E+1) * ng_max * NWC] gate/up chunk counters per (entry, group, consumer warp)
   int ng_max;
-  unsigned* entry_done;     // [E+1] gate/up groups finished per expert (+ shared)
+  unsigned* entry_done;     // [E+1] gate/up (group, consumer warp) shares finished per expert (+ shared)
   unsigned* grid_cnt;       // grid barrier arrivals, never reset: NB per launch
   unsigned* grid_gen;       // launches completed (the last arriver of each grid barrier adds 1)
   float* y;                 // [M][H] or null
@@ -94,7 +94,6 @@ struct __align__(128) LayerSmem {
   unsigned rs0[MAX_NB + 1];          // first unit of each CTA's range, per phase
   unsigned rs1[MAX_NB + 1];
   int dead;
-  int flag;
   unsigned gen0;
 };
 
@@ -259,11 +258,19 @@ TSM_DEV float down_value(const LayerSmem& s, const LayerParams& p, unsigned owne
   const unsigned g0 = (unsigned)grp * (unsigned)s.cpre1[s.r.nE] + (unsigned)s.cpre1[j];
   const int rel = h - grp * gs * 16;
   const int off = ((rel >> 4) * 16 + (rel & 15)) * 16 + n;
+  // the contributors' slots in CTA order, four loads in flight at a time
   float v = 0.f;
-  for (int b2 = bf; b2 <= bl; ++b2) {
-    if (s.rs1[b2] == s.rs1[b2 + 1]) continue;  // empty range
-    const int slot = s.rs1[b2] >= g0 ? 0 : 1;
-    v += ld_cg(p.partial1 + ((size_t)b2 * 2 + slot) * SLOT_FLOATS + off);
+  for (int b2 = bf; b2 <= bl; b2 += 4) {
+    float t[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int bb = b2 + q;
+      t[q] = 0.f;  // past bl or an empty range: adds nothing
+      if (bb <= bl && s.rs1[bb] != s.rs1[bb + 1])
+        t[q] = ld_cg(p.partial1 + ((size_t)bb * 2 + (s.rs1[bb] >= g0 ? 0 : 1)) * SLOT_FLOATS + off);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v += t[q];
   }
   return v;
 }
@@ -300,35 +307,78 @@ TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid,
   const unsigned* tab = reinterpret_cast<const unsigned*>(&s.r.part[0][0][0]);
   int lo, hi;
   combine_range(p, NB, lo, hi);
-  for (int i = lo + ctid; i < hi; i += NWC * 32) {
-    const int t = i / H, h = i - t * H, grp = h / (gs * 16);
-    float v[MAX_K + 1];
+  const int KP = K + (p.rp.has_shared ? 1 : 0);
+  if ((hi - lo) * KP > 2 * NWC * 32) {
+    // many outputs: one thread per output, its K (+1) values loaded together
+    for (int i = lo + ctid; i < hi; i += NWC * 32) {
+      const int t = i / H, h = i - t * H, grp = h / (gs * 16);
+      float v[MAX_K + 1];
 #pragma unroll
-    for (int k = 0; k < MAX_K; ++k) {
-      v[k] = 0.f;
+      for (int k = 0; k < MAX_K; ++k) {
+        v[k] = 0.f;
+        if (k < K) {
+          const int pos = s.r.rpos[t * K + k];
+          const int j = s.r.rj[pos];
+          const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
+          v[k] = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
+        }
+      }
+      v[MAX_K] = 0.f;
+      if (p.rp.has_shared) {
+        const int j = s.r.nT;
+        const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
+        v[MAX_K] = down_value(s, p, own, grp, gs, j, t, h, MK + t);
+      }
+      float y = 0.f;
+#pragma unroll
+      for (int k = 0; k < MAX_K; ++k)
+        if (k < K) y = fmaf(s.r.w[t * K + k], v[k], y);
+      y += v[MAX_K];
+      if (p.y) p.y[(size_t)t * H + h] = y;
+      if (p.resid) {
+        __nv_bfloat16* r = p.resid + (size_t)t * H + h;
+        *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
+      }
+    }
+    return;
+  }
+  // few outputs (small M): two passes, so the loads of all (output, slot)
+  // pairs are in flight together: (1) each pair's down value -- the K slots,
+  // then the shared expert -- into the idle weight ring; (2) each output sums
+  // its values in slot order (the same operations as above).
+  float* vbuf = reinterpret_cast<float*>(&s.w[0][0]);
+  const int cap = (int)((sizeof(s.w) + sizeof(s.x)) / sizeof(float)) / KP;  // outputs per batch
+  for (int base = lo; base < hi; base += cap) {
+    const int nb = min(cap, hi - base);
+    for (int q = ctid; q < nb * KP; q += NWC * 32) {
+      const int o = q / KP, k = q - o * KP, i = base + o;
+      const int t = i / H, h = i - t * H, grp = h / (gs * 16);
+      float v;
       if (k < K) {
         const int pos = s.r.rpos[t * K + k];
         const int j = s.r.rj[pos];
         const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-        v[k] = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
+        v = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
+      } else {
+        const int j = s.r.nT;
+        const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
+        v = down_value(s, p, own, grp, gs, j, t, h, MK + t);
+      }
+      vbuf[q] = v;
+    }
+    bar_sync(1, NWC * 32);
+    for (int o = ctid; o < nb; o += NWC * 32) {
+      const int i = base + o, t = i / H, h = i - t * H;
+      float y = 0.f;
+      for (int k = 0; k < K; ++k) y = fmaf(s.r.w[t * K + k], vbuf[o * KP + k], y);
+      if (p.rp.has_shared) y += vbuf[o * KP + K];
+      if (p.y) p.y[(size_t)t * H + h] = y;
+      if (p.resid) {
+        __nv_bfloat16* r = p.resid + (size_t)t * H + h;
+        *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
       }
     }
-    v[MAX_K] = 0.f;
-    if (p.rp.has_shared) {
-      const int j = s.r.nT;
-      const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-      v[MAX_K] = down_value(s, p, own, grp, gs, j, t, h, MK + t);
-    }
-    float y = 0.f;
-#pragma unroll
-    for (int k = 0; k < MAX_K; ++k)
-      if (k < K) y = fmaf(s.r.w[t * K + k], v[k], y);
-    y += v[MAX_K];
-    if (p.y) p.y[(size_t)t * H + h] = y;
-    if (p.resid) {
-      __nv_bfloat16* r = p.resid + (size_t)t * H + h;
-      *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
-    }
+    bar_sync(1, NWC * 32);  // vbuf is rewritten by the next batch
   }
 }
 
@@ -359,13 +409,13 @@ TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int 
   __threadfence();
 }
 
-// A finished gate/up group: count it for its entry once every consumer's
-// acts are written.  The CTA-wide barrier orders all consumers' stores before
-// one thread's gpu-scope fence (cumulative) and increment; that thread's warp
-// rotates with the group so no warp always pays for the fence.
-TSM_DEV void entry_group_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int warp, int lane) {
-  bar_sync(1, NWC * 32);
-  if (warp == (sg.j * 7 + sg.grp) % NWC && lane == 0) {
+// A warp's share of a finished gate/up group (its tiles' acts written):
+// count it for the entry.  __syncwarp orders the warp's stores before lane
+// 0's gpu-scope fence (cumulative) and increment; an entry is complete when
+// its count reaches ngroups * NWC.
+TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int lane) {
+  __syncwarp();
+  if (lane == 0) {
     __threadfence();
     atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
   }
@@ -396,7 +446,7 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
           }
         }
     }
-    entry_group_done(p, sg, s, warp, lane);
+    entry_warp_done(p, sg, s, lane);
   } else {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
@@ -489,45 +539,58 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
     }
   }
   if (PH == 1) return;  // down partials are combined after the grid barrier
-  // gate/up: the last contributor of the group finishes it.  The barrier
-  // orders every consumer's partial stores before thread 0's gpu-scope fence.
-  bar_sync(1, NWC * 32);
-  const int key = (sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp;
-  if (ctid == 0) {
+  // gate/up: per warp (its own tiles), the last contributing CTA finishes the
+  // group.  __syncwarp orders the warp's partial stores before lane 0's
+  // gpu-scope fence and chunk count; no other warp of the CTA waits.
+  const unsigned key = ((unsigned)(sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp) * NWC + warp;
+  __syncwarp();
+  unsigned last = 0;
+  if (lane == 0) {
     __threadfence();
     const unsigned inc = (unsigned)(sg.c1 - sg.c0);
-    s.flag = (atomicAdd(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks);
+    last = atomicAdd(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks;
   }
-  bar_sync(1, NWC * 32);
-  if (!s.flag) return;
-  __threadfence();
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
+  __threadfence();  // the other contributors' slots, published before their counts
 #pragma unroll
   for (int r = 0; r < RW; ++r)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[r][nt][0] = acc[r][nt][1] = acc[r][nt][2] = acc[r][nt][3] = 0.f;
   const int bf = owner_tab(rs, NB, (unsigned)sg.g0);
   const int bl = owner_tab(rs, NB, (unsigned)(sg.g0 + sg.chunks - 1));
-  for (int b2 = bf; b2 <= bl; ++b2) {
-    if (rs[b2] == rs[b2 + 1]) continue;  // empty range
-    const int slot = rs[b2] >= (unsigned)sg.g0 ? 0 : 1;
-    const float* sp = slots + ((size_t)b2 * 2 + slot) * SLOT_FLOATS;
+  // the contributors' slots in CTA order, two CTAs' loads in flight at a time
+  for (int b2 = bf; b2 <= bl; b2 += 2) {
+    float2 v[2][RW][NT][2];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
-      const int jt = warp * RW + r;
-      if (jt >= sg.ntg) break;
+    for (int q = 0; q < 2; ++q) {
+      const int bb = b2 + q;
+      const bool use = bb <= bl && rs[bb] != rs[bb + 1];  // past bl or an empty range: adds nothing
+      const float* sp = slots + ((size_t)bb * 2 + (use && rs[bb] < (unsigned)sg.g0 ? 1 : 0)) * SLOT_FLOATS;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int col = nt * 8 + 2 * c;
-        const float2 v0 = ld_cg2(sp + (jt * 16 + g) * 16 + col);
-        const float2 v1 = ld_cg2(sp + (jt * 16 + g + 8) * 16 + col);
-        acc[r][nt][0] += v0.x;
-        acc[r][nt][1] += v0.y;
-        acc[r][nt][2] += v1.x;
-        acc[r][nt][3] += v1.y;
+      for (int r = 0; r < RW; ++r) {
+        const int jt = warp * RW + r;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int col = nt * 8 + 2 * c;
+          const bool ld = use && jt < sg.ntg;
+          v[q][r][nt][0] = ld ? ld_cg2(sp + (jt * 16 + g) * 16 + col) : make_float2(0.f, 0.f);
+          v[q][r][nt][1] = ld ? ld_cg2(sp + (jt * 16 + g + 8) * 16 + col) : make_float2(0.f, 0.f);
+        }
       }
     }
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[r][nt][0] += v[q][r][nt][0].x;
+          acc[r][nt][1] += v[q][r][nt][0].y;
+          acc[r][nt][2] += v[q][r][nt][1].x;
+          acc[r][nt][3] += v[q][r][nt][1].y;
+        }
   }
-  if (ctid == 0) p.cnt_group[key] = 0u;
+  if (lane == 0) p.cnt_group[key] = 0u;
   group_epilogue<PH, NT>(s, p, sg, acc, warp, lane, ctid);
 }
 
@@ -582,7 +645,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
           k_issued += kk;
         }
         if (lane == 0 && alive) {
-          const unsigned need = PH == 1 ? (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups) : (unsigned)p.rp.S;
+          const unsigned need = PH == 1 ? (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups) * NWC : (unsigned)p.rp.S;
           const unsigned* flag = PH == 1 ? p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]) : p.xh_cnt;
           const unsigned long long t0 = globaltimer();
           while (ld_acquire_u32(flag) < need) {

@@ -74,7 +74,7 @@ struct ts_moe {
   float* partial0 = nullptr;
   float* partial1 = nullptr;
   unsigned* entry_done = nullptr;
-  unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group) chunk counters
+  unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group, consumer warp) chunk counters
   unsigned* grid = nullptr;     // {grid barrier arrivals, launches, x slices written, router items published}
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
@@ -353,7 +353,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B + (E + 1) + 4 + 1;  // + grid[4] + error word
+    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + 4 + 1;  // + grid[4] + error word
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -381,7 +381,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
     h->cnt_gB = cn;
-    h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B;
+    h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B * NWC;
     h->grid = h->entry_done + (E + 1);  // grid barrier arrivals, launches, x slices written, router items published
     h->err = h->grid + 4;
     // zeros: counters, error word, and the padding columns of x / acts
