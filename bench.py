@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--M", type=int, default=16)
     ap.add_argument("--cfg", type=int, default=5)
     ap.add_argument("--layers", type=int, default=0, help="override the number of layers (0 = the workload's)")
-    ap.add_argument("--sweep", action="store_true", help="also time M in {1,2,4,8,16} (extra key m_sweep)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip timing M in {1,2,4,8,16} (key m_sweep)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -199,7 +199,7 @@ def run_ours(args, rank, world, local):
     if args.layers:
         shape = shape.replace(num_layers=args.layers)
     M = args.M
-    shape = shape.replace(max_tokens=max(M, 16 if args.sweep else M))
+    shape = shape.replace(max_tokens=max(M, 16 if (not args.no_sweep) else M))
     NL, H = shape.num_layers, shape.hidden
     layers = [synth.make_layer(shape, l, device=dev) for l in range(NL)]
     moe = binding.MoE(shape, layers)
@@ -325,7 +325,7 @@ def run_ours(args, rank, world, local):
     d2h = o_h.numel() * 2
 
     sweep = None
-    if args.sweep:
+    if (not args.no_sweep):
         sweep = {}
         for Ms in (1, 2, 4, 8, 16):
             o2 = rs.clone()

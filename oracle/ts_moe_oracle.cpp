@@ -16,7 +16,7 @@
 //   3. selection logits l'[e] = l[e] + b[e] (FP32 add) when a router bias is
 //      present; the bias is added BEFORE top-k          [gpt-oss state:
 //                                                        router_bias]
-//   4. S = top-K of l' by (value desc, index asc)
+//   4. S = top-K of l' by (value desc, index asc) (sigmoid scoring: of s + b, below)
 //   5. weights: softmax over the selected experts (SOFTMAX_WEIGHT, norm_w
 //      false: with per-expert ones "selection reduces to softmax over the
 //      selected")                                       [llama / gpt-oss state:
@@ -25,6 +25,14 @@
 //      the selected indices, with no renormalisation  [deepseek2 state, layer
 //                                                      sketch: "softmax(f @
 //                                                      router) top-6, NO renorm"]
+//      or, for sigmoid scoring (the MiniMax flow of the llama state page:
+//      `router_scoring_func` "sigmoid" with an FP32 `e_score_correction_bias`
+//      per expert), scores s[e] = sigmoid(l[e]); the correction bias moves
+//      only the selection, S = top-K of s[e] + b[e]; and the weights are the
+//      selected scores renormalised, w_j = s[S_j] / sum_{i in S} s[i]
+//      (reading: the pages name the rule and the bias but not the weight
+//      formula; this is the plainest one consistent with "the bias only
+//      moves the selection")
 //      then w_j *= per-expert scale (ones when absent)
 //   6. per selected expert j: g = Wg x, u = Wu x, a = act(g, u), y += w_j Wd a
 //      act = SwiGLU silu(g)*u, or the clamped SwiGLU of the gpt-oss family
@@ -208,8 +216,14 @@ void oracle_select(const oracle_cfg* c, const float* bias, const float* pes, con
   for (int m = 0; m < M; ++m) {
     const float* l = logits32 + (size_t)m * E;
     for (int e = 0; e < E; ++e) {
-      ls[e] = (bias && c->bias_mode != 0) ? (float)((double)l[e] + (double)bias[e]) : l[e];
-      sc[e] = (c->bias_mode == 1 && bias) ? (double)ls[e] : (double)l[e];
+      if (c->score == 2) {  // sigmoid scores; the bias only moves the selection
+        const double sg = 1.0 / (1.0 + std::exp(-(double)l[e]));
+        ls[e] = (bias && c->bias_mode != 0) ? (float)(sg + (double)bias[e]) : (float)sg;
+        sc[e] = sg;
+      } else {
+        ls[e] = (bias && c->bias_mode != 0) ? (float)((double)l[e] + (double)bias[e]) : l[e];
+        sc[e] = (c->bias_mode == 1 && bias) ? (double)ls[e] : (double)l[e];
+      }
       if (lsel) lsel[(size_t)m * E + e] = ls[e];
     }
     int* sel = idx + (size_t)m * K;
@@ -224,7 +238,11 @@ void oracle_select(const oracle_cfg* c, const float* bias, const float* pes, con
       for (int j = 0; j < K; ++j) sel[j] = order[j];
     }
     double* wm = w + (size_t)m * K;
-    if (c->score == 0) {
+    if (c->score == 2) {
+      double den = 0.0;
+      for (int j = 0; j < K; ++j) den += sc[sel[j]];
+      for (int j = 0; j < K; ++j) wm[j] = sc[sel[j]] / den;
+    } else if (c->score == 0) {
       double mx = -INFINITY;
       for (int j = 0; j < K; ++j) mx = std::max(mx, sc[sel[j]]);
       double den = 0.0;

@@ -43,6 +43,7 @@ FMT_Q8_0 = 0
 FMT_MXFP4 = 1
 SCORE_SOFTMAX_SELECTED = 0
 SCORE_SOFTMAX_ALL_NORENORM = 1
+SCORE_SIGMOID_RENORM = 2
 BIAS_NONE = 0
 BIAS_LOGITS = 1
 BIAS_SELECT_ONLY = 2

@@ -251,6 +251,53 @@ def test_bias_moves_selection_only_through_biased_logits(mode):
         assert np.array_equal(idx_f, idx) and np.array_equal(w_f, w)
 
 
+def test_sigmoid_scores_two_experts_closed_form():
+    # sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4: slot order by score, weights 3/4 / (5/4) = 0.6 and 0.4
+    shape = _tiny(E=2, K=2, score=2)
+    idx, w, lsel = O.Oracle(shape, _layer_np(shape)).select(np.array([[0.0, math.log(3.0)]], np.float32))
+    assert list(idx[0]) == [1, 0]
+    assert abs(w[0, 0] - 0.6) < 1e-7 and abs(w[0, 1] - 0.4) < 1e-7
+    assert abs(lsel[0, 0] - 0.5) == 0 and abs(lsel[0, 1] - 0.75) < 1e-7
+    shape1 = _tiny(E=2, K=1, score=2)
+    _, w1, _ = O.Oracle(shape1, _layer_np(shape1)).select(np.array([[-2.0, 1.0]], np.float32))
+    assert w1[0, 0] == 1.0
+
+
+def test_sigmoid_scoring_invariants():
+    shape = _tiny(E=8, K=3, score=2)
+    L = _layer_np(shape)
+    rng = np.random.default_rng(21)
+    logits = rng.normal(0, 2, (30, 8)).astype(np.float32)
+    idx, w, _ = O.Oracle(shape, L).select(logits)
+    # sigmoid is increasing: without a bias the set and slot order are those of the logits
+    idx_soft, _, _ = O.Oracle(shape.replace(score=0), L).select(logits)
+    assert np.array_equal(idx, idx_soft)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-15, rtol=0)
+    for m in range(30):
+        s = expit(logits[m, idx[m]].astype(np.float64))
+        assert np.allclose(w[m], s / s.sum(), atol=1e-15, rtol=0)
+    # the correction bias only moves the selection: selection on s + b, weights from s alone
+    b = rng.normal(0, 0.3, 8).astype(np.float32)
+    sb = shape.replace(bias_mode=2)
+    idx_b, w_b, lsel_b = O.Oracle(sb, dict(L, bias=b)).select(logits)
+    for m in range(30):
+        key = (expit(logits[m].astype(np.float64)) + b.astype(np.float64)).astype(np.float32)
+        assert np.array_equal(lsel_b[m], key)
+        assert list(idx_b[m]) == list(BF.topk_bruteforce(key, 3))
+        s = expit(logits[m, idx_b[m]].astype(np.float64))
+        assert np.allclose(w_b[m], s / s.sum(), atol=1e-15, rtol=0)
+    big = np.zeros(8, np.float32)
+    big[6] = 10.0  # beyond any score difference: expert 6 is always selected first
+    idx_g, _, _ = O.Oracle(sb, dict(L, bias=big)).select(logits)
+    assert np.all(idx_g[:, 0] == 6)
+    # K = E: all experts, weights = scores / their sum
+    sE = _tiny(E=6, K=6, score=2)
+    idx_e, w_e, _ = O.Oracle(sE, _layer_np(sE)).select(logits[:, :6])
+    for m in range(30):
+        s = expit(logits[m, :6].astype(np.float64))
+        assert np.allclose(w_e[m], (s / s.sum())[idx_e[m]], atol=1e-15, rtol=0)
+
+
 # --------------------------------------------------------------------------- activations
 
 def test_activation_closed_forms():
