@@ -48,8 +48,16 @@ enum { TS_FMT_Q8_0 = 0, TS_FMT_MXFP4 = 1 };
 /* Top-k rule.  SOFTMAX_SELECTED: softmax over the K selected experts (llama /
  * gpt-oss state pages, `per_expert_ones`: "selection reduces to softmax over the
  * selected").  SOFTMAX_ALL_NORENORM: softmax over all E experts, the K largest
- * kept with no renormalisation (deepseek2 state page, layer sketch). */
-enum { TS_SCORE_SOFTMAX_SELECTED = 0, TS_SCORE_SOFTMAX_ALL_NORENORM = 1 };
+ * kept with no renormalisation (deepseek2 state page, layer sketch).
+ * SIGMOID_RENORM: see below. */
+enum {
+  TS_SCORE_SOFTMAX_SELECTED = 0,     /* softmax over the selected experts (llama / gpt-oss state pages) */
+  TS_SCORE_SOFTMAX_ALL_NORENORM = 1, /* full softmax at the selected indices, no renorm (deepseek2 layer sketch) */
+  TS_SCORE_SIGMOID_RENORM = 2        /* sigmoid scores s = sigmoid(l); S = top-K of s + b (router_bias as the
+                                        correction bias, bias_mode TS_BIAS_NONE or TS_BIAS_SELECT_ONLY);
+                                        w = s over S renormalised to sum 1 (llama state page, MiniMax flow:
+                                        router_scoring_func "sigmoid", e_score_correction_bias) */
+};
 /* Router bias (gpt-oss state page, `router_bias`: added to the logits BEFORE
  * top-k).  LOGITS: selection and weights both use l + b.  SELECT_ONLY: l + b
  * selects, the weights use the unbiased l. */

@@ -25,8 +25,11 @@
 // (gpt-oss state page, `router_bias`: added BEFORE the top-k), and forms the
 // weights: softmax over the selected ("selection reduces to softmax over the
 // selected", `per_expert_ones`), or the full softmax over all experts taken at
-// the selected indices without renormalisation (deepseek2 layer sketch),
-// times the per-expert scale.  The reference does this part on the host after
+// the selected indices without renormalisation (deepseek2 layer sketch), or --
+// with sigmoid scoring (llama state page, MiniMax flow) -- the sigmoid scores
+// s of the selected experts renormalised to sum 1, the selection then being by
+// s + b with the bias as a selection-only correction; times the per-expert
+// scale.  The reference does this part on the host after
 // reading the logits back; here it never leaves the device.
 //
 // The (token, slot) pairs are then grouped by expert into the route list the
@@ -365,13 +368,15 @@ TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lan
   const int t = warp;
   const bool biased = p.bias && p.bias_mode != 0;
   const bool score_biased = p.bias && p.bias_mode == 1;
+  const bool sig = p.score == 2;  // sigmoid scores; the bias is a selection-only correction
   unsigned key[PER];
   float vsc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
     const float l = e < p.E ? s.lg[t][e] : -INFINITY;
-    const float ls = (e < p.E && biased) ? l + s.bias[e] : l;
+    const float base = sig ? 1.f / (1.f + expf(-l)) : l;
+    const float ls = (e < p.E && biased) ? base + s.bias[e] : base;
     key[i] = e < p.E ? order_key(ls) : 0u;
     vsc[i] = score_biased ? ls : l;
     if (e < p.E) {
@@ -401,6 +406,22 @@ TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lan
     if (lane == k) selk = bi;
   }
   const bool act = lane < p.K;
+  if (sig) {  // weights: the selected sigmoid scores renormalised to sum 1
+    const float sk = act ? 1.f / (1.f + expf(-s.lg[t][selk])) : 0.f;
+    float den = sk;
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (act) {
+      const float wv = sk / den * s.pes[selk];
+      s.idx[t * p.K + lane] = selk;
+      s.w[t * p.K + lane] = wv;
+      atomicOr(&s.tmask[selk], 1u << t);
+      if (p.idx) p.idx[t * p.K + lane] = selk;
+      if (p.w) p.w[t * p.K + lane] = wv;
+      if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
+      if (p.w_out) p.w_out[t * p.K + lane] = wv;
+    }
+    return;
+  }
   // score logit of the selected expert, recomputed exactly as above
   float sck = -INFINITY;
   if (act) {

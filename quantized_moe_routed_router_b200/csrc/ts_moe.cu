@@ -122,7 +122,11 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
   if (c->num_layers < 1 || c->num_layers > 1024) return bad("num_layers must be in [1, 1024]");
   if (c->max_tokens < 1 || c->max_tokens > TS_MOE_MAX_TOKENS) return bad("max_tokens must be in [1, 16]");
   if (c->expert_fmt != TS_FMT_Q8_0 && c->expert_fmt != TS_FMT_MXFP4) return bad("unknown expert_fmt");
-  if (c->score != TS_SCORE_SOFTMAX_SELECTED && c->score != TS_SCORE_SOFTMAX_ALL_NORENORM) return bad("unknown score");
+  if (c->score != TS_SCORE_SOFTMAX_SELECTED && c->score != TS_SCORE_SOFTMAX_ALL_NORENORM &&
+      c->score != TS_SCORE_SIGMOID_RENORM)
+    return bad("unknown score");
+  if (c->score == TS_SCORE_SIGMOID_RENORM && c->bias_mode == TS_BIAS_LOGITS)
+    return bad("sigmoid scoring takes its correction bias as TS_BIAS_SELECT_ONLY");
   if (c->bias_mode < TS_BIAS_NONE || c->bias_mode > TS_BIAS_SELECT_ONLY) return bad("unknown bias_mode");
   if (c->act != TS_ACT_SWIGLU && c->act != TS_ACT_SWIGLU_CLAMPED) return bad("unknown act");
   if (c->act == TS_ACT_SWIGLU_CLAMPED &&
@@ -710,7 +714,10 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   if (K < 1 || K > TS_MOE_MAX_TOPK || K > E) return fail(nullptr, TS_MOE_EINVAL, "top_k must be in [1, min(8, E)]");
   if (H <= 0 || H % 32 || H > 16384) return fail(nullptr, TS_MOE_EINVAL, "hidden must be a positive multiple of 32, <= 16384");
   if (M < 0 || M > TS_MOE_MAX_TOKENS) return fail(nullptr, TS_MOE_EINVAL, "M must be in [0, 16]");
-  if (score != TS_SCORE_SOFTMAX_SELECTED && score != TS_SCORE_SOFTMAX_ALL_NORENORM) return fail(nullptr, TS_MOE_EINVAL, "unknown score");
+  if (score != TS_SCORE_SOFTMAX_SELECTED && score != TS_SCORE_SOFTMAX_ALL_NORENORM && score != TS_SCORE_SIGMOID_RENORM)
+    return fail(nullptr, TS_MOE_EINVAL, "unknown score");
+  if (score == TS_SCORE_SIGMOID_RENORM && bias_mode == TS_BIAS_LOGITS)
+    return fail(nullptr, TS_MOE_EINVAL, "sigmoid scoring takes its correction bias as TS_BIAS_SELECT_ONLY");
   if (bias_mode < TS_BIAS_NONE || bias_mode > TS_BIAS_SELECT_ONLY) return fail(nullptr, TS_MOE_EINVAL, "unknown bias_mode");
   if ((bias_mode != TS_BIAS_NONE) != (router_bias != nullptr))
     return fail(nullptr, TS_MOE_EINVAL, "router_bias must be given iff bias_mode != NONE");

@@ -96,6 +96,17 @@ def test_bias_and_shared_consistency(B):
     assert B.validate(ok, _small_layers(ok))[0] == 0
 
 
+def test_sigmoid_scoring_takes_a_selection_only_bias(B):
+    L = _small_layers(SHAPE)
+    for l in L:
+        l.bias = np.zeros(4, np.float32)
+    sig = SHAPE.replace(score=synth.SCORE_SIGMOID_RENORM)
+    st, msg = B.validate(sig.replace(bias_mode=1), L, bias_mode=1, score=2)
+    assert st == 1 and "sigmoid" in msg
+    assert B.validate(sig.replace(bias_mode=2), L, bias_mode=2, score=2)[0] == 0
+    assert B.validate(sig, _small_layers(sig), score=2)[0] == 0
+
+
 def test_open_without_gpu_fails_cleanly(B):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")

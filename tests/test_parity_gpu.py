@@ -25,6 +25,10 @@ SMALL = {
     "e256_k8": S("e256", 128, 64, 256, 8, cfg_id=107),
     "mx_large_k_window_split": S("mxk", 1088, 96, 4, 2, expert_fmt=MX, cfg_id=108),
     "q8_wide_inter": S("q8w", 64, 2080, 3, 2, cfg_id=109),
+    # sigmoid scores with a selection-only correction bias (the MiniMax flow)
+    "q8_sigmoid_correction_bias": S("sig", 256, 128, 16, 4, score=2, bias_mode=2, cfg_id=111),
+    "mx_sigmoid_e256_k8": S("sigmx", 128, 128, 256, 8, expert_fmt=MX, score=2, bias_mode=2, cfg_id=112),
+    "q8_sigmoid_no_bias": S("sig0", 64, 64, 8, 2, score=2, cfg_id=113),
 }
 
 
