@@ -19,7 +19,7 @@ enum : unsigned {
   ERR_TIMEOUT_XEMPTY = 1u << 3,  // producer gave up waiting for a free activation window
   ERR_BAD_INDEX = 1u << 4,       // an expert / token index read from the route list was out of range
   ERR_BAD_META = 1u << 5,        // route metadata inconsistent with the launch
-  ERR_TIMEOUT_GRID = 1u << 6,    // a CTA gave up waiting for the down row groups it combines
+  ERR_TIMEOUT_GRID = 1u << 6,    // a CTA gave up waiting at the grid-wide barrier
   ERR_TIMEOUT_ACTS = 1u << 7,    // a down producer gave up waiting for an expert's acts
   ERR_TIMEOUT_XSTAGE = 1u << 8,  // the routing gave up waiting for the bulk copy of x
   ERR_TIMEOUT_XH = 1u << 9,      // a producer gave up waiting for the shared FP16 x

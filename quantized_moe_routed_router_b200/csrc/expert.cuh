@@ -49,7 +49,6 @@ constexpr int WSTAGE = GS_MAX * KS * UNIT_BYTES;
 constexpr int XWIN = 16 * XROW;
 constexpr int SLOT_FLOATS = GS_MAX * 16 * 16;
 constexpr int MAX_NB = 512;                // CTAs per launch (one per SM)
-constexpr int MAX_ROW_GROUPS = 72;         // down row groups (H / 16 tiles in groups of >= 15)
 static_assert(GS_MAX == NWC * RW, "a group is one tile per consumer-warp slot");
 static_assert(ROUTE_WARPS <= NWC + 1, "routing uses the first ROUTE_WARPS warps");
 
@@ -76,8 +75,8 @@ struct LayerParams {
   unsigned* cnt_group;      // [(E+1) * ng_max * NWC] gate/up chunk counters per (entry, group, consumer warp)
   int ng_max;
   unsigned* entry_done;     // [E+1] gate/up (group, consumer warp) shares finished per expert (+ shared)
-  unsigned* grp_done;       // [gC.ngroups] down (segment, consumer warp) shares finished per row group
-  unsigned* exit_cnt;       // CTAs done; the last one resets every per-launch counter
+  unsigned* grid_cnt;       // grid barrier arrivals, never reset: NB per launch
+  unsigned* grid_gen;       // launches completed (the last arriver of each grid barrier adds 1)
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
   unsigned* err;
@@ -94,8 +93,8 @@ struct __align__(128) LayerSmem {
   int cpre1[MAX_ENTRIES + 1];        // down: first unit of each entry inside a group (group-major)
   unsigned rs0[MAX_NB + 1];          // first unit of each CTA's range, per phase
   unsigned rs1[MAX_NB + 1];
-  unsigned need[MAX_ROW_GROUPS];     // down (segment, warp) shares expected per row group
   int dead;
+  unsigned gen0;
 };
 
 struct Seg {
@@ -292,15 +291,8 @@ TSM_DEV bool combine_prepare(LayerSmem& s, const LayerParams& p, int NB, int cti
   unsigned* tab = reinterpret_cast<unsigned*>(&s.r.part[0][0][0]);
   constexpr int TAB_CAP = (int)(sizeof(s.r.part) / sizeof(unsigned));
   const bool use_tab = p.gC.ngroups * nE <= TAB_CAP;
-  // owners of every (row group, entry) and, per row group, the shares its
-  // contributing CTAs' consumer warps will publish (s.need starts at zero)
-  for (int i = ctid; i < p.gC.ngroups * nE; i += NWC * 32) {
-    const unsigned own = down_owners(s, p, NB, i / nE, i % nE);
-    if (use_tab) tab[i] = own;
-    unsigned cnt = 0;
-    for (int b2 = (int)(own & 0xFFFF); b2 <= (int)(own >> 16); ++b2) cnt += s.rs1[b2] != s.rs1[b2 + 1];
-    if (cnt) atomicAdd(&s.need[i / nE], cnt * NWC);
-  }
+  if (use_tab)
+    for (int i = ctid; i < p.gC.ngroups * nE; i += NWC * 32) tab[i] = down_owners(s, p, NB, i / nE, i % nE);
   int lo, hi;
   combine_range(p, NB, lo, hi);
   r0 = (p.resid && lo + ctid < hi) ? __bfloat162float(p.resid[lo + ctid]) : 0.f;
@@ -390,29 +382,24 @@ TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid,
   }
 }
 
-// Before the combine: wait (bounded) until every down segment of the row
-// groups that this CTA's output slice [lo, hi) touches is published -- each
-// consumer warp of each CTA whose range meets (row group, entry) counts once
-// on the row group's counter.  The expected counts (s.need, from the
-// partition tables in combine_prepare); no CTA waits for row groups it does
-// not read.
-TSM_DEV void wait_rows(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
-  bar_sync(1, NWC * 32);  // s.need complete
+// Grid-wide barrier among the consumer warps of all CTAs (one CTA per SM, all
+// resident).  The arrival counter is never reset: launch number gen0 (read at
+// the start, before any CTA of this launch can arrive) is complete when it
+// reaches (gen0 + 1) * NB, which every CTA polls directly; the last arriver
+// also advances the launch counter for the next launch.  Bounded: a CTA that
+// waits longer than WAIT_LIMIT_NS records ERR_TIMEOUT_GRID and goes on.
+TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
+  bar_sync(1, NWC * 32);  // orders every consumer's stores before thread 0's gpu-scope fence
   if (ctid == 0) {
-    int lo, hi;
-    combine_range(p, NB, lo, hi);
-    const int H = p.rp.H, span = p.gC.gs * 16, ng = p.gC.ngroups;
-    int g0 = 0, g1 = ng - 1;  // a slice across a token boundary may touch every row group
-    if (hi > lo && lo / H == (hi - 1) / H) {
-      g0 = (lo % H) / span;
-      g1 = ((hi - 1) % H) / span;
-    }
-    const unsigned long long t0 = globaltimer();
-    for (int g = g0; g <= g1 && hi > lo; ++g) {
-      while (ld_acquire_u32(p.grp_done + g) < s.need[g]) {
+    __threadfence();
+    const unsigned target = (s.gen0 + 1u) * (unsigned)NB;
+    if (atomicAdd(p.grid_cnt, 1u) + 1u == target) {
+      atomicAdd(p.grid_gen, 1u);
+    } else {
+      const unsigned long long t0 = globaltimer();
+      while ((int)(ld_acquire_u32(p.grid_cnt) - target) < 0) {
         if (globaltimer() - t0 > WAIT_LIMIT_NS) {
           atomicOr(p.err, ERR_TIMEOUT_GRID);
-          g = g1;  // give up on the rest too
           break;
         }
       }
@@ -422,37 +409,16 @@ TSM_DEV void wait_rows(const LayerSmem& s, const LayerParams& p, int NB, int cti
   __threadfence();
 }
 
-// After the combine: the last CTA to finish resets the per-launch counters
-// (every wait of this launch is over by then); the next launch reads them
-// only after its dependency wait, i.e. after this grid has completed.
-TSM_DEV void exit_last_resets(const LayerParams& p, int NB, int ctid) {
-  bar_sync(1, NWC * 32);
-  if (ctid == 0) {
-    __threadfence();
-    if (atomicAdd(p.exit_cnt, 1u) == (unsigned)NB - 1) {
-      __threadfence();
-      for (int e = 0; e <= p.rp.E; ++e) p.entry_done[e] = 0u;
-      for (int g = 0; g < p.gC.ngroups; ++g) p.grp_done[g] = 0u;
-      *p.route_cnt = 0u;
-      *p.xh_cnt = 0u;
-      *p.exit_cnt = 0u;
-    }
-  }
-}
-
 // A warp's share of a finished gate/up group (its tiles' acts written):
 // count it for the entry.  __syncwarp orders the warp's stores before lane
 // 0's gpu-scope fence (cumulative) and increment; an entry is complete when
 // its count reaches ngroups * NWC.
-TSM_DEV void warp_publish(unsigned* counter, int lane) {
+TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int lane) {
   __syncwarp();
   if (lane == 0) {
     __threadfence();
-    atomicAdd(counter, 1u);
+    atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
   }
-}
-TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int lane) {
-  warp_publish(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), lane);
 }
 
 // Group epilogue with complete sums in acc.
@@ -500,7 +466,6 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
           }
         }
     }
-    warp_publish(p.grp_done + sg.grp, lane);
   }
 }
 
@@ -573,10 +538,7 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
       }
     }
   }
-  if (PH == 1) {  // down partials are added up by the combine once the row group is complete
-    warp_publish(p.grp_done + sg.grp, lane);
-    return;
-  }
+  if (PH == 1) return;  // down partials are combined after the grid barrier
   // gate/up: per warp (its own tiles), the last contributing CTA finishes the
   // group.  __syncwarp orders the warp's partial stores before lane 0's
   // gpu-scope fence and chunk count; no other warp of the CTA waits.
@@ -793,9 +755,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   grid_dep_launch();
   if (tid == 0) {
     if (rcta) slice_issue_x(rp, s.r, rcs, xs);
+    s.gen0 = ld_acquire_u32(p.grid_gen);
   }
   route_init_smem(s.r, rc, tid);
-  if (tid < MAX_ROW_GROUPS) s.need[tid] = 0u;
   __syncthreads();
   if (rcta) {
     mbar_wait(&s.r.xbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
@@ -946,9 +908,15 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   }
   float r0;
   const bool use_tab = combine_prepare(s, p, NB, tid, r0);
-  wait_rows(s, p, NB, tid);
+  grid_barrier(s, p, NB, tid);
   final_combine(s, p, NB, tid, use_tab, r0);
-  exit_last_resets(p, NB, tid);
+  if (b == 0) {  // every readiness wait of this launch is over
+    for (int e = tid; e <= rp.E; e += NWC * 32) p.entry_done[e] = 0u;
+    if (tid == 0) {
+      *p.route_cnt = 0u;
+      *p.xh_cnt = 0u;
+    }
+  }
 }
 
 }  // namespace tsm

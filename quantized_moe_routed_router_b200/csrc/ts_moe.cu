@@ -75,8 +75,7 @@ struct ts_moe {
   float* partial1 = nullptr;
   unsigned* entry_done = nullptr;
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group, consumer warp) chunk counters
-  unsigned* grp_done = nullptr; // down: (segment, warp) shares finished per row group
-  unsigned* grid = nullptr;     // {CTAs done, (unused), x slices written, router items published}
+  unsigned* grid = nullptr;     // {grid barrier arrivals, launches, x slices written, router items published}
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
   uint8_t* counters = nullptr;
@@ -267,11 +266,6 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   h->gR = make_router_geom(E, H);
   h->gB = make_geom(I / 8, H, fmt);
   h->gC = make_geom(H / 16, I, fmt);
-  if (h->gC.ngroups > MAX_ROW_GROUPS) {  // cannot happen for hidden <= 16384 (groups of >= 15 tiles)
-    g_open_error = "too many down row groups";
-    ts_moe_close(h);
-    return TS_MOE_EUNSUPPORTED;
-  }
   if (S) {
     h->gBs = make_geom(S / 8, H, TS_FMT_Q8_0);
     h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
@@ -363,7 +357,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + h->gC.ngroups + 4 + 1;  // + grid[4] + error word
+    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + 4 + 1;  // + grid[4] + error word
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -392,8 +386,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->counters_bytes = n_cnt * 4;
     h->cnt_gB = cn;
     h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B * NWC;
-    h->grp_done = h->entry_done + (E + 1);
-    h->grid = h->grp_done + h->gC.ngroups;  // CTAs done, (unused), x slices written, router items published
+    h->grid = h->entry_done + (E + 1);  // grid barrier arrivals, launches, x slices written, router items published
     h->err = h->grid + 4;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
@@ -603,8 +596,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   lp.cnt_group = h->cnt_gB;
   lp.ng_max = h->ng_max_B;
   lp.entry_done = h->entry_done;
-  lp.grp_done = h->grp_done;
-  lp.exit_cnt = h->grid;
+  lp.grid_cnt = h->grid;
+  lp.grid_gen = h->grid + 1;
   lp.xh_cnt = h->grid + 2;
   lp.route_cnt = h->grid + 3;
   lp.y = y;
@@ -636,7 +629,7 @@ ts_moe_status ts_moe_device_status(ts_moe* h, void* stream) {
   TSM_CUDA(h, cudaMemset(h->counters, 0, h->counters_bytes));
   char buf[384];
   std::snprintf(buf, sizeof buf, "device error word 0x%x (bit0/1: weight-stage wait gave up, bit2/3: activation-window "
-                "wait gave up, bit4: bad index, bit5: bad route metadata, bit6: wait for the down row groups gave up, bit7: "
+                "wait gave up, bit4: bad index, bit5: bad route metadata, bit6: grid barrier wait gave up, bit7: "
                 "wait for an expert's activations gave up, bit8: wait for the staged x gave up, bit9: wait for the "
                 "shared FP16 x gave up, bit10: wait for the router logits gave up)", err);
   return fail(h, TS_MOE_EDEVICE, buf);
