@@ -22,6 +22,11 @@ uint64_t ts_moe_debug_range_start(uint64_t U, int NB, int b);
 int ts_moe_debug_owner_of(uint64_t U, int NB, uint64_t u);
 /* Partial-sum slot (0 or 1) CTA b uses for the group whose first unit is g0. */
 int ts_moe_debug_partial_slot(uint64_t U, int NB, int b, uint64_t g0);
+/* Group-aligned gate/up partition (used when ts_moe_debug_use_aligned(G, NB)):
+ * first unit of CTA b (0 <= b <= NB) when G groups of `chunks` units each
+ * are split so that every CTA stays inside one group. */
+uint64_t ts_moe_debug_aligned_start(int G, int NB, int chunks, int b);
+int ts_moe_debug_use_aligned(int G, int NB);
 /* Tiles per group chosen for an expert matrix of `tiles` 16-row tiles. */
 int ts_moe_debug_group_size(int tiles);
 /* The validation ts_moe_open performs before any CUDA call; same status and

@@ -67,6 +67,9 @@ def _load():
     lib.ts_moe_debug_owner_of.argtypes = [C.c_uint64, i32, C.c_uint64]
     lib.ts_moe_debug_partial_slot.argtypes = [C.c_uint64, i32, i32, C.c_uint64]
     lib.ts_moe_debug_group_size.argtypes = [i32]
+    lib.ts_moe_debug_aligned_start.argtypes = [i32, i32, i32, i32]
+    lib.ts_moe_debug_aligned_start.restype = C.c_uint64
+    lib.ts_moe_debug_use_aligned.argtypes = [i32, i32]
     lib.ts_moe_debug_validate.argtypes = [C.POINTER(Config), C.POINTER(LayerWeights)]
     lib.ts_moe_route_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
     for f in ("ts_moe_open", "ts_moe_route", "ts_moe_forward", "ts_moe_device_status", "ts_moe_get_info",

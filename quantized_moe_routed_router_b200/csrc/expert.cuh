@@ -848,13 +848,23 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   __syncthreads();
   const long long U0 = s.upre0[nE];
   const long long U1 = (long long)p.gC.ngroups * s.cpre1[nE];
+  // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
+  const int G0 = nT * p.gB.ngroups + (hs ? p.gBs.ngroups : 0);
+  const bool aligned = use_aligned(G0, NB);
   for (int i = tid; i <= NB; i += NTHREADS) {
-    s.rs0[i] = (unsigned)range_start((uint64_t)U0, NB, i);
+    if (aligned && i < NB) {
+      const int g = aligned_group_of(i, G0, NB);
+      const bool shg = g >= nT * p.gB.ngroups;
+      const int j = shg ? nT : g / p.gB.ngroups, grp = shg ? g - nT * p.gB.ngroups : g % p.gB.ngroups;
+      const int ch = shg ? p.gBs.chunks : p.gB.chunks;
+      s.rs0[i] = (unsigned)(s.upre0[j] + (long long)grp * ch + aligned_offset(i, G0, NB, ch));
+    } else {
+      s.rs0[i] = (unsigned)range_start((uint64_t)U0, NB, i);
+    }
     s.rs1[i] = (unsigned)range_start((uint64_t)U1, NB, i);
   }
   __syncthreads();
   const long long a0 = s.rs0[b], a1 = s.rs0[b + 1], d0 = s.rs1[b], d1 = s.rs1[b + 1];
-  (void)hs;
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp

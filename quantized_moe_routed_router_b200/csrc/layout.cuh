@@ -93,4 +93,20 @@ TSM_HD int owner_of(uint64_t U, int NB, uint64_t u) { return (int)(((u + 1) * (u
 // group is b's first segment (b's range starts inside it), else 1 (its last).
 TSM_HD int partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return range_start(U, NB, b) >= g0 ? 0 : 1; }
 
+// Group-aligned partition, for few groups (G <= NB): CTA i works in group
+// floor(i * G / NB) only, and the CTAs of one group split its chunks evenly,
+// so no CTA carries two partial groups (a CTA that did would finish its second
+// group late and, as its last contributor, also pay for its reduction).
+TSM_HD int aligned_group_of(int i, int G, int NB) { return (int)((long long)i * G / NB); }
+TSM_HD int aligned_first_cta(int g, int G, int NB) { return (int)(((long long)g * NB + G - 1) / G); }
+// First unit of CTA i inside its group of `chunks` units.
+TSM_HD int aligned_offset(int i, int G, int NB, int chunks) {
+  const int g = aligned_group_of(i, G, NB);
+  const int f = aligned_first_cta(g, G, NB), n = aligned_first_cta(g + 1, G, NB) - f;
+  return (int)((long long)chunks * (i - f) / n);
+}
+// Used when the busiest CTA then does at most 10 % more than the mean
+// (G <= NB and NB <= 1.1 * G * floor(NB / G)); otherwise plain contiguous ranges.
+TSM_HD bool use_aligned(int G, int NB) { return G >= 1 && G <= NB && 10LL * NB <= 11LL * G * (NB / G); }
+
 }  // namespace tsm

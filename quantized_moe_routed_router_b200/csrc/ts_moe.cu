@@ -795,6 +795,11 @@ uint64_t ts_moe_debug_range_start(uint64_t U, int NB, int b) { return range_star
 int ts_moe_debug_owner_of(uint64_t U, int NB, uint64_t u) { return owner_of(U, NB, u); }
 int ts_moe_debug_partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return partial_slot(U, NB, b, g0); }
 int ts_moe_debug_group_size(int tiles) { return pick_group_size(tiles); }
+uint64_t ts_moe_debug_aligned_start(int G, int NB, int chunks, int b) {
+  if (b >= NB) return (uint64_t)G * chunks;
+  return (uint64_t)aligned_group_of(b, G, NB) * chunks + aligned_offset(b, G, NB, chunks);
+}
+int ts_moe_debug_use_aligned(int G, int NB) { return use_aligned(G, NB) ? 1 : 0; }
 ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers) {
   return validate(cfg, layers);
 }

@@ -155,6 +155,25 @@ def test_split_groups_use_distinct_slots(B, chunks, ngroups, NB):
             assert sum(min(g1, starts[b + 1]) - max(g0, starts[b]) for b in workers) == chunks
 
 
+@pytest.mark.parametrize("G,NB,chunks", [(48, 148, 45), (49, 148, 45), (37, 148, 45), (4, 148, 90), (1, 148, 45),
+                                          (148, 148, 45), (12, 148, 45), (70, 148, 64), (88, 148, 45)])
+def test_aligned_partition_keeps_each_cta_in_one_group(G, NB, chunks):
+    from quantized_moe_routed_router_b200 import binding as B
+    lib = B.lib
+    starts = [lib.ts_moe_debug_aligned_start(G, NB, chunks, b) for b in range(NB + 1)]
+    assert starts[0] == 0 and starts[-1] == G * chunks
+    assert all(a <= b for a, b in zip(starts, starts[1:]))          # contiguous cover of every unit once
+    for b in range(NB):
+        if starts[b + 1] > starts[b]:
+            assert starts[b] // chunks == (starts[b + 1] - 1) // chunks  # never two groups in one range
+    if lib.ts_moe_debug_use_aligned(G, NB):
+        sizes = [starts[b + 1] - starts[b] for b in range(NB)]
+        assert max(sizes) <= 1.1 * (G * chunks / NB) + 1                # the busiest CTA within 10 %
+    assert lib.ts_moe_debug_use_aligned(48, 148) == 1                   # M = 1, 4 experts x 12 groups
+    assert lib.ts_moe_debug_use_aligned(88, 148) == 0                   # 1.68 CTAs per group: too uneven
+    assert lib.ts_moe_debug_use_aligned(200, 148) == 0                  # more groups than CTAs
+
+
 def test_group_sizes_divide_or_cap():
     from quantized_moe_routed_router_b200 import binding as B
     for tiles in (1, 8, 15, 16, 17, 32, 33, 88, 176, 180, 352, 360, 1792, 97):
