@@ -353,8 +353,10 @@ def run_ours(args, rank, world, local):
             "config": {"workload": f"{shape.name}, {NL} layers x M={M} tokens (independent x per layer)",
                        "hidden": H, "moe_inter": shape.moe_inter, "experts": shape.num_experts,
                        "top_k": shape.top_k, "M": M, "layers": NL, "parallelism": f"replicas x{world}",
-                       "l2": "weights (~10 GB) far exceed the 126 MB L2; no flush needed",
-                       "graph": "CUDA graph of 24 ts_moe_forward calls per step"},
+                       "l2": (f"each step streams {algo_bytes / 1e9:.2f} GB of weights (stack "
+                              f"{NL * (shape.num_experts * shape.expert_bytes() + shape.router_bytes() + shape.shared_bytes()) / 1e9:.1f} GB), "
+                              "far beyond the 126 MB L2; no flush needed"),
+                       "graph": f"CUDA graph of {NL} ts_moe_forward calls per step"},
             "GB_per_s": round(gbs, 1), "frac_of_8TBs": round(gbs / 8000.0, 4),
             "frac_of_measured_hbm": round(gbs / peak, 4),
             "algorithmic_bytes_per_step": int(algo_bytes),

@@ -116,6 +116,12 @@ CONFIGS = {
                 score=SCORE_SOFTMAX_ALL_NORENORM, shared_inter=2816, cfg_id=4),
     5: MoEShape("gpt-oss-20b-shaped-mxfp4-24-layer-stack", 2880, 2880, 32, 4, expert_fmt=FMT_MXFP4,
                 bias_mode=BIAS_LOGITS, act=ACT_SWIGLU_CLAMPED, num_layers=24, cfg_id=5),
+    # beyond the five: the rows that come next on the same kernels
+    # the deepseek2 dense lead layer (dense SwiGLU, width 10944) as E = 1, K = 1, 24 layers (1.7 GB)
+    6: MoEShape("deepseek2-dense-lead-shaped-q8_0-24-layer-stack", 2048, 10944, 1, 1, num_layers=24, cfg_id=6),
+    # sigmoid scoring with a selection-only correction bias (the MiniMax flow), MiniMax-M2-like widths
+    7: MoEShape("minimax-m2-shaped-q8_0-sigmoid-4-layer-stack", 3072, 1536, 256, 8, score=SCORE_SIGMOID_RENORM,
+                bias_mode=BIAS_SELECT_ONLY, num_layers=4, cfg_id=7),
 }
 
 

@@ -147,6 +147,17 @@ def test_workload_full_size(cfg, M):
     assert rep.max_err_y <= 1e-2 * rep.rms_y
 
 
+# dense FFN on the same kernels (E = 1, K = 1, weight 1): the deepseek2 dense lead
+# layer (hidden 2048, dense width 10944, Q8_0) and a Mixtral-width dense FFN
+@pytest.mark.parametrize("name,H,I,fmt", [("dense_lead_ds2", 2048, 10944, Q8), ("dense_mixtral_width", 4096, 14336, Q8),
+                                          ("dense_mx", 2880, 2880, MX)])
+@pytest.mark.parametrize("M", [1, 16])
+def test_dense_ffn(name, H, I, fmt, M):
+    shape = S(name, H, I, 1, 1, expert_fmt=fmt, cfg_id=120 + H % 7 + fmt, max_tokens=16)
+    rep = parity.check_shape(shape, M)
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
 def test_workload_24_layer_stack_sampled():
     """The 24-layer gpt-oss-shaped stack in the launch configuration the
     benchmark times (one handle, all layers resident, M = 16 and M = 1): every
