@@ -139,27 +139,11 @@ TSM_DEV unsigned ld_acquire_u32(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-TSM_DEV void st_release_u32(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-TSM_DEV int ld_cg_i(const int* p) {
-  int v;
-  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
 
 // ----------------------------------------------------------------------------- tensor core MMA (m16n8k16, f16 x f16 -> f32)
 // A fragment (4 regs of f16x2): {row g, k 2c..2c+1}, {row g+8, k 2c..}, {row g, k 2c+8..}, {row g+8, k 2c+8..}
 // B fragment (2 regs): {k 2c..2c+1, col g}, {k 2c+8.., col g};  C/D: {row g, col 2c..2c+1}, {row g+8, col 2c..}
 // with g = lane / 4, c = lane % 4.
-TSM_DEV void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // D = A * B (accumulator input zero).
 TSM_DEV void mma_f16_zc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
