@@ -42,13 +42,22 @@ struct MatGeom {
   uint64_t bytes;  // bytes per expert matrix = tiles * chunks * 544
 };
 
-// Largest tile count per group in [15, 30] that divides `tiles` (equal groups
-// keep the work partition balanced); otherwise 30 with a short last group.
+// Tiles per group: the group is one tile per consumer-warp slot (GS_MAX), so
+// the size in [15, 30] that keeps the most slots busy -- tiles over
+// ceil(tiles / g) * GS_MAX -- wins, ties going to the larger size (whole
+// 30-tile groups take the unguarded MMA path); the last group may be short.
 inline int pick_group_size(int tiles) {
   if (tiles <= GS_MAX) return tiles;
-  for (int g = GS_MAX; g >= GS_MAX / 2; --g)
-    if (tiles % g == 0) return g;
-  return GS_MAX;
+  int best = GS_MAX;
+  long long best_slots = 0;  // slots of the best so far (fewer = more busy)
+  for (int g = GS_MAX; g >= GS_MAX / 2; --g) {
+    const long long slots = (long long)((tiles + g - 1) / g) * GS_MAX;
+    if (best_slots == 0 || slots < best_slots) {
+      best = g;
+      best_slots = slots;
+    }
+  }
+  return best;
 }
 
 inline MatGeom make_geom(int rows_tiles, int kdim, int fmt) {

@@ -174,15 +174,16 @@ def test_aligned_partition_keeps_each_cta_in_one_group(G, NB, chunks):
     assert lib.ts_moe_debug_use_aligned(200, 148) == 0                  # more groups than CTAs
 
 
-def test_group_sizes_divide_or_cap():
+def test_group_sizes_keep_the_most_warp_slots_busy():
     from quantized_moe_routed_router_b200 import binding as B
-    for tiles in (1, 8, 15, 16, 17, 32, 33, 88, 176, 180, 352, 360, 1792, 97):
+    for tiles in (1, 8, 15, 16, 17, 30, 31, 32, 33, 88, 128, 176, 180, 192, 256, 352, 360, 1368, 1792, 97):
         gs = B.lib.ts_moe_debug_group_size(tiles)
-        assert 1 <= gs <= 30
         if tiles <= 30:
             assert gs == tiles
-        elif any(tiles % g == 0 for g in range(15, 31)):
-            assert tiles % gs == 0 and gs >= 15
-            assert not any(tiles % g == 0 for g in range(gs + 1, 31))
-        else:
-            assert gs == 30
+            continue
+        assert 15 <= gs <= 30
+        slots = lambda g: -(-tiles // g) * 30
+        best = min(slots(g) for g in range(15, 31))
+        assert slots(gs) == best                                      # fewest idle consumer-warp slots
+        assert gs == max(g for g in range(15, 31) if slots(g) == best)  # ties: the larger group
+    assert B.lib.ts_moe_debug_group_size(256) == 30 and B.lib.ts_moe_debug_group_size(360) == 30
