@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--M", type=int, default=16)
     ap.add_argument("--cfg", type=int, default=5)
     ap.add_argument("--layers", type=int, default=0, help="override the number of layers (0 = the workload's)")
-    ap.add_argument("--no-sweep", action="store_true", help="skip timing M in {1,2,4,8,16} (key m_sweep)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip timing M in {1,2,4,8,16} (key m_sweep) and the chunked M = 64 (key prefill_chunked)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -129,6 +129,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = os.path.join(ROOT, "quantized_moe_routed_router_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_kernel_traffic.json")
+PREFILL_M = 64  # the chunked-prefill point of the sweep: four 16-token launches per layer
 
 
 def kernel_sources_sha256() -> str:
@@ -199,7 +200,7 @@ def run_ours(args, rank, world, local):
     if args.layers:
         shape = shape.replace(num_layers=args.layers)
     M = args.M
-    shape = shape.replace(max_tokens=max(M, 16 if (not args.no_sweep) else M))
+    shape = shape.replace(max_tokens=max(M, PREFILL_M if (not args.no_sweep) else M))
     NL, H = shape.num_layers, shape.hidden
     layers = [synth.make_layer(shape, l, device=dev) for l in range(NL)]
     moe = binding.MoE(shape, layers)
@@ -211,32 +212,36 @@ def run_ours(args, rank, world, local):
     torch.cuda.empty_cache()
 
     master = 1000 + rank  # each replica draws its own micro-batches
-    xs = torch.stack([synth.make_x(shape, l, 16, device=dev, master=master) for l in range(NL)])  # [NL,16,H]
-    rs = torch.stack([synth.make_x(shape, l, 16, device=dev, master=master, tensor=synth.T_RESID) for l in range(NL)])
+    Mr = max(16, M)
+    xs = torch.stack([synth.make_x(shape, l, Mr, device=dev, master=master) for l in range(NL)])  # [NL,Mr,H]
+    rs = torch.stack([synth.make_x(shape, l, Mr, device=dev, master=master, tensor=synth.T_RESID) for l in range(NL)])
     stream = torch.cuda.Stream(device=dev)
 
-    def touched_bytes(Mx):
+    def touched_bytes(Mx, src=xs):
+        """Weight bytes one step streams: per layer, per launch of up to 16
+        tokens, the touched experts + router (+ shared)."""
         idx = torch.empty(Mx, shape.top_k, dtype=torch.int32, device=dev)
         w = torch.empty(Mx, shape.top_k, device=dev)
-        tot, n_touched = 0, []
+        n_touched = []
         with torch.cuda.stream(stream):
             for l in range(NL):
-                moe.route(l, xs[l, :Mx], idx, w, stream=stream)
+                moe.route(l, src[l, :Mx], idx, w, stream=stream)
                 stream.synchronize()
-                n = len(set(idx.cpu().numpy().ravel().tolist()))
-                n_touched.append(n)
-        per_layer = [n * info.expert_bytes + info.router_bytes + info.shared_bytes for n in n_touched]
-        return sum(per_layer), n_touched, per_layer
+                ih = idx.cpu().numpy()
+                n_touched.append([len(set(ih[c:c + 16].ravel().tolist())) for c in range(0, Mx, 16)])
+        per_layer = [sum(n * info.expert_bytes + info.router_bytes + info.shared_bytes for n in nl)
+                     for nl in n_touched]
+        return sum(per_layer), [n for nl in n_touched for n in nl], per_layer
 
-    def make_graph(Mx, out):
+    def make_graph(Mx, out, src=xs):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             for l in range(NL):  # eager warm-up of every layer once
-                moe.forward(l, xs[l, :Mx], out[l, :Mx], None, stream=stream)
+                moe.forward(l, src[l, :Mx], out[l, :Mx], None, stream=stream)
             stream.synchronize()
             with torch.cuda.graph(g, stream=stream):
                 for l in range(NL):
-                    moe.forward(l, xs[l, :Mx], out[l, :Mx], None, stream=stream)
+                    moe.forward(l, src[l, :Mx], out[l, :Mx], None, stream=stream)
         return g
 
     def time_graph(g, steps, warmup, sampler=None):
@@ -324,7 +329,7 @@ def run_ours(args, rank, world, local):
     h2d = x_h.numel() * 2 + r_h.numel() * 2
     d2h = o_h.numel() * 2
 
-    sweep = None
+    sweep = prefill = None
     if (not args.no_sweep):
         sweep = {}
         for Ms in (1, 2, 4, 8, 16):
@@ -337,6 +342,18 @@ def run_ours(args, rank, world, local):
                               "frac_of_8TBs": round(b2 / (ms2 * 1e-3) / 8e12, 4),
                               "touched_experts_per_layer": round(sum(nt2) / len(nt2), 2)}
             del g2
+        # chunked prefill: M = 64 tokens per layer run as four 16-token launches
+        xp = torch.stack([synth.make_x(shape, l, PREFILL_M, device=dev, master=master) for l in range(NL)])
+        op = torch.stack([synth.make_x(shape, l, PREFILL_M, device=dev, master=master, tensor=synth.T_RESID)
+                          for l in range(NL)])
+        gp = make_graph(PREFILL_M, op, xp)
+        bp, ntp, _ = touched_bytes(PREFILL_M, xp)
+        msp, _ = time_graph(gp, max(20, args.steps // 2), args.warmup)
+        prefill = {"M": PREFILL_M, "launches_per_layer": (PREFILL_M + 15) // 16,
+                   "tokens_per_s": round(world * PREFILL_M / (msp * 1e-3), 1), "ms_per_step": round(msp, 4),
+                   "streamed_GB_per_s": round(bp / (msp * 1e-3) / 1e9, 1),
+                   "touched_experts_per_launch": round(sum(ntp) / len(ntp), 2)}
+        del gp, xp, op
 
     cpu = None
     if need_cpu:
@@ -370,6 +387,7 @@ def run_ours(args, rank, world, local):
         }
         if sweep:
             line["m_sweep"] = sweep
+            line["prefill_chunked"] = prefill
         print(json.dumps(line), flush=True)
     moe.close()
 

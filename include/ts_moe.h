@@ -1,13 +1,16 @@
 /*
  * ts_moe.h -- C ABI of the B200 (sm_100a) routed MoE half of a decoder layer.
  *
- * One call of ts_moe_forward runs, for a micro-batch of M <= 16 tokens, the
- * routed half that the turbospark-runtime family-state pages describe:
+ * One call of ts_moe_forward runs, for M tokens, the routed half that the
+ * turbospark-runtime family-state pages describe:
  *   router GEMV to FP32 logits -> family top-k rule -> each selected expert's
  *   gate/up GEMV, SwiGLU (or clamped SwiGLU), down GEMV -> weighted sum
  *   (+ optional shared expert) -> added back to the residual stream.
  * Every step runs in this library's CUDA kernels on the caller's stream; the
  * host does no per-call arithmetic, no allocation and no synchronisation.
+ * One kernel launch takes at most TS_MOE_MAX_TOKENS (16) tokens, the pages'
+ * micro-batch; a call with more runs as ceil(M / 16) launches over consecutive
+ * 16-row blocks (full blocks first), as the pages' chunked-prefill driver does.
  *
  * Conventions
  *   - "device" pointers are CUDA device addresses on cfg->device; "host"
@@ -31,7 +34,8 @@ extern "C" {
 #endif
 
 #define TS_MOE_ABI_VERSION 1u
-#define TS_MOE_MAX_TOKENS 16 /* micro-batch cap: MAX_PREFILL_BATCH = 16 (llama / gpt-oss state pages) */
+#define TS_MOE_MAX_TOKENS 16     /* tokens per launch: MAX_PREFILL_BATCH = 16 (llama / gpt-oss state pages) */
+#define TS_MOE_MAX_PREFILL 65536 /* largest max_tokens: calls above 16 tokens run in 16-token chunks */
 #define TS_MOE_MAX_TOPK 8    /* PHASE2_FIXED_SLOTS = 8 (deepseek2 state page, `build`) */
 #define TS_MOE_MAX_EXPERTS 256
 
@@ -76,7 +80,7 @@ typedef struct {
   int32_t num_experts;   /* E, 1..256 */
   int32_t top_k;         /* K, 1..min(8, E) */
   int32_t num_layers;    /* layers held by this handle, 1..1024 */
-  int32_t max_tokens;    /* largest M any call will pass, 1..16 */
+  int32_t max_tokens;    /* largest M any call will pass, 1..65536 (the workspace holds min(max_tokens, 16)) */
   int32_t expert_fmt;    /* TS_FMT_*; router and shared expert are always Q8_0 */
   int32_t score;         /* TS_SCORE_* */
   int32_t bias_mode;     /* TS_BIAS_* */
@@ -121,8 +125,9 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
  * idx: device [M][K] int32 selected experts in slot order (descending
  * selection logit, lower index first on ties); w: device [M][K] float32
  * weights; logits: device [M][E] float32 router logits before any bias, or
- * NULL.  0 <= M <= max_tokens (M = 0 is a no-op).  Asynchronous on `stream`
- * (a cudaStream_t, NULL = legacy default stream). */
+ * NULL.  0 <= M <= max_tokens (M = 0 is a no-op; M > 16 runs in 16-token
+ * chunks, one launch each).  Asynchronous on `stream` (a cudaStream_t, NULL =
+ * legacy default stream). */
 ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
                            void* stream);
 
@@ -130,8 +135,11 @@ ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* 
  * post-attention-norm activations, `moe_x`).  resid: device [M][H] BF16,
  * updated in place to bf16(resid + y), or NULL.  y: device [M][H] float32
  * routed(+shared) sum (`h2`), or NULL.  At least one of resid / y must be
- * non-NULL.  Asynchronous on `stream`; allocates nothing; calls on one handle
- * must not overlap on the device (they share the handle's workspace). */
+ * non-NULL.  0 <= M <= max_tokens; M > 16 runs as ceil(M / 16) launches of
+ * one 16-row block each (the remainder last), each token's result the same as
+ * in a call of its own block.  Asynchronous on `stream`; allocates nothing;
+ * calls on one handle must not overlap on the device (they share the
+ * handle's workspace). */
 ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word that
@@ -156,7 +164,8 @@ typedef struct {
 ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
 
 /* Optional timing hooks for profiling: when set, ts_moe_forward records
- * events[0] before and events[1] after its layer kernel on the call's stream
+ * events[0] before and events[1] after its layer kernel launches (one per
+ * 16-token chunk) on the call's stream
  * (cudaEvent_t values; events[2] and events[3] must be valid events and are
  * reserved; NULL clears).  An event between two forwards separates their
  * kernels, so a timed run without hooks is the throughput number. */

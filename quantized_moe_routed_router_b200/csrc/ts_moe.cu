@@ -119,7 +119,7 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
   if (c->top_k < 1 || c->top_k > TS_MOE_MAX_TOPK || c->top_k > c->num_experts)
     return bad("top_k must be in [1, min(8, num_experts)] (the 8-slot phase-2 reduce)");
   if (c->num_layers < 1 || c->num_layers > 1024) return bad("num_layers must be in [1, 1024]");
-  if (c->max_tokens < 1 || c->max_tokens > TS_MOE_MAX_TOKENS) return bad("max_tokens must be in [1, 16]");
+  if (c->max_tokens < 1 || c->max_tokens > TS_MOE_MAX_PREFILL) return bad("max_tokens must be in [1, 65536]");
   if (c->expert_fmt != TS_FMT_Q8_0 && c->expert_fmt != TS_FMT_MXFP4) return bad("unknown expert_fmt");
   if (c->score != TS_SCORE_SOFTMAX_SELECTED && c->score != TS_SCORE_SOFTMAX_ALL_NORENORM &&
       c->score != TS_SCORE_SIGMOID_RENORM)
@@ -256,7 +256,9 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   ts_moe* h = new ts_moe();
   h->cfg = *cfg;
   const ts_moe_config& c = h->cfg;
-  const int H = c.hidden, I = c.moe_inter, E = c.num_experts, K = c.top_k, S = c.shared_inter, Mx = c.max_tokens;
+  const int H = c.hidden, I = c.moe_inter, E = c.num_experts, K = c.top_k, S = c.shared_inter;
+  // The workspace holds one launch's tokens: a call with more runs in chunks.
+  const int Mx = std::min(c.max_tokens, TS_MOE_MAX_TOKENS);
   const int fmt = c.expert_fmt;
   h->sm_count = prop.multiProcessorCount;
   h->nb = std::min(h->sm_count, MAX_NB);
@@ -549,17 +551,29 @@ static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t
   return TS_MOE_OK;
 }
 
+// A call of M tokens runs as ceil(M / 16) launches over consecutive row blocks:
+// full 16-token chunks first, the remainder last.  Tokens are independent in
+// the routed half, so the chunking changes no token's route or its math (the
+// chunked-prefill driver of the gpt-oss state page, `BatchedRoutedScratch`,
+// feeds the routed half MAX_PREFILL_BATCH rows at a time the same way).
+static inline int chunk_rows(int M, int m0) { return std::min(TS_MOE_MAX_TOKENS, M - m0); }
+
 ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
                            void* stream) {
   ts_moe_status s = check_call(h, layer, x, M);
   if (s != TS_MOE_OK) return s;
   if (M == 0) return TS_MOE_OK;
   if (!idx || !w) return fail(h, TS_MOE_EINVAL, "idx and w must be non-NULL");
-  RouteParams rp = route_params(h, layer, x, M);
-  rp.idx_out = idx;
-  rp.w_out = w;
-  rp.logits_out = logits;
-  return launch_route(h, rp, (cudaStream_t)stream);
+  const int H = h->cfg.hidden, E = h->cfg.num_experts, K = h->cfg.top_k;
+  for (int m0 = 0; m0 < M; m0 += TS_MOE_MAX_TOKENS) {
+    RouteParams rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0));
+    rp.idx_out = idx + (size_t)m0 * K;
+    rp.w_out = w + (size_t)m0 * K;
+    rp.logits_out = logits ? logits + (size_t)m0 * E : nullptr;
+    s = launch_route(h, rp, (cudaStream_t)stream);
+    if (s != TS_MOE_OK) return s;
+  }
+  return TS_MOE_OK;
 }
 
 ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream) {
@@ -572,7 +586,6 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   const LayerDev& d = h->layers[layer];
   LayerParams lp;
   std::memset(&lp, 0, sizeof(lp));
-  lp.rp = route_params(h, layer, x, M);
   lp.xh = h->xh;
   lp.part_pub = h->part_pub;
   lp.max_pub = h->max_pub;
@@ -600,21 +613,25 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   lp.grid_gen = h->grid + 1;
   lp.xh_cnt = h->grid + 2;
   lp.route_cnt = h->grid + 3;
-  lp.y = y;
-  lp.resid = (__nv_bfloat16*)resid;
   lp.err = h->err;
   lp.act = c.act;
   lp.alpha = c.act_alpha;
   lp.limit = c.act_limit;
 
   const size_t smem = sizeof(LayerSmem);
-  cudaError_t e;
+  const int H = c.hidden;
   if (h->timing) cudaEventRecord(h->ev[0], st);
-  if (c.expert_fmt == TS_FMT_MXFP4)
-    e = launch_pdl(layer_kernel<1>, h->nb, NTHREADS, smem, st, lp);
-  else
-    e = launch_pdl(layer_kernel<0>, h->nb, NTHREADS, smem, st, lp);
-  if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
+  for (int m0 = 0; m0 < M; m0 += TS_MOE_MAX_TOKENS) {
+    lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0));
+    lp.y = y ? y + (size_t)m0 * H : nullptr;
+    lp.resid = resid ? (__nv_bfloat16*)resid + (size_t)m0 * H : nullptr;
+    cudaError_t e;
+    if (c.expert_fmt == TS_FMT_MXFP4)
+      e = launch_pdl(layer_kernel<1>, h->nb, NTHREADS, smem, st, lp);
+    else
+      e = launch_pdl(layer_kernel<0>, h->nb, NTHREADS, smem, st, lp);
+    if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
+  }
   if (h->timing) cudaEventRecord(h->ev[1], st);
   return TS_MOE_OK;
 }

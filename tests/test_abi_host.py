@@ -56,7 +56,7 @@ SHAPE = synth.MoEShape("t", 64, 64, 4, 2, cfg_id=77, max_tokens=4)
     (dict(num_experts=300), 1, "num_experts"),
     (dict(top_k=9), 1, "top_k"),
     (dict(top_k=5), 1, "top_k"),           # > num_experts (4)
-    (dict(max_tokens=17), 1, "max_tokens"),
+    (dict(max_tokens=65537), 1, "max_tokens"),
     (dict(max_tokens=0), 1, "max_tokens"),
     (dict(expert_fmt=2), 1, "expert_fmt"),
     (dict(score=3), 1, "score"),
@@ -71,6 +71,13 @@ def test_open_time_refusals(B, over, status, frag):
     st, msg = B.validate(SHAPE, _small_layers(SHAPE), **over)
     assert st == status, msg
     assert frag in msg
+
+
+@pytest.mark.parametrize("mt", [16, 17, 64, 65536])
+def test_max_tokens_above_one_launch_is_accepted(B, mt):
+    """Calls above 16 tokens run in 16-token launches, so max_tokens may exceed 16."""
+    st, msg = B.validate(SHAPE, _small_layers(SHAPE), max_tokens=mt)
+    assert st == 0, msg
 
 
 def test_bias_and_shared_consistency(B):

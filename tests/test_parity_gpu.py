@@ -136,6 +136,51 @@ def test_batch_rows_match_single_token_calls():
         assert (y1[0] - yb[m]).abs().max() <= 1e-4 * rms
 
 
+# --------------------------------------------------------------------------- chunked prefill (M > 16)
+# A call of M > 16 tokens runs as 16-token launches over consecutive row blocks.
+
+@pytest.mark.parametrize("name,M", [("q8_all_norenorm_shared", 37), ("mx_odd_blocks_clamped_bias", 40),
+                                    ("q8_sigmoid_correction_bias", 33), ("e256_k8", 64), ("one_expert", 17)])
+def test_chunked_prefill_small(name, M):
+    shape = SMALL[name].replace(max_tokens=M)
+    rep = parity.check_shape(shape, M)
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
+def test_chunked_prefill_equals_calls_per_block():
+    """Each 16-row block of a chunked call gives bit-for-bit what a call of that
+    block alone gives (y, the updated residual, and the routing)."""
+    from quantized_moe_routed_router_b200 import binding
+    shape = SMALL["q8_all_norenorm_shared"].replace(max_tokens=45)
+    M, H, K = 45, shape.hidden, shape.top_k
+    moe = binding.MoE(shape, [synth.make_layer(shape, 0, device="cuda")])
+    x = synth.make_x(shape, 0, M, device="cuda")
+    r = synth.make_x(shape, 0, M, device="cuda", tensor=synth.T_RESID)
+    y_all, o_all = torch.empty(M, H, device="cuda"), r.clone()
+    i_all = torch.empty(M, K, dtype=torch.int32, device="cuda")
+    w_all = torch.empty(M, K, device="cuda")
+    moe.forward(0, x, o_all, y_all)
+    moe.route(0, x, i_all, w_all)
+    for m0 in range(0, M, 16):
+        m1 = min(M, m0 + 16)
+        y_b, o_b = torch.empty(m1 - m0, H, device="cuda"), r[m0:m1].clone()
+        i_b = torch.empty(m1 - m0, K, dtype=torch.int32, device="cuda")
+        w_b = torch.empty(m1 - m0, K, device="cuda")
+        moe.forward(0, x[m0:m1].contiguous(), o_b, y_b)
+        moe.route(0, x[m0:m1].contiguous(), i_b, w_b)
+        torch.cuda.synchronize()
+        assert torch.equal(y_b, y_all[m0:m1]) and torch.equal(o_b, o_all[m0:m1])
+        assert torch.equal(i_b, i_all[m0:m1]) and torch.equal(w_b, w_all[m0:m1])
+    moe.device_status()
+
+
+def test_chunked_prefill_gptoss_full_size_sampled():
+    """The gpt-oss-shaped MXFP4 layer at M = 40 (16 + 16 + 8), sampled rows from every block."""
+    shape = synth.CONFIGS[3].replace(max_tokens=40)
+    rep = parity.check_shape(shape, 40, rows=[0, 7, 15, 16, 25, 31, 32, 39])
+    assert rep.max_err_y <= 1e-2 * rep.rms_y
+
+
 # --------------------------------------------------------------------------- the five workloads at full size
 
 @pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 16), (4, 16)])
