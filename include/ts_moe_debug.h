@@ -1,8 +1,9 @@
 /*
- * ts_moe_debug.h -- host-only helpers exported for tests.  They expose the
+ * ts_moe_debug.h -- helpers exported for tests.  All but the last expose the
  * pure arithmetic the kernels use to split work between CTAs and the open-time
- * validation, so both can be checked on a machine without a GPU.  None of
- * them touches device memory or the CUDA runtime.
+ * validation, so both can be checked on a machine without a GPU; they touch
+ * neither device memory nor the CUDA runtime.  The last one changes a
+ * handle's device counters so that a test can make a bounded wait run out.
  */
 #ifndef TS_MOE_DEBUG_H
 #define TS_MOE_DEBUG_H
@@ -32,6 +33,16 @@ int ts_moe_debug_group_size(int tiles);
 /* The validation ts_moe_open performs before any CUDA call; same status and
  * message (ts_moe_last_error(NULL)). */
 ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers);
+
+/* Failure-path test hook.  Synchronises `stream`, then moves the handle's
+ * grid-barrier launch counter two launches ahead of its arrival counter, so
+ * that the grid barrier of the next ts_moe_forward cannot complete: every CTA
+ * gives up after the bounded wait (2 s), sets the "grid barrier wait gave up"
+ * bit (0x40) of the device error word, and the kernel runs to its end.  The
+ * next ts_moe_device_status returns TS_MOE_EDEVICE and re-zeroes the
+ * counters, after which calls work normally again.  TS_MOE_ECUDA if a copy
+ * fails.  Not for production use. */
+ts_moe_status ts_moe_debug_skew_barrier(ts_moe* h, void* stream);
 
 #ifdef __cplusplus
 }

@@ -72,8 +72,10 @@ def _load():
     lib.ts_moe_debug_use_aligned.argtypes = [i32, i32]
     lib.ts_moe_debug_validate.argtypes = [C.POINTER(Config), C.POINTER(LayerWeights)]
     lib.ts_moe_route_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
+    lib.ts_moe_debug_skew_barrier.argtypes = [vp, vp]
     for f in ("ts_moe_open", "ts_moe_route", "ts_moe_forward", "ts_moe_device_status", "ts_moe_get_info",
-              "ts_moe_set_timing_events", "ts_moe_close", "ts_moe_debug_validate", "ts_moe_route_noalloc"):
+              "ts_moe_set_timing_events", "ts_moe_close", "ts_moe_debug_validate", "ts_moe_route_noalloc",
+              "ts_moe_debug_skew_barrier"):
         getattr(lib, f).restype = C.c_int
     return lib
 

@@ -807,7 +807,7 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   return TS_MOE_OK;
 }
 
-// ----------------------------------------------------------------------------- debug helpers (host-only arithmetic)
+// ----------------------------------------------------------------------------- debug helpers (host-only arithmetic; one failure-path test hook)
 uint64_t ts_moe_debug_range_start(uint64_t U, int NB, int b) { return range_start(U, NB, b); }
 int ts_moe_debug_owner_of(uint64_t U, int NB, uint64_t u) { return owner_of(U, NB, u); }
 int ts_moe_debug_partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return partial_slot(U, NB, b, g0); }
@@ -817,6 +817,17 @@ uint64_t ts_moe_debug_aligned_start(int G, int NB, int chunks, int b) {
   return (uint64_t)aligned_group_of(b, G, NB) * chunks + aligned_offset(b, G, NB, chunks);
 }
 int ts_moe_debug_use_aligned(int G, int NB) { return use_aligned(G, NB) ? 1 : 0; }
+ts_moe_status ts_moe_debug_skew_barrier(ts_moe* h, void* stream) {
+  if (!h) return TS_MOE_EINVAL;
+  TSM_CUDA(h, cudaSetDevice(h->cfg.device));
+  TSM_CUDA(h, cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned gen = 0;
+  TSM_CUDA(h, cudaMemcpy(&gen, h->grid + 1, 4, cudaMemcpyDeviceToHost));
+  gen += 2u;  // the next launch waits for (gen + 1) * NB arrivals; only NB more come
+  TSM_CUDA(h, cudaMemcpy(h->grid + 1, &gen, 4, cudaMemcpyHostToDevice));
+  return TS_MOE_OK;
+}
+
 ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers) {
   return validate(cfg, layers);
 }
