@@ -63,7 +63,7 @@ def load(name: str):
     H, I, E, K, S = (int(cfg[k]) for k in ("H", "I", "E", "K", "S"))
     fmt = {"q8_0": synth.FMT_Q8_0, "mxfp4": synth.FMT_MXFP4}[cfg["fmt"]]
     shape = synth.MoEShape(name, H, I, E, K, expert_fmt=fmt,
-                           score={"sel": 0, "all": 1}[cfg["score"]],
+                           score={"sel": 0, "all": 1, "sigmoid": 2}[cfg["score"]],
                            bias_mode={"none": 0, "logits": 1, "select_only": 2}[cfg["bias"]],
                            act={"swiglu": 0, "clamped": 1}[cfg["act"]], shared_inter=S, max_tokens=1)
 

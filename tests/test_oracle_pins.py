@@ -360,7 +360,7 @@ def test_layer_with_threads_equals_single_thread():
 
 
 @pytest.mark.parametrize("name", ["two_expert_swiglu_sel_k2.txt", "deepseek2_all_norenorm_shared_k1.txt",
-                                  "gptoss_clamped_bias_mxfp4_k2.txt"])
+                                  "gptoss_clamped_bias_mxfp4_k2.txt", "minimax_sigmoid_correction_bias_k2.txt"])
 def test_hand_computed_examples(name):
     shape, L, x, resid, expect = golden_loader.load(name)
     r = O.Oracle(shape, L).forward(x, resid)
