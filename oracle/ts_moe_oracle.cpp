@@ -8,7 +8,12 @@
 // What it computes, step by step, for each token m of a micro-batch (the
 // order of the pages; citations are page title + section):
 //   1. dequantise a weight row from its block format (Q8_0: fp16 scale times
-//      int8; MXFP4: E2M1 code times 2^(e-127))                 [format defs]
+//      int8; MXFP4: E2M1 code times 2^(e-127); INT4-affine: fp16 scale times
+//      a 4-bit code plus an fp16 offset)                       [format defs]
+//      INT4-affine is only named by the pages ("that seam is INT4-affine
+//      only", llama state page, `BatchedRoutedScratch`); its block -- 32
+//      weights, fp16 d and m, w = d * q + m with q in [0, 15] -- is this
+//      library's reading, matched to the 32-element blocks of the other formats
 //   2. router logits  l[e] = sum_n Wr[e,n] * s[n] * x[n]  with s the per-element
 //      router x-scale (all ones when absent), stored as FP32 as the pages'
 //      `router_logits_f32` buffer is                 [llama state: router_ones,
@@ -93,8 +98,13 @@ double e8m0_to_double(int e) { return e == 255 ? NAN : std::ldexp(1.0, e - 127);
 
 const int FMT_Q8_0 = 0;
 const int FMT_MXFP4 = 1;
+const int FMT_INT4_AFFINE = 2;
 
-size_t row_bytes(int fmt, int cols) { return (size_t)(cols / 32) * (fmt == FMT_Q8_0 ? 34 : 17); }
+// Bytes of one 32-weight block: Q8_0 {fp16 d; int8 q[32]}, MXFP4 {e8m0 e;
+// u8 qs[16]}, INT4-affine {fp16 d; fp16 m; u8 qs[16]}.
+size_t block_bytes(int fmt) { return fmt == FMT_Q8_0 ? 34 : fmt == FMT_MXFP4 ? 17 : 20; }
+
+size_t row_bytes(int fmt, int cols) { return (size_t)(cols / 32) * block_bytes(fmt); }
 
 // Dequantise one row of `cols` weights.
 void dequant_row(int fmt, const uint8_t* row, int cols, double* out) {
@@ -105,12 +115,21 @@ void dequant_row(int fmt, const uint8_t* row, int cols, double* out) {
       uint16_t dbits = (uint16_t)(blk[0] | (blk[1] << 8));
       double d = half_to_double(dbits);
       for (int i = 0; i < 32; ++i) out[b * 32 + i] = d * (double)(int8_t)blk[2 + i];
-    } else {
+    } else if (fmt == FMT_MXFP4) {
       const uint8_t* blk = row + (size_t)b * 17;
       double s = e8m0_to_double(blk[0]);
       for (int j = 0; j < 16; ++j) {
         out[b * 32 + 2 * j] = s * e2m1_to_double(blk[1 + j] & 15);
         out[b * 32 + 2 * j + 1] = s * e2m1_to_double(blk[1 + j] >> 4);
+      }
+    } else {
+      // INT4-affine: element 2j is the low nibble of qs[j], 2j+1 the high one
+      const uint8_t* blk = row + (size_t)b * 20;
+      double d = half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+      double m = half_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+      for (int j = 0; j < 16; ++j) {
+        out[b * 32 + 2 * j] = d * (double)(blk[4 + j] & 15) + m;
+        out[b * 32 + 2 * j + 1] = d * (double)(blk[4 + j] >> 4) + m;
       }
     }
   }

@@ -16,6 +16,13 @@ Block formats (the byte layouts the library's C ABI accepts):
   high nibble; each nibble is an E2M1 code (sign bit 3, magnitudes
   0, .5, 1, 1.5, 2, 3, 4, 6).  The gpt-oss state page names the format
   ("MXFP4 routed pair"); the nibble order is this library's reading.
+* INT4-affine, 20 bytes per 32 weights: ``{uint16 d; uint16 m (IEEE fp16
+  bits); uint8 qs[16]}``; element 2j is the low nibble of ``qs[j]``, element
+  2j+1 the high nibble; each nibble is an unsigned code q in [0, 15] and the
+  weight is ``d * q + m``.  The llama state page only names the format
+  ("that seam is INT4-affine only"); block size, field types and layout are
+  this library's reading, matched to the 32-element blocks of the others.
+  The oracle defines it; the CUDA library does not accept it yet.
 
 Matrices are row-major in blocks: a ``[R][C]`` matrix is R rows of C/32 blocks.
 Expert tensors stack E such matrices: gate/up ``[E][I][H]``, down ``[E][H][I]``.
@@ -25,6 +32,9 @@ Encoding rules (input preparation, not the method):
 * MXFP4 (OCP MX v1.0 conversion): ``X = floor(log2(amax)) - 2``, ``e = X + 127``
   clamped to [0, 254]; codes are ``w / 2^X`` rounded to nearest-even on the
   E2M1 grid and saturated to +-6; an all-zero block gets e = 0.
+* INT4-affine (min/max): ``m = fp16(min)``, ``d = fp16((max - min) / 15)``,
+  ``q = clamp(rint((w - m) / d), 0, 15)`` with the fp16-rounded d and m
+  (q = 0 when d = 0).
 
 Seeds: every tensor draws from its own ``torch.Generator`` seeded from
 (master seed, config id, layer, tensor id).  The same generator on the same
@@ -41,6 +51,7 @@ import torch
 
 FMT_Q8_0 = 0
 FMT_MXFP4 = 1
+FMT_INT4_AFFINE = 2  # oracle only: the CUDA library refuses it (unknown expert_fmt)
 SCORE_SOFTMAX_SELECTED = 0
 SCORE_SOFTMAX_ALL_NORENORM = 1
 SCORE_SIGMOID_RENORM = 2
@@ -52,13 +63,14 @@ ACT_SWIGLU_CLAMPED = 1
 
 Q8_0_BLOCK_BYTES = 34
 MXFP4_BLOCK_BYTES = 17
+INT4_AFFINE_BLOCK_BYTES = 20
 
 # tensor ids used in the per-tensor seed
 T_ROUTER, T_BIAS, T_GATE, T_UP, T_DOWN, T_SH_GATE, T_SH_UP, T_SH_DOWN, T_X, T_RESID, T_PES, T_XSCALE = range(12)
 
 
 def block_bytes(fmt: int) -> int:
-    return Q8_0_BLOCK_BYTES if fmt == FMT_Q8_0 else MXFP4_BLOCK_BYTES
+    return {FMT_Q8_0: Q8_0_BLOCK_BYTES, FMT_MXFP4: MXFP4_BLOCK_BYTES, FMT_INT4_AFFINE: INT4_AFFINE_BLOCK_BYTES}[fmt]
 
 
 def row_bytes(fmt: int, cols: int) -> int:
@@ -193,8 +205,28 @@ def encode_mxfp4(w: torch.Tensor) -> torch.Tensor:
     return out.reshape(R, C // 32 * 17)
 
 
+def encode_int4_affine(w: torch.Tensor) -> torch.Tensor:
+    """float32 [R, C] -> uint8 [R, C/32*20] INT4-affine blocks (min/max encoder)."""
+    R, C = w.shape
+    assert C % 32 == 0
+    b = w.reshape(R, C // 32, 32)
+    lo, hi = b.amin(dim=-1), b.amax(dim=-1)
+    m16 = lo.to(torch.float16)
+    d16 = ((hi - lo) / 15.0).to(torch.float16)
+    m, d = m16.to(torch.float32), d16.to(torch.float32)
+    safe = torch.where(d > 0, d, torch.ones_like(d))
+    q = torch.where(d.unsqueeze(-1) > 0, torch.round((b - m.unsqueeze(-1)) / safe.unsqueeze(-1)), torch.zeros_like(b))
+    q = q.clamp(0, 15).to(torch.int32)
+    qs = (q[..., 0::2] | (q[..., 1::2] << 4)).to(torch.uint8)
+    out = torch.empty((R, C // 32, 20), dtype=torch.uint8, device=w.device)
+    out[:, :, 0:2] = d16.contiguous().view(torch.uint8).reshape(R, C // 32, 2)
+    out[:, :, 2:4] = m16.contiguous().view(torch.uint8).reshape(R, C // 32, 2)
+    out[:, :, 4:] = qs
+    return out.reshape(R, C // 32 * 20)
+
+
 def encode(fmt: int, w: torch.Tensor) -> torch.Tensor:
-    return encode_q8_0(w) if fmt == FMT_Q8_0 else encode_mxfp4(w)
+    return {FMT_Q8_0: encode_q8_0, FMT_MXFP4: encode_mxfp4, FMT_INT4_AFFINE: encode_int4_affine}[fmt](w)
 
 
 # ----------------------------------------------------------------------------- layer weights

@@ -32,8 +32,17 @@ def decode_mxfp4(blob: np.ndarray, rows: int, cols: int) -> np.ndarray:
     return (scale[..., None] * E2M1_TABLE[codes]).reshape(rows, cols)
 
 
+def decode_int4_affine(blob: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    b = np.ascontiguousarray(blob, np.uint8).reshape(rows, cols // 32, 20)
+    d = b[:, :, 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    m = b[:, :, 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    qs = b[:, :, 4:]
+    q = np.stack([qs & 15, qs >> 4], axis=-1).reshape(rows, cols // 32, 32).astype(np.float64)
+    return (d[..., None] * q + m[..., None]).reshape(rows, cols)
+
+
 def decode(fmt: int, blob, rows, cols):
-    return decode_q8_0(blob, rows, cols) if fmt == 0 else decode_mxfp4(blob, rows, cols)
+    return (decode_q8_0, decode_mxfp4, decode_int4_affine)[fmt](blob, rows, cols)
 
 
 def act_np(kind: int, g, u, alpha=1.702, limit=7.0):
@@ -59,10 +68,12 @@ def layer_bruteforce(shape, L: dict, x_bits: np.ndarray, resid_bits=None):
     Wr = decode_q8_0(L["router"], E, H)
     logits = ((X * s) @ Wr.T).astype(np.float32)
     bias = L.get("bias")
+    # sigmoid scoring selects on sigmoid(l) (+ the correction bias) instead of l
+    base = expit(logits.astype(np.float64)) if shape.score == 2 else logits.astype(np.float64)
     if bias is not None and shape.bias_mode != 0:
-        lsel = (logits.astype(np.float64) + np.asarray(bias, np.float64)).astype(np.float32)
+        lsel = (base + np.asarray(bias, np.float64)).astype(np.float32)
     else:
-        lsel = logits.copy()
+        lsel = base.astype(np.float32)
     score = lsel.astype(np.float64) if (shape.bias_mode == 1 and bias is not None) else logits.astype(np.float64)
     idx = np.stack([topk_bruteforce(lsel[m], K) for m in range(M)]).astype(np.int32)
     G = np.zeros((M, E))
@@ -70,8 +81,11 @@ def layer_bruteforce(shape, L: dict, x_bits: np.ndarray, resid_bits=None):
     for m in range(M):
         if shape.score == 0:
             pw = softmax(score[m, idx[m]])
-        else:
+        elif shape.score == 1:
             pw = softmax(score[m])[idx[m]]
+        else:
+            sel = base[m, idx[m]]
+            pw = sel / sel.sum()
         pes = L.get("pes")
         if pes is not None:
             pw = pw * np.asarray(pes, np.float64)[idx[m]]

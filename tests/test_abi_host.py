@@ -58,7 +58,7 @@ SHAPE = synth.MoEShape("t", 64, 64, 4, 2, cfg_id=77, max_tokens=4)
     (dict(top_k=5), 1, "top_k"),           # > num_experts (4)
     (dict(max_tokens=65537), 1, "max_tokens"),
     (dict(max_tokens=0), 1, "max_tokens"),
-    (dict(expert_fmt=2), 1, "expert_fmt"),
+    (dict(expert_fmt=2), 1, "expert_fmt"),      # INT4-affine: defined in the oracle only so far
     (dict(score=3), 1, "score"),
     (dict(bias_mode=7), 1, "bias_mode"),
     (dict(act=5), 1, "act"),

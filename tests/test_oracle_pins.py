@@ -1,7 +1,8 @@
 """Pins the FP64 oracle to things other than itself (no GPU needed).
 
 * block formats: exhaustive decode of every fp16 / bf16 bit pattern against
-  numpy / torch, every E2M1 code against the OCP MX table, E8M0 against ldexp;
+  numpy / torch, every E2M1 code against the OCP MX table, E8M0 against ldexp,
+  every INT4-affine code against d * q + m and the encoder's exact round trip;
 * router / top-k / weights against brute-force sorts and library softmax;
 * the invariants the pages fix (softmax over the selected with per-expert
   ones; deepseek2 weights are the full softmax with no renorm so they sum to
@@ -121,6 +122,51 @@ def test_dequant_mxfp4_exhaustive():
         ref[0::2] = [sign(c) * table[c & 7] * s for c in lo]
         ref[1::2] = [sign(c) * table[c & 7] * s for c in hi]
         assert np.array_equal(got[r], ref)
+
+
+def test_dequant_int4_affine_exhaustive():
+    """Every 4-bit code in both nibble positions, under fp16 scales and offsets
+    of both signs, subnormal, zero and large, against d * q + m with numpy's
+    own fp16 decoding."""
+    pairs = [(0.03125, 0.0), (0.03125, -0.25), (1.0, -7.5), (6.1e-5, 3.0e-8), (3.0e-8, -6.1e-5),
+             (0.0, 0.5), (1.5, 1000.0), (-0.125, 0.0625), (4096.0, -65504.0)]
+    rows = len(pairs)
+    blob = np.zeros((rows, 1, 20), np.uint8)
+    lo = np.arange(16)
+    hi = (np.arange(16) * 7 + 3) % 16
+    for r, (d, m) in enumerate(pairs):
+        blob[r, 0, 0:2] = np.array([d], np.float16).view(np.uint8)
+        blob[r, 0, 2:4] = np.array([m], np.float16).view(np.uint8)
+        blob[r, 0, 4:] = lo | (hi << 4)
+    got = O.dequant(synth.FMT_INT4_AFFINE, blob.reshape(rows, -1), rows, 32)
+    for r, (d, m) in enumerate(pairs):
+        d16, m16 = float(np.float16(d)), float(np.float16(m))
+        ref = np.empty(32)
+        ref[0::2] = d16 * lo + m16
+        ref[1::2] = d16 * hi + m16
+        assert np.array_equal(got[r], ref), r
+
+
+def test_int4_affine_encoder_round_trip():
+    """Blocks whose values lie on an fp16-exact grid m + d*q come back exactly
+    (this ties the encoder's byte layout to the oracle's independent decoder);
+    N(0, 0.02) blocks come back within half a step plus the fp16 rounding of m."""
+    rng = np.random.default_rng(11)
+    R, C = 6, 128
+    d = np.ldexp(1.0, -rng.integers(3, 9, (R, C // 32)))
+    m = -d * rng.integers(0, 40, (R, C // 32))
+    q = rng.integers(0, 16, (R, C // 32, 32))
+    q[:, :, 0], q[:, :, 1] = 0, 15                      # the encoder's min and max sit on the grid
+    w = (m[..., None] + d[..., None] * q).reshape(R, C)
+    blob = synth.encode_int4_affine(torch.tensor(w, dtype=torch.float32)).numpy()
+    assert blob.shape == (R, C // 32 * synth.INT4_AFFINE_BLOCK_BYTES)
+    assert np.array_equal(O.dequant(synth.FMT_INT4_AFFINE, blob, R, C), w)
+    w2 = rng.normal(0, 0.02, (R, C)).astype(np.float32)
+    deq = O.dequant(synth.FMT_INT4_AFFINE, synth.encode_int4_affine(torch.tensor(w2)).numpy(), R, C)
+    b = w2.reshape(R, C // 32, 32).astype(np.float64)
+    step = ((b.max(-1) - b.min(-1)) / 15.0)[..., None]
+    err = np.abs(deq.reshape(R, C // 32, 32) - b)
+    assert np.all(err <= 0.5 * step * (1 + 2e-3) + 2e-3 * np.abs(b.min(-1))[..., None] + 1e-9)
 
 
 # --------------------------------------------------------------------------- router / selection
@@ -323,6 +369,11 @@ CASES = [
     dict(fmt=1, score=0, bias=2, act=1, S=0, E=5, K=3),
     dict(fmt=0, score=1, bias=0, act=0, S=96, E=6, K=3),
     dict(fmt=0, score=0, bias=0, act=0, S=0, E=4, K=4),
+    dict(fmt=0, score=2, bias=2, act=0, S=0, E=8, K=3),
+    dict(fmt=1, score=2, bias=0, act=1, S=0, E=6, K=2),
+    dict(fmt=2, score=0, bias=0, act=0, S=0, E=4, K=2),
+    dict(fmt=2, score=1, bias=0, act=0, S=96, E=6, K=3),
+    dict(fmt=2, score=0, bias=1, act=1, S=0, E=5, K=3),
 ]
 
 
