@@ -194,3 +194,25 @@ def test_group_sizes_keep_the_most_warp_slots_busy():
         assert slots(gs) == best                                      # fewest idle consumer-warp slots
         assert gs == max(g for g in range(15, 31) if slots(g) == best)  # ties: the larger group
     assert B.lib.ts_moe_debug_group_size(256) == 30 and B.lib.ts_moe_debug_group_size(360) == 30
+
+
+def _header_constants():
+    """Enum and #define values of include/ts_moe.h, parsed from the text."""
+    txt = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "ts_moe.h")).read(), flags=re.S)
+    vals = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(TS_\w+)\s*=\s*(\d+)", txt)}
+    vals.update({m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+(TS_\w+)\s+(\d+)u?\b", txt)})
+    return vals
+
+
+def test_header_constants_match_the_binding_and_the_generator(B):
+    h = _header_constants()
+    assert h["TS_MOE_ABI_VERSION"] == B.TS_MOE_ABI_VERSION
+    assert (h["TS_FMT_Q8_0"], h["TS_FMT_MXFP4"]) == (synth.FMT_Q8_0, synth.FMT_MXFP4)
+    assert "TS_FMT_INT4_AFFINE" not in h            # the library does not accept it yet
+    assert (h["TS_SCORE_SOFTMAX_SELECTED"], h["TS_SCORE_SOFTMAX_ALL_NORENORM"], h["TS_SCORE_SIGMOID_RENORM"]) == \
+        (synth.SCORE_SOFTMAX_SELECTED, synth.SCORE_SOFTMAX_ALL_NORENORM, synth.SCORE_SIGMOID_RENORM)
+    assert (h["TS_BIAS_NONE"], h["TS_BIAS_LOGITS"], h["TS_BIAS_SELECT_ONLY"]) == \
+        (synth.BIAS_NONE, synth.BIAS_LOGITS, synth.BIAS_SELECT_ONLY)
+    assert (h["TS_ACT_SWIGLU"], h["TS_ACT_SWIGLU_CLAMPED"]) == (synth.ACT_SWIGLU, synth.ACT_SWIGLU_CLAMPED)
+    assert (h["TS_MOE_MAX_TOKENS"], h["TS_MOE_MAX_TOPK"], h["TS_MOE_MAX_EXPERTS"]) == (16, 8, 256)
+    assert h["TS_MOE_OK"] == 0 and h["TS_MOE_EDEVICE"] == 5
