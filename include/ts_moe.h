@@ -50,8 +50,8 @@ typedef enum {
 
 enum { TS_FMT_Q8_0 = 0, TS_FMT_MXFP4 = 1 };
 /* Top-k rule.  SOFTMAX_SELECTED: softmax over the K selected experts (llama /
- * gpt-oss state pages, `per_expert_ones`: "selection reduces to softmax over the
- * selected").  SOFTMAX_ALL_NORENORM: softmax over all E experts, the K largest
+ * gpt-oss state pages, `per_expert_ones`: with unit per-expert scales the
+ * weights are exactly that softmax).  SOFTMAX_ALL_NORENORM: softmax over all E experts, the K largest
  * kept with no renormalisation (deepseek2 state page, layer sketch).
  * SIGMOID_RENORM: see below. */
 enum {
@@ -97,7 +97,7 @@ typedef struct {
  * per_expert_scale are always HOST memory; the other blobs live where
  * cfg->weights_mem says. */
 typedef struct {
-  const void* router;             /* [E][H] Q8_0 (llama state page: "INT8 router kernel" with an fp16 block scale) */
+  const void* router;             /* [E][H] Q8_0 (llama state page, `router_ones`: an int8 router GEMV; here int8 with an fp16 block scale) */
   const uint16_t* router_xscale;  /* [H] BF16 per-element x scale, or NULL = ones (`router_ones`) */
   const float* router_bias;       /* [E], finite; required iff bias_mode != NONE (`router_bias`) */
   const float* per_expert_scale;  /* [E], or NULL = ones (`per_expert_ones`); multiplies the weights */
@@ -121,7 +121,10 @@ typedef struct ts_moe ts_moe;
  * at token 1").  *out is set only on TS_MOE_OK.  Synchronises the device. */
 ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* layers, ts_moe** out);
 
-/* Router GEMV + top-k only (steps a1-a3).  x: device [M][H] BF16 (row-major).
+/* Router GEMV + top-k only: the int8 router GEMV to FP32 logits with the
+ * per-element x scale (llama state page, `router_ones`, `router_logits_f32`),
+ * the router bias added before the top-k (gpt-oss state page, `router_bias`)
+ * and the family's weight rule (see TS_SCORE_*).  x: device [M][H] BF16 (row-major).
  * idx: device [M][K] int32 selected experts in slot order (descending
  * selection logit, lower index first on ties); w: device [M][K] float32
  * weights; logits: device [M][E] float32 router logits before any bias, or
@@ -141,6 +144,13 @@ ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* 
  * calls on one handle must not overlap on the device (they share the
  * handle's workspace). */
 ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream);
+/* The layer kernel runs one CTA per SM and relies on all of them being
+ * resident at once (a grid-wide barrier and cross-CTA readiness waits);
+ * ts_moe_open refuses with TS_MOE_EUNSUPPORTED when the occupancy calculator
+ * says they cannot be.  Kernels of the same process running concurrently on
+ * other streams can still hold SMs; if they do so for longer than the 2 s wait
+ * limit, the forward gives up, its y is invalid, and ts_moe_device_status
+ * reports TS_MOE_EDEVICE. */
 
 /* Synchronises `stream`, then reads and clears the device error word that
  * kernels set on a bounded wait that gave up or an index found out of range.
@@ -171,32 +181,38 @@ ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
  * kernels, so a timed run without hooks is the throughput number. */
 ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4);
 
-/* Router GEMV + top-k for callers that cannot allocate device memory -- no
- * counterpart in the paper; this is a library convenience.  Some callers
- * cannot call cudaMalloc at the point where they need routing: code that
- * runs while a stream is being captured into a CUDA graph (allocation is not
- * capturable), engines that hand all device memory to their own pool and
- * forbid other allocations, or plugins that are given only a stream and
- * buffers.  They cannot use ts_moe_open (which allocates the weight arena
- * and workspace), so this entry point takes the raw router itself and keeps
- * all of its scratch in one file-scope device array of
- * TS_MOE_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
- * until the process exits.  It performs no allocation of any kind.
+/* Router GEMV + top-k for callers that cannot allocate device memory.  This
+ * entry point has no counterpart in the paper; it is a convenience of this
+ * library.  ts_moe_open allocates a weight arena and a workspace, and some
+ * callers cannot allocate at all: inference engines that hand every byte of
+ * device memory to their own pool when they start and forbid allocations
+ * afterwards, and plugins or extensions that are given only a stream and
+ * buffers the host application owns.  This call takes the raw router itself
+ * and keeps all of its scratch in one file-scope device array of
+ * TS_MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.  It calls no allocator of any kind.
  *
  * router: device [E][H] Q8_0 blocks (as in ts_moe_layer_weights.router);
  * router_bias, per_expert_scale: DEVICE [E] float32 or NULL (bias required
  * iff bias_mode != TS_BIAS_NONE); the router x-scale is taken as ones.
  * x: device [M][H] BF16, 16-byte aligned; idx: device [M][K] int32; w: device
- * [M][K] float32; logits: device [M][E] float32 or NULL.  Same semantics and
- * results as ts_moe_route on a handle opened with this router.
+ * [M][K] float32; logits: device [M][E] float32 or NULL.  The results are the
+ * ones ts_moe_route gives on a handle opened with the same router and no
+ * x-scale (both cut the router GEMV the same way for a given SM count).
  * Limits: 1 <= E <= 256, 1 <= K <= min(8, E), H a positive multiple of 32,
- * 0 <= M <= 16, and the scratch (repacked router + staged x + route state)
- * must fit in TS_MOE_NOALLOC_SCRATCH_BYTES, else TS_MOE_EINVAL with the
- * required size in ts_moe_last_error(NULL).
+ * 0 <= M <= 16, and the scratch (repacked router + route state) must fit in
+ * TS_MOE_NOALLOC_SCRATCH_BYTES, else TS_MOE_EINVAL with the required size in
+ * ts_moe_last_error(NULL).
+ * Errors found on the device cannot be returned by this asynchronous call, so
+ * they are reported in its outputs: a non-finite router block scale, bias or
+ * per-expert scale, a token whose logits are all NaN (x holding NaN), or a
+ * bounded wait that gave up makes every idx entry -1 and every w entry 0
+ * (logits are then unspecified).  Check idx[0] >= 0 after synchronising if that matters.
  * The first call on a device looks up the scratch array's device address and
- * sets a kernel attribute; make that first call before any stream capture.
- * Every call shares the one array and leaves its contents behind: calls that
- * overlap on the GPU (different streams, or graphs replayed concurrently)
+ * sets a kernel attribute with that device current; make that first call before
+ * any stream capture.  Every call shares the one array and leaves its contents
+ * behind (the words that must start at zero are cleared by each call): calls
+ * that overlap on the GPU (different streams, or concurrent graph replays)
  * race and must be serialised by the caller.  Asynchronous on `stream`. */
 #define TS_MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
 ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias, const float* per_expert_scale,

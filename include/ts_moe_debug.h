@@ -30,6 +30,12 @@ uint64_t ts_moe_debug_aligned_start(int G, int NB, int chunks, int b);
 int ts_moe_debug_use_aligned(int G, int NB);
 /* Tiles per group chosen for an expert matrix of `tiles` 16-row tiles. */
 int ts_moe_debug_group_size(int tiles);
+/* CTAs per layer-kernel launch on a device with `sm_count` SMs (one per SM). */
+int ts_moe_debug_layer_ctas(int sm_count);
+/* 1 when `nb` CTAs of the layer kernel can all be resident at once given
+ * `per_sm` of them per SM (the occupancy calculator's answer) on `sm_count`
+ * SMs; ts_moe_open refuses with TS_MOE_EUNSUPPORTED when this is 0. */
+int ts_moe_debug_coresident(int per_sm, int sm_count, int nb);
 /* The validation ts_moe_open performs before any CUDA call; same status and
  * message (ts_moe_last_error(NULL)). */
 ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers);

@@ -19,6 +19,14 @@ SRC = os.path.join(HERE, "ts_moe_oracle.cpp")
 LIB = os.path.join(HERE, "libts_moe_oracle.so")
 
 
+def nthreads() -> int:
+    """Host threads the oracle runs on: the cores this process may use."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle with g++ (plain IEEE FP64, no fast-math)."""
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):

@@ -10,8 +10,9 @@
 //   1. dequantise a weight row from its block format (Q8_0: fp16 scale times
 //      int8; MXFP4: E2M1 code times 2^(e-127); INT4-affine: fp16 scale times
 //      a 4-bit code plus an fp16 offset)                       [format defs]
-//      INT4-affine is only named by the pages ("that seam is INT4-affine
-//      only", llama state page, `BatchedRoutedScratch`); its block -- 32
+//      INT4-affine is only named by the pages (gpt-oss state page,
+//      `BatchedRoutedScratch`: the batched-GEMV seam takes only INT4-affine
+//      tensors); its block -- 32
 //      weights, fp16 d and m, w = d * q + m with q in [0, 15] -- is this
 //      library's reading, matched to the 32-element blocks of the other formats
 //   2. router logits  l[e] = sum_n Wr[e,n] * s[n] * x[n]  with s the per-element
@@ -23,8 +24,8 @@
 //                                                        router_bias]
 //   4. S = top-K of l' by (value desc, index asc) (sigmoid scoring: of s + b, below)
 //   5. weights: softmax over the selected experts (SOFTMAX_WEIGHT, norm_w
-//      false: with per-expert ones "selection reduces to softmax over the
-//      selected")                                       [llama / gpt-oss state:
+//      false: with all per-expert scales 1 the weights are exactly the
+//      softmax of the selected logits)                  [llama / gpt-oss state:
 //                                                        per_expert_ones]
 //      or, for the deepseek2 rule, the full softmax over all experts taken at
 //      the selected indices, with no renormalisation  [deepseek2 state, layer
@@ -44,8 +45,8 @@
 //      (gate <= L, |up| <= L, g*sigmoid(alpha g)*(u+1))    [gpt-oss state
 //                                                           header]
 //   7. shared expert (deepseek2): y += Wd_s act(Wg_s x, Wu_s x), weight 1
-//                                 [deepseek2 state: "x += routed_sum + shared
-//                                  SwiGLU(f)"]
+//                                 [deepseek2 state, layer sketch: the
+//                                  shared SwiGLU joins the routed sum]
 //   8. out = resid + y, also rounded to BF16          [llama state: h2 "added
 //                                                     back to the stream"]
 // All arithmetic after the FP32 logits buffer is FP64.

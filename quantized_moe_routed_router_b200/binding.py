@@ -70,6 +70,8 @@ def _load():
     lib.ts_moe_debug_aligned_start.argtypes = [i32, i32, i32, i32]
     lib.ts_moe_debug_aligned_start.restype = C.c_uint64
     lib.ts_moe_debug_use_aligned.argtypes = [i32, i32]
+    lib.ts_moe_debug_coresident.argtypes = [i32, i32, i32]
+    lib.ts_moe_debug_layer_ctas.argtypes = [i32]
     lib.ts_moe_debug_validate.argtypes = [C.POINTER(Config), C.POINTER(LayerWeights)]
     lib.ts_moe_route_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
     lib.ts_moe_debug_skew_barrier.argtypes = [vp, vp]

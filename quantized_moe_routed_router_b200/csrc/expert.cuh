@@ -13,7 +13,8 @@
 //                 that expert is done, prefetching its weights meanwhile;
 //   4. combine -- after a bounded grid-wide barrier each CTA forms 1/NB of
 //                 y[t] = sum_k w[t][k] down_k[t] (+ shared, deepseek2 state
-//                 page: "y = shared + sum(w * expert)") and resid += y.
+//                 page, `shared_out`: the shared output seeds the sum) and
+//                 resid += y.
 //
 // Work split: the (entry, group, chunk) units of each GEMV phase are cut into
 // one equal contiguous range per CTA (stream-K), so every SM streams the same

@@ -4,7 +4,7 @@
 // open into the 16-row MMA fragment layout of the experts, one 16-expert tile
 // after another (rows past E are zero), and the FP32 logits come out of
 // m16n8k16 MMAs with the block scale folded in per 32-block (llama state page,
-// `router_ones`: the INT8 router kernel scales x[n] per element;
+// `router_ones`: the int8 router GEMV scales x[n] per element;
 // `router_logits_f32`: one FP32 row of logits per token).
 //
 // The GEMV is cut into items (tile j, slice c): slice c is the K range of
@@ -23,8 +23,8 @@
 // One warp per token then selects the top K by (selection logit desc, index
 // asc), where the selection logit is l + b when a router bias is present
 // (gpt-oss state page, `router_bias`: added BEFORE the top-k), and forms the
-// weights: softmax over the selected ("selection reduces to softmax over the
-// selected", `per_expert_ones`), or the full softmax over all experts taken at
+// weights: softmax over the selected (`per_expert_ones`: with unit per-expert
+// scales the weights are exactly that softmax), or the full softmax over all experts taken at
 // the selected indices without renormalisation (deepseek2 layer sketch), or --
 // with sigmoid scoring (llama state page, MiniMax flow) -- the sigmoid scores
 // s of the selected experts renormalised to sum 1, the selection then being by
@@ -82,6 +82,8 @@ struct RouteParams {
   int* idx_out;            // optional user outputs
   float* w_out;
   float* logits_out;
+  const unsigned* pre_err; // route_kernel only: a word an earlier kernel of the same call set on bad input, or null
+  int sentinel;            // route_kernel only: on any error, overwrite idx_out / w_out with -1 / 0
 };
 
 // Routing results, in the shared memory of the kernel that routes.
@@ -561,6 +563,21 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
 // ---------------------------------------------------------------------------- standalone route kernel
 constexpr int ROUTE_THREADS = ROUTE_WARPS * 32;
 
+// End of a route_kernel run with p.sentinel set: if this call's error word or
+// the earlier kernel's word (p.pre_err) holds any bit, every (token, slot) of
+// idx_out / w_out becomes -1 / 0, so a failed call cannot pass for a routing.
+// Needs a CTA barrier after every write of idx_out / w_out and every error bit.
+TSM_DEV void route_sentinel(const RouteParams& p, int tid) {
+  __shared__ unsigned bad;
+  if (tid == 0) bad = *reinterpret_cast<volatile unsigned*>(p.err) | (p.pre_err ? *p.pre_err : 0u);
+  __syncthreads();
+  if (!bad) return;
+  for (int i = tid; i < p.M * p.K; i += ROUTE_THREADS) {
+    if (p.idx_out) p.idx_out[i] = -1;
+    if (p.w_out) p.w_out[i] = 0.f;
+  }
+}
+
 // One CTA: the items (j, c) in slice order, each slice's x staged by bulk copy,
 // router units read from global memory; logits accumulated in slice order.
 // Dynamic shared memory: RouteState, then the slice buffers (SliceSmem).
@@ -581,6 +598,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
   grid_dep_wait();
   grid_dep_launch();
   if (tid == 0) slice_issue_x(p, s, 0, xs);
+  // the bias and per-expert scale are device inputs here: a non-finite one is an error of the call
+  if (tid < p.E && !(isfinite(rc.b) && isfinite(rc.s))) atomicOr(p.err, ERR_BAD_ROUTER_INPUT);
   route_init_smem(s, rc, tid);
   for (int i = tid; i < p.M * MAX_E; i += ROUTE_THREADS) s.lg[i / MAX_E][i % MAX_E] = 0.f;
   if (tid < MAX_TOK) s.gmax[tid] = 0.f;
@@ -610,6 +629,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
   route_topk(p, s, warp, lane);
   __syncthreads();
   route_list(p, s, warp, lane, tid, ROUTE_THREADS);
+  if (p.sentinel) route_sentinel(p, tid);
 }
 
 }  // namespace tsm

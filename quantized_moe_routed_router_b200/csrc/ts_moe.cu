@@ -192,6 +192,27 @@ int choose_slices(int M, int C, int T, int E, int nb, bool split) {
   return best;
 }
 
+// CTAs of one layer-kernel launch on a device with `sm_count` SMs: one per SM.
+int layer_ctas(int sm_count) { return std::min(sm_count, MAX_NB); }
+
+// Router slicing (count S and chunks per slice CS) for M tokens.  The handle
+// path and the allocation-free entry point both take it from here, so that for
+// the same router and SM count both sum a logit's partial products in the same
+// order (the allocation-free path matches a handle opened without an x-scale).
+bool router_slicing(int M, const MatGeom& gR, int E, int nb, bool split, int& S, int& CS) {
+  const int s = choose_slices(M, gR.chunks, gR.tiles, E, nb, split);
+  if (s == 0) return false;
+  CS = (gR.chunks + s - 1) / s;
+  S = (gR.chunks + CS - 1) / CS;
+  return true;
+}
+
+// The layer kernel's grid barrier and readiness waits need all `nb` CTAs
+// resident at once.  With `per_sm` CTAs of it fitting on one SM (from the
+// occupancy calculator) and `sm_count` SMs, that holds on an otherwise idle
+// device iff per_sm >= 1 and nb <= per_sm * sm_count.
+bool coresident(int per_sm, int sm_count, int nb) { return per_sm >= 1 && (long long)nb <= (long long)per_sm * sm_count; }
+
 template <typename... Args>
 cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t lc = {};
@@ -261,7 +282,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   const int Mx = std::min(c.max_tokens, TS_MOE_MAX_TOKENS);
   const int fmt = c.expert_fmt;
   h->sm_count = prop.multiProcessorCount;
-  h->nb = std::min(h->sm_count, MAX_NB);
+  h->nb = layer_ctas(h->sm_count);
   h->Hp = round_up(H, 64);
   h->Ip = round_up(I, 64);
   h->Sp = S ? round_up(S, 64) : 0;
@@ -281,7 +302,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
           break;
         }
   for (int m = 1; m <= Mx; ++m) {
-    h->slices[m] = choose_slices(m, h->gR.chunks, h->gR.tiles, E, h->nb, h->any_xscale);
+    int S_m = 0, CS_m = 0;
+    h->slices[m] = router_slicing(m, h->gR, E, h->nb, h->any_xscale, S_m, CS_m) ? S_m : 0;
     if (h->slices[m] == 0) {
       g_open_error = "no router slicing fits these sizes (too many experts for the SM count, or hidden too large)";
       ts_moe_close(h);
@@ -400,6 +422,22 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   if ((st = set_smem_attrs(h)) != TS_MOE_OK) {
     g_open_error = h->error;
     return cleanup(st);
+  }
+  {
+    // every CTA of a layer launch must be resident at once (grid barrier)
+    int per_sm = 0;
+    ce = fmt == TS_FMT_MXFP4
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<1>, NTHREADS, sizeof(LayerSmem))
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<0>, NTHREADS, sizeof(LayerSmem));
+    if (ce != cudaSuccess) {
+      g_open_error = std::string("occupancy query: ") + cudaGetErrorString(ce);
+      return cleanup(TS_MOE_ECUDA);
+    }
+    if (!coresident(per_sm, h->sm_count, h->nb)) {
+      g_open_error = "the layer kernel's " + std::to_string(h->nb) + " CTAs cannot all be resident at once (" +
+                     std::to_string(per_sm) + " per SM on " + std::to_string(h->sm_count) + " SMs)";
+      return cleanup(TS_MOE_EUNSUPPORTED);
+    }
   }
 
   // ---- upload + repack every layer
@@ -527,8 +565,7 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.idx = h->idx;
   rp.w = h->w;
   rp.shift = h->shift;
-  rp.CS = (h->gR.chunks + h->slices[M] - 1) / h->slices[M];
-  rp.S = (h->gR.chunks + rp.CS - 1) / rp.CS;
+  router_slicing(M, h->gR, rp.E, h->nb, h->any_xscale, rp.S, rp.CS);  // fits: checked at open
   rp.meta = h->meta;
   rp.routes = h->routes;
   rp.rpos = h->rpos;
@@ -644,11 +681,11 @@ ts_moe_status ts_moe_device_status(ts_moe* h, void* stream) {
   TSM_CUDA(h, cudaMemcpy(&err, h->err, 4, cudaMemcpyDeviceToHost));
   if (!err) return TS_MOE_OK;
   TSM_CUDA(h, cudaMemset(h->counters, 0, h->counters_bytes));
-  char buf[384];
+  char buf[512];
   std::snprintf(buf, sizeof buf, "device error word 0x%x (bit0/1: weight-stage wait gave up, bit2/3: activation-window "
                 "wait gave up, bit4: bad index, bit5: bad route metadata, bit6: grid barrier wait gave up, bit7: "
                 "wait for an expert's activations gave up, bit8: wait for the staged x gave up, bit9: wait for the "
-                "shared FP16 x gave up, bit10: wait for the router logits gave up)", err);
+                "shared FP16 x gave up, bit10: wait for the router logits gave up, bit11: non-finite router bias or per-expert scale)", err);
   return fail(h, TS_MOE_EDEVICE, buf);
 }
 
@@ -795,13 +832,13 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   rp.idx_out = idx;
   rp.w_out = w;
   rp.logits_out = logits;
+  rp.pre_err = errw + 1;  // the repack's bad-scale word
+  rp.sentinel = 1;
   int nsm = 0;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
-  const int S = choose_slices(M, gR.chunks, gR.tiles, E, std::min(nsm, MAX_NB), false);
-  if (S == 0) return fail(nullptr, TS_MOE_EUNSUPPORTED, "no router slicing fits these sizes");
-  rp.CS = (gR.chunks + S - 1) / S;
-  rp.S = (gR.chunks + rp.CS - 1) / rp.CS;
+  if (!router_slicing(M, gR, E, layer_ctas(nsm), false, rp.S, rp.CS))
+    return fail(nullptr, TS_MOE_EUNSUPPORTED, "no router slicing fits these sizes");
   e = launch_pdl(route_kernel, 1, ROUTE_THREADS, route_smem(rp), s, rp);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("route_kernel launch: ") + cudaGetErrorString(e));
   return TS_MOE_OK;
@@ -817,6 +854,8 @@ uint64_t ts_moe_debug_aligned_start(int G, int NB, int chunks, int b) {
   return (uint64_t)aligned_group_of(b, G, NB) * chunks + aligned_offset(b, G, NB, chunks);
 }
 int ts_moe_debug_use_aligned(int G, int NB) { return use_aligned(G, NB) ? 1 : 0; }
+int ts_moe_debug_coresident(int per_sm, int sm_count, int nb) { return coresident(per_sm, sm_count, nb) ? 1 : 0; }
+int ts_moe_debug_layer_ctas(int sm_count) { return layer_ctas(sm_count); }
 ts_moe_status ts_moe_debug_skew_barrier(ts_moe* h, void* stream) {
   if (!h) return TS_MOE_EINVAL;
   TSM_CUDA(h, cudaSetDevice(h->cfg.device));

@@ -9,20 +9,20 @@ Block formats (the byte layouts the library's C ABI accepts):
 
 * Q8_0, 34 bytes per 32 weights: ``{uint16 d (IEEE fp16 bits, little endian);
   int8 q[32]}``; element i of the block is ``d * q[i]``.  The pages fix only
-  that the Q8_0 dots walk whole 32-element blocks (deepseek2 state page,
-  ``build``: "the Q8_0 dots walk whole 32-element blocks").
+  that Q8_0 dot products step over 32-element blocks (deepseek2 state page,
+  ``build``).
 * MXFP4, 17 bytes per 32 weights: ``{uint8 e (E8M0 scale 2^(e-127));
   uint8 qs[16]}``; element 2j is the low nibble of ``qs[j]``, element 2j+1 the
   high nibble; each nibble is an E2M1 code (sign bit 3, magnitudes
-  0, .5, 1, 1.5, 2, 3, 4, 6).  The gpt-oss state page names the format
-  ("MXFP4 routed pair"); the nibble order is this library's reading.
+  0, .5, 1, 1.5, 2, 3, 4, 6).  The gpt-oss state page names MXFP4 as the
+  format of its routed experts; the nibble order is this library's reading.
 * INT4-affine, 20 bytes per 32 weights: ``{uint16 d; uint16 m (IEEE fp16
   bits); uint8 qs[16]}``; element 2j is the low nibble of ``qs[j]``, element
   2j+1 the high nibble; each nibble is an unsigned code q in [0, 15] and the
-  weight is ``d * q + m``.  The llama state page only names the format
-  ("that seam is INT4-affine only"); block size, field types and layout are
-  this library's reading, matched to the 32-element blocks of the others.
-  The oracle defines it; the CUDA library does not accept it yet.
+  weight is ``d * q + m``.  The gpt-oss state page only names the format
+  (`BatchedRoutedScratch`: the batched-GEMV seam takes INT4-affine tensors
+  only); block size, field types and layout are this library's reading,
+  matched to the 32-element blocks of the others.
 
 Matrices are row-major in blocks: a ``[R][C]`` matrix is R rows of C/32 blocks.
 Expert tensors stack E such matrices: gate/up ``[E][I][H]``, down ``[E][H][I]``.

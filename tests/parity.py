@@ -37,11 +37,7 @@ class ParityReport:
     idx_equal: bool
 
 
-def nthreads() -> int:
-    try:
-        return max(1, len(os.sched_getaffinity(0)))
-    except Exception:
-        return os.cpu_count() or 1
+nthreads = O.nthreads
 
 
 def host_layer(L: synth.LayerBlobs) -> dict:
@@ -126,16 +122,18 @@ def run_layer(moe, shape, layer: int, x: torch.Tensor, resid: torch.Tensor):
             out.float().cpu().numpy())
 
 
-def check_shape(shape, M: int, device="cuda", layer: int = 0, rows=None, moe=None, layers=None):
-    """Builds (or reuses) a handle for `shape`, runs one layer at M tokens, compares with the oracle."""
+def check_shape(shape, M: int, device="cuda", layer: int = 0, rows=None, moe=None, layers=None, gen_device=None):
+    """Builds (or reuses) a handle for `shape`, runs one layer at M tokens, compares with the oracle.
+    Inputs are drawn on `gen_device` (default: `device`) and copied to `device`."""
     from quantized_moe_routed_router_b200 import binding
+    gen = gen_device or device
     if layers is None:
-        layers = [synth.make_layer(shape, l, device=device) for l in range(shape.num_layers)]
+        layers = [synth.make_layer(shape, l, device=gen) for l in range(shape.num_layers)]
     own = moe is None
     if own:
         moe = binding.MoE(shape, layers)
-    x = synth.make_x(shape, layer, M, device=device)
-    resid = synth.make_x(shape, layer, M, device=device, tensor=synth.T_RESID)
+    x = synth.make_x(shape, layer, M, device=gen).to(device)
+    resid = synth.make_x(shape, layer, M, device=gen, tensor=synth.T_RESID).to(device)
     idx, w, lg, y, out = run_layer(moe, shape, layer, x, resid)
     rep = compare(shape, layers[layer].host_numpy(), x, resid, idx, w, y, out, lg, rows=rows)
     if own:

@@ -216,3 +216,16 @@ def test_header_constants_match_the_binding_and_the_generator(B):
     assert (h["TS_ACT_SWIGLU"], h["TS_ACT_SWIGLU_CLAMPED"]) == (synth.ACT_SWIGLU, synth.ACT_SWIGLU_CLAMPED)
     assert (h["TS_MOE_MAX_TOKENS"], h["TS_MOE_MAX_TOPK"], h["TS_MOE_MAX_EXPERTS"]) == (16, 8, 256)
     assert h["TS_MOE_OK"] == 0 and h["TS_MOE_EDEVICE"] == 5
+
+
+def test_coresidency_rule_of_the_layer_kernel(B):
+    """The layer kernel's grid barrier needs every CTA resident at once: open
+    refuses when the occupancy calculator allows none per SM, or fewer than the
+    launch needs (the rule ts_moe_open applies, checked without a GPU)."""
+    lib = B.lib
+    nb = lib.ts_moe_debug_layer_ctas(148)
+    assert nb == 148 and lib.ts_moe_debug_layer_ctas(600) == 512      # one CTA per SM, at most 512
+    assert lib.ts_moe_debug_coresident(1, 148, nb) == 1
+    assert lib.ts_moe_debug_coresident(0, 148, nb) == 0               # does not fit on an SM at all
+    assert lib.ts_moe_debug_coresident(1, 100, nb) == 0               # fewer SMs than CTAs
+    assert lib.ts_moe_debug_coresident(2, 74, nb) == 1

@@ -183,7 +183,9 @@ def test_chunked_prefill_gptoss_full_size_sampled():
 
 # --------------------------------------------------------------------------- the five workloads at full size
 
-@pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 16), (4, 16)])
+# cfg 3 at every M of the benchmark's sweep: the router slicing, the read-back
+# of the router items and the gate/up partition all switch with M
+@pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 2), (3, 4), (3, 8), (3, 16), (4, 16)])
 def test_workload_full_size(cfg, M):
     shape = synth.CONFIGS[cfg]
     if M > shape.max_tokens:
@@ -205,16 +207,17 @@ def test_dense_ffn(name, H, I, fmt, M):
 
 def test_workload_24_layer_stack_sampled():
     """The 24-layer gpt-oss-shaped stack in the launch configuration the
-    benchmark times (one handle, all layers resident, M = 16 and M = 1): every
-    layer's outputs are checked on sampled tokens against the oracle."""
+    benchmark times (one handle, all layers resident) at every M of its sweep
+    (16, 8, 4, 2, 1): every layer's outputs are checked on sampled tokens
+    against the oracle, three layers on the whole micro-batch."""
     from quantized_moe_routed_router_b200 import binding
     shape = synth.CONFIGS[5]
     layers = [synth.make_layer(shape, l, device="cuda") for l in range(shape.num_layers)]
     moe = binding.MoE(shape, layers)
     rng = np.random.default_rng(5)
-    for M in (16, 1):
+    for M in (16, 8, 4, 2, 1):
         for l in range(shape.num_layers):
-            rows = [0] if M == 1 else sorted(rng.choice(16, 2, replace=False).tolist())
+            rows = [0] if M == 1 else sorted(rng.choice(M, 2, replace=False).tolist())
             if l in (0, 11, 23):
                 rows = None                              # whole micro-batch on three layers
             rep = parity.check_shape(shape, M, layer=l, rows=rows, moe=moe, layers=layers)

@@ -1,14 +1,17 @@
 """The allocation-free router entry point (ts_moe_route_noalloc), through the C ABI.
 
-Some callers cannot allocate device memory when they need routing -- code
-running under CUDA-graph stream capture, engines that own all device memory in
-their own pool, plugins handed only a stream and buffers -- so they cannot
-open a handle.  ts_moe_route_noalloc takes the raw router and keeps its scratch
-in the library's static device array.  Here its results are checked against
-the handle-based ts_moe_route on the same router and inputs, on two calls in a
-row (the static scratch keeps the previous call's contents), with the
-tolerances the parity tests use (experts bit-exact, weights within 1e-5,
-logits within 1e-4 of the largest)."""
+Some callers cannot allocate device memory at all -- engines that give every
+byte of device memory to their own pool at start-up, plugins handed only a
+stream and buffers -- so they cannot open a handle (ts_moe_open allocates a
+weight arena and a workspace).  ts_moe_route_noalloc takes the raw router and
+keeps its scratch in the library's static device array.  Its results are
+checked here against the handle-based ts_moe_route on the same router and
+inputs, on two calls in a row (the static scratch keeps the previous call's
+contents), with the tolerances the parity tests use (experts bit-exact, weights
+within 1e-5, logits within 1e-4 of the largest).  Errors the device finds are
+reported in the outputs (every idx -1, every w 0); that path is checked with a
+router whose block scale is NaN and a bias holding NaN, each followed by a good
+call on the same scratch."""
 import numpy as np
 import pytest
 import torch
@@ -60,3 +63,47 @@ def test_route_noalloc_refuses_oversized_scratch():
     with pytest.raises(binding.TsMoeError) as ei:
         binding.route_noalloc(router, None, None, 256, 16384, 8, 0, 0, x, idx, w)
     assert ei.value.status == 1 and "scratch" in str(ei.value)
+
+
+def _route_pair(shape, L, router, bias_d, x):
+    from quantized_moe_routed_router_b200 import binding
+    E, H, K, M = shape.num_experts, shape.hidden, shape.top_k, x.shape[0]
+    idx = torch.full((M, K), 7, dtype=torch.int32, device="cuda")
+    w = torch.full((M, K), 0.5, device="cuda")
+    binding.route_noalloc(router, bias_d, None, E, H, K, shape.score, shape.bias_mode, x, idx, w)
+    torch.cuda.synchronize()
+    return idx, w
+
+
+def test_route_noalloc_reports_device_errors_in_its_outputs():
+    """A NaN router block scale (refused by ts_moe_open, here found on the
+    device) and a NaN bias each turn every idx into -1 and every w into 0; the
+    next good call on the same scratch routes normally again."""
+    from quantized_moe_routed_router_b200 import binding
+    shape = synth.CONFIGS[3].replace(moe_inter=64, max_tokens=16)
+    L = synth.make_layer(shape, 0, device="cuda")
+    moe = binding.MoE(shape, [L])
+    E, K = shape.num_experts, shape.top_k
+    bias_d = torch.from_numpy(L.bias).cuda()
+    x = synth.make_x(shape, 1, 16, device="cuda")
+    ref_idx = torch.empty(16, K, dtype=torch.int32, device="cuda")
+    ref_w = torch.empty(16, K, device="cuda")
+    moe.route(0, x, ref_idx, ref_w)
+
+    bad_router = L.router.clone()
+    bad_router[5, 34 * 3:34 * 3 + 2] = torch.tensor([0x00, 0x7E], dtype=torch.uint8)   # fp16 NaN scale, expert 5 block 3
+    idx, w = _route_pair(shape, L, bad_router, bias_d, x)
+    assert torch.all(idx == -1) and torch.all(w == 0)
+
+    idx, w = _route_pair(shape, L, L.router, bias_d, x)              # the same scratch, good inputs again
+    assert torch.equal(idx, ref_idx) and (w - ref_w).abs().max().item() <= 1e-5
+
+    bad_bias = bias_d.clone()
+    bad_bias[E - 1] = float("nan")
+    idx, w = _route_pair(shape, L, L.router, bad_bias, x)
+    assert torch.all(idx == -1) and torch.all(w == 0)
+
+    idx, w = _route_pair(shape, L, L.router, bias_d, x)
+    assert torch.equal(idx, ref_idx) and (w - ref_w).abs().max().item() <= 1e-5
+    moe.device_status()
+    moe.close()
