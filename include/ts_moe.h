@@ -19,7 +19,10 @@
  *     blocks:  Q8_0 block = { uint16 d (IEEE fp16 bits); int8 q[32] } (34 B),
  *     element i = d * q[i];  MXFP4 block = { uint8 e (E8M0, 2^(e-127));
  *     uint8 qs[16] } (17 B), element 2j = low nibble of qs[j], element 2j+1 =
- *     high nibble, each an E2M1 code (bit 3 sign; magnitudes 0,.5,1,1.5,2,3,4,6).
+ *     high nibble, each an E2M1 code (bit 3 sign; magnitudes 0,.5,1,1.5,2,3,4,6);
+ *     INT4-affine block = { uint16 d; uint16 m (IEEE fp16 bits); uint8 qs[16] }
+ *     (20 B), element 2j = low nibble of qs[j], element 2j+1 = high nibble, each
+ *     an unsigned code q in [0, 15], element = d * q + m.
  *   - BF16 values are passed as their 16-bit patterns (little-endian uint16).
  *   - Every function returns a ts_moe_status; on failure ts_moe_last_error()
  *     gives a one-line reason.  Nothing aborts, prints or throws.
@@ -48,7 +51,10 @@ typedef enum {
   TS_MOE_EDEVICE = 5       /* a kernel reported an error through the device error word */
 } ts_moe_status;
 
-enum { TS_FMT_Q8_0 = 0, TS_FMT_MXFP4 = 1 };
+/* Expert weight formats.  INT4_AFFINE is named by the gpt-oss state page
+ * (`BatchedRoutedScratch`: its batched-GEMV seam takes INT4-affine tensors
+ * only); the block layout above is this library's reading of it. */
+enum { TS_FMT_Q8_0 = 0, TS_FMT_MXFP4 = 1, TS_FMT_INT4_AFFINE = 2 };
 /* Top-k rule.  SOFTMAX_SELECTED: softmax over the K selected experts (llama /
  * gpt-oss state pages, `per_expert_ones`: with unit per-expert scales the
  * weights are exactly that softmax).  SOFTMAX_ALL_NORENORM: softmax over all E experts, the K largest
@@ -81,7 +87,7 @@ typedef struct {
   int32_t top_k;         /* K, 1..min(8, E) */
   int32_t num_layers;    /* layers held by this handle, 1..1024 */
   int32_t max_tokens;    /* largest M any call will pass, 1..65536 (the workspace holds min(max_tokens, 16)) */
-  int32_t expert_fmt;    /* TS_FMT_*; router and shared expert are always Q8_0 */
+  int32_t expert_fmt;    /* TS_FMT_*; router and shared expert are always Q8_0 (a shared expert needs Q8_0 experts) */
   int32_t score;         /* TS_SCORE_* */
   int32_t bias_mode;     /* TS_BIAS_* */
   int32_t act;           /* TS_ACT_* (the shared expert uses the same rule) */
@@ -112,7 +118,8 @@ typedef struct {
 typedef struct ts_moe ts_moe;
 
 /* Validates cfg and layers[0 .. num_layers-1] (shapes, enums, finiteness of
- * the bias, E8M0 = 255 and non-finite Q8_0 scales are refused with
+ * the bias, E8M0 = 255, non-finite Q8_0 scales and non-finite INT4-affine
+ * scales or offsets are refused with
  * TS_MOE_EINVAL; sizes for which the router GEMV cannot be cut into per-CTA
  * items that fit the SM count and shared memory with TS_MOE_EUNSUPPORTED), then on
  * cfg->device allocates the repacked weight arena and the per-call workspace

@@ -40,14 +40,13 @@ int ts_moe_debug_coresident(int per_sm, int sm_count, int nb);
  * message (ts_moe_last_error(NULL)). */
 ts_moe_status ts_moe_debug_validate(const ts_moe_config* cfg, const ts_moe_layer_weights* layers);
 
-/* Failure-path test hook.  Synchronises `stream`, then moves the handle's
- * grid-barrier launch counter two launches ahead of its arrival counter, so
- * that the grid barrier of the next ts_moe_forward cannot complete: every CTA
- * gives up after the bounded wait (2 s), sets the "grid barrier wait gave up"
- * bit (0x40) of the device error word, and the kernel runs to its end.  The
- * next ts_moe_device_status returns TS_MOE_EDEVICE and re-zeroes the
- * counters, after which calls work normally again.  TS_MOE_ECUDA if a copy
- * fails.  Not for production use. */
+/* Failure-path test hook.  Synchronises `stream`, then marks the handle so
+ * that in the next layer-kernel launch CTA 0 does not arrive at the grid
+ * barrier.  The barrier cannot complete: every CTA gives up after the bounded
+ * wait (2 s), sets the "grid barrier wait gave up" bit (0x40) of the device
+ * error word, and the kernel runs to its end.  The next ts_moe_device_status
+ * returns TS_MOE_EDEVICE and re-zeroes the counters, after which calls work
+ * normally again.  Not for production use. */
 ts_moe_status ts_moe_debug_skew_barrier(ts_moe* h, void* stream);
 
 #ifdef __cplusplus

@@ -135,6 +135,27 @@ TSM_DEV float2 ld_cg2(const float* p) {
   asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
   return v;
 }
+TSM_DEV unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+// Adds v at gpu scope with release semantics (this thread's earlier writes, and
+// those ordered before them by a CTA barrier, are visible before the add); no
+// value comes back, so the thread does not wait for the round trip.
+TSM_DEV void red_release_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+TSM_DEV void red_release_add_u32(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Atomic add at gpu scope with acquire-release semantics: earlier writes are
+// published with it, and writes published by the adds it reads are visible after.
+TSM_DEV unsigned atom_acq_rel_add_u32(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 TSM_DEV unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -186,6 +207,21 @@ TSM_DEV uint32_t u8x2_to_f16x2(uint32_t w) {
   const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
   h = __hsub2(h, off);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// INT4-affine codes: a word of eight nibbles (layout in repack.cuh) to the
+// four f16x2 A registers by masks alone.  Nibbles 0/4 masked into the
+// mantissas of 0x6400 (1024) give 1024 + q, nibbles 1/5 give 1024 + 16 q, and
+// the word shifted right by 8 gives nibbles 2/6 and 3/7 the same way.  The
+// registers of tile row g (0 and 2) hold 1024 + q, those of row g + 8 (1 and
+// 3) hold 1024 + 16 q, both exact; the consumer removes the 1024 and the 16
+// per row with the block's column sums (see mma_chunk).
+TSM_DEV void i4x8_to_f16x8_biased(uint32_t w, uint32_t (&out)[4]) {
+  const uint32_t w8 = w >> 8;
+  out[0] = (w & 0x000F000Fu) | 0x64006400u;
+  out[1] = (w & 0x00F000F0u) | 0x64006400u;
+  out[2] = (w8 & 0x000F000Fu) | 0x64006400u;
+  out[3] = (w8 & 0x00F000F0u) | 0x64006400u;
 }
 
 // E8M0 byte `k` of w as an FP32 power of two (2^(e-127)); e = 0 maps to 0.0

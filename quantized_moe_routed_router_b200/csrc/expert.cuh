@@ -41,7 +41,10 @@ namespace tsm {
 constexpr int NWC = 15;                    // consumer warps
 constexpr int RW = 2;                      // tiles per consumer warp
 constexpr int NTHREADS = (NWC + 1) * 32;   // + one producer warp
-constexpr int KS = 2;                      // chunks per weight stage
+constexpr int KS = 2;                      // chunks per weight stage (Q8_0, MXFP4)
+constexpr int KS_I4 = 3;                   // chunks per weight stage (INT4-affine: 320-byte units)
+template <int FMT> constexpr int stage_chunks() { return FMT == FMT_INT4_AFFINE ? KS_I4 : KS; }
+template <int FMT> constexpr int unit_b() { return FMT == FMT_INT4_AFFINE ? UNIT_BYTES_I4 : UNIT_BYTES; }
 constexpr int NSW = 4;                     // weight stages in the ring
 constexpr int NSX = 2;                     // activation windows in the ring
 constexpr int KW = 512;                    // K elements per activation window
@@ -51,6 +54,7 @@ constexpr int XWIN = 16 * XROW;
 constexpr int SLOT_FLOATS = GS_MAX * 16 * 16;
 constexpr int MAX_NB = 512;                // CTAs per launch (one per SM)
 static_assert(GS_MAX == NWC * RW, "a group is one tile per consumer-warp slot");
+static_assert(GS_MAX * KS_I4 * UNIT_BYTES_I4 <= WSTAGE, "an INT4-affine stage fits the weight ring");
 static_assert(ROUTE_WARPS <= NWC + 1, "routing uses the first ROUTE_WARPS warps");
 
 struct LayerParams {
@@ -76,8 +80,8 @@ struct LayerParams {
   unsigned* cnt_group;      // [(E+1) * ng_max * NWC] gate/up chunk counters per (entry, group, consumer warp)
   int ng_max;
   unsigned* entry_done;     // [E+1] gate/up (group, consumer warp) shares finished per expert (+ shared)
-  unsigned* grid_cnt;       // grid barrier arrivals, never reset: NB per launch
-  unsigned* grid_gen;       // launches completed (the last arriver of each grid barrier adds 1)
+  unsigned long long* grid_cnt;  // grid barrier arrivals, never reset: NB per launch (64-bit: never wraps)
+  int debug_skip_arrival;   // test hook: CTA 0 does not arrive, so the barrier's bounded wait runs out
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
   unsigned* err;
@@ -90,12 +94,10 @@ struct __align__(128) LayerSmem {
   uint8_t x[NSX][XWIN];
   uint64_t wfull[NSW], wempty[NSW], xfull[NSX], xempty[NSX];
   RouteState r;
-  long long upre0[MAX_ENTRIES + 1];  // gate/up: first unit of each entry (entry-major)
-  int cpre1[MAX_ENTRIES + 1];        // down: first unit of each entry inside a group (group-major)
-  unsigned rs0[MAX_NB + 1];          // first unit of each CTA's range, per phase
-  unsigned rs1[MAX_NB + 1];
+  unsigned rs0[MAX_NB + 1];          // gate/up: first unit of each CTA's range
+  unsigned rs1[MAX_NB + 1];          // down: first unit of each CTA's range
   int dead;
-  unsigned gen0;
+  unsigned long long gen0;  // launches completed before this one
 };
 
 struct Seg {
@@ -107,6 +109,28 @@ struct Seg {
   long long g0;   // unit index of the (entry, group)'s first chunk
 };
 
+// First unit of entry j (touched experts, then the shared expert as entry nT):
+// gate/up units are entry-major, so entry j starts at upre0(j); down units are
+// group-major, and inside a group entry j starts at cpre1(j).
+TSM_DEV long long upre0(const LayerParams& p, int nT, int j) {
+  return (long long)min(j, nT) * p.gB.ngroups * p.gB.chunks + (j > nT ? (long long)p.gBs.ngroups * p.gBs.chunks : 0);
+}
+TSM_DEV int cpre1(const LayerParams& p, int nT, int j) { return min(j, nT) * p.gC.chunks + (j > nT ? p.gCs.chunks : 0); }
+
+// First unit of CTA b's range in phase PH (b = NB: the total), from the unit
+// counts alone: plain contiguous ranges, or for gate/up with few groups the
+// group-aligned partition (aligned_* in layout.cuh).
+template <int PH>
+TSM_DEV unsigned cta_start(const LayerParams& p, int nT, int nE, int NB, bool aligned, int G0, int b) {
+  if (PH == 1) return (unsigned)range_start((uint64_t)p.gC.ngroups * cpre1(p, nT, nE), NB, b);
+  if (!aligned || b >= NB) return (unsigned)range_start((uint64_t)upre0(p, nT, nE), NB, b);
+  const int g = aligned_group_of(b, G0, NB);
+  const bool shg = g >= nT * p.gB.ngroups;
+  const int j = shg ? nT : g / p.gB.ngroups, grp = shg ? g - nT * p.gB.ngroups : g % p.gB.ngroups;
+  const int ch = shg ? p.gBs.chunks : p.gB.chunks;
+  return (unsigned)(upre0(p, nT, j) + (long long)grp * ch + aligned_offset(b, G0, NB, ch));
+}
+
 // Next segment (one entry's group, a run of its chunks) of [u, u1) of phase PH
 // (0: entry-major gate/up units, 1: group-major down units).
 template <int PH>
@@ -114,24 +138,27 @@ TSM_DEV bool next_seg(const LayerSmem& s, const LayerParams& p, long long& u, lo
   if (u >= u1) return false;
   const MatGeom& gr = PH == 0 ? p.gB : p.gC;
   const MatGeom& gsh = PH == 0 ? p.gBs : p.gCs;
+  const int nT = s.r.nT;
+  // unit indices fit in 32 bits (at most 257 entries x 546 groups x 512 chunks)
+  const unsigned uu = (unsigned)u;
   int grp, c0;
-  long long base;
+  unsigned base;
   if (PH == 1) {
-    const int upg = s.cpre1[s.r.nE];
-    grp = (int)(u / upg);
-    const int r = (int)(u - (long long)grp * upg);
-    j = 0;
-    while (r >= s.cpre1[j + 1]) ++j;
-    c0 = r - s.cpre1[j];
-    base = (long long)grp * upg + s.cpre1[j];
+    const unsigned upg = (unsigned)cpre1(p, nT, s.r.nE);
+    grp = (int)(uu / upg);
+    const int r = (int)(uu - (unsigned)grp * upg);
+    j = r < nT * gr.chunks ? r / gr.chunks : nT;
+    c0 = r - cpre1(p, nT, j);
+    base = (unsigned)grp * upg + (unsigned)cpre1(p, nT, j);
   } else {
-    while (u >= s.upre0[j + 1]) ++j;
-    const bool sh = p.rp.has_shared && j == s.r.nT;
-    const int chunks = sh ? gsh.chunks : gr.chunks;
-    const long long local = u - s.upre0[j];
-    grp = (int)(local / chunks);
-    c0 = (int)(local - (long long)grp * chunks);
-    base = s.upre0[j] + (long long)grp * chunks;
+    const unsigned ub = (unsigned)(gr.ngroups * gr.chunks);
+    j = uu < (unsigned)nT * ub ? (int)(uu / ub) : nT;
+    const bool sh = p.rp.has_shared && j == nT;
+    const unsigned chunks = (unsigned)(sh ? gsh.chunks : gr.chunks);
+    const unsigned e0 = (unsigned)upre0(p, nT, j);
+    grp = (int)((uu - e0) / chunks);
+    c0 = (int)(uu - e0 - (unsigned)grp * chunks);
+    base = e0 + (unsigned)grp * chunks;
   }
   sg.j = j;
   sg.sh = p.rp.has_shared && j == s.r.nT;
@@ -178,7 +205,8 @@ TSM_DEV float act_fn(int act, float alpha, float limit, float g, float u) {
 template <int FMT, int NT, bool FULL = false>
 TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, int warp, const uint8_t* xc,
                        int lane) {
-  constexpr int STEPS = FMT == 1 ? 4 : 2;
+  constexpr int STEPS = FMT == FMT_MXFP4 ? 4 : 2;
+  constexpr int UB = unit_b<FMT>();
   const int g = lane >> 2, c = lane & 3;
   uint32_t b[STEPS][NT][2];
 #pragma unroll
@@ -189,14 +217,55 @@ TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, i
       b[s][nt][0] = v.x;
       b[s][nt][1] = v.y;
     }
+  // INT4-affine: the block's column sums of B (an MMA with an all-ones A), for
+  // the offset term m * sum(x); lane (g, c) gets columns 2c, 2c + 1 in [0], [1]
+  float csum[NT][4];
+  if constexpr (FMT == FMT_INT4_AFFINE) {
+    const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      mma_f16_zc(csum[nt], ones, b[0][nt][0], b[0][nt][1]);
+      mma_f16_acc(csum[nt], ones, b[1][nt][0], b[1][nt][1]);
+    }
+  }
 #pragma unroll
   for (int r = 0; r < RW; ++r) {
     const int jt = warp * RW + r;
     if (!FULL && jt >= ntg) break;
-    const uint8_t* t = chunk + jt * UNIT_BYTES;
+    const uint8_t* t = chunk + jt * UB;
+    if constexpr (FMT == FMT_INT4_AFFINE) {
+      // One block.  The MMA gives D = sum((1024 + q) x) = 1024 S + Q for row g
+      // and sum((1024 + 16 q) x) = 1024 S + 16 Q for row g + 8 (S = sum(x), Q =
+      // sum(q x)), so d Q + m S = d D + (m - 1024 d) S for row g and
+      // (d / 16) D + (m - 64 d) S for row g + 8.
+      const uint2 qw = *reinterpret_cast<const uint2*>(t + lane * 8);
+      const uint2 dm = *reinterpret_cast<const uint2*>(t + QUANT_BYTES_I4 + g * 8);
+      float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dm.x));
+      float2 m = __half22float2(*reinterpret_cast<const __half2*>(&dm.y));
+      m.x = fmaf(-1024.f, d.x, m.x);
+      m.y = fmaf(-64.f, d.y, m.y);
+      d.y *= 0.0625f;
+      uint32_t a0[4], a1[4];
+      i4x8_to_f16x8_biased(qw.x, a0);
+      i4x8_to_f16x8_biased(qw.y, a1);
+      float tmp[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_f16_zc(tmp[nt], a0, b[0][nt][0], b[0][nt][1]);
+        mma_f16_acc(tmp[nt], a1, b[1][nt][0], b[1][nt][1]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        acc[r][nt][0] = fmaf(d.x, tmp[nt][0], fmaf(m.x, csum[nt][0], acc[r][nt][0]));
+        acc[r][nt][1] = fmaf(d.x, tmp[nt][1], fmaf(m.x, csum[nt][1], acc[r][nt][1]));
+        acc[r][nt][2] = fmaf(d.y, tmp[nt][2], fmaf(m.y, csum[nt][0], acc[r][nt][2]));
+        acc[r][nt][3] = fmaf(d.y, tmp[nt][3], fmaf(m.y, csum[nt][1], acc[r][nt][3]));
+      }
+      continue;
+    }
     const uint4 q = *reinterpret_cast<const uint4*>(t + lane * 16);
     const uint32_t sc = *reinterpret_cast<const uint32_t*>(t + QUANT_BYTES + g * 4);
-    if constexpr (FMT == 1) {
+    if constexpr (FMT == FMT_MXFP4) {
       const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
@@ -245,34 +314,61 @@ TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, i
 TSM_DEV unsigned down_owners(const LayerSmem& s, const LayerParams& p, int NB, int grp, int j) {
   const bool sh = p.rp.has_shared && j == s.r.nT;
   const unsigned C = (unsigned)(sh ? p.gCs.chunks : p.gC.chunks);
-  const unsigned g0 = (unsigned)grp * (unsigned)s.cpre1[s.r.nE] + (unsigned)s.cpre1[j];
+  const unsigned g0 = (unsigned)grp * (unsigned)cpre1(p, s.r.nT, s.r.nE) + (unsigned)cpre1(p, s.r.nT, j);
   return (unsigned)owner_tab(s.rs1, NB, g0) | ((unsigned)owner_tab(s.rs1, NB, g0 + C - 1) << 16);
 }
 
-// Value of the down output of entry j, column n, row h (row group `grp`):
-// written to P when one CTA covered the whole (group, entry) segment, else
-// the sum of the contributing CTAs' partial slots in CTA order.
-TSM_DEV float down_value(const LayerSmem& s, const LayerParams& p, unsigned owners, int grp, int gs, int j, int n,
+// Loads of the down output of entry j, column n, row h (row group `grp`): the
+// value written to P when one CTA covered the whole (group, entry) segment,
+// else the contributing CTAs' partial slots, to be added in CTA order.
+// down_loads issues the first DV_LOADS of them (predicated, all in flight
+// together) into t and returns how many it covered; down_rest adds the rest.
+constexpr int DV_LOADS = 4;
+
+struct DownSrc {
+  const float* base;  // P row, or the partial-slot base of contributor bf
+  int bf, bl;         // contributing CTAs (bf == bl: one owner, value in P)
+  unsigned g0;        // first unit of the segment
+  int off;            // element offset inside a partial slot
+};
+
+TSM_DEV DownSrc down_src(const LayerSmem& s, const LayerParams& p, unsigned owners, int grp, int gs, int j, int n,
                          int h, int route) {
-  const int bf = owners & 0xFFFF, bl = owners >> 16;
-  if (bf == bl) return ld_cg(p.P + (size_t)route * p.rp.H + h);
-  const unsigned g0 = (unsigned)grp * (unsigned)s.cpre1[s.r.nE] + (unsigned)s.cpre1[j];
+  DownSrc d;
+  d.bf = owners & 0xFFFF;
+  d.bl = owners >> 16;
+  d.g0 = (unsigned)grp * (unsigned)cpre1(p, s.r.nT, s.r.nE) + (unsigned)cpre1(p, s.r.nT, j);
   const int rel = h - grp * gs * 16;
-  const int off = ((rel >> 4) * 16 + (rel & 15)) * 16 + n;
-  // the contributors' slots in CTA order, four loads in flight at a time
-  float v = 0.f;
-  for (int b2 = bf; b2 <= bl; b2 += 4) {
-    float t[4];
+  d.off = ((rel >> 4) * 16 + (rel & 15)) * 16 + n;
+  d.base = p.P + (size_t)route * p.rp.H + h;
+  return d;
+}
+
+TSM_DEV const float* slot_ptr(const LayerSmem& s, const LayerParams& p, const DownSrc& d, int bb) {
+  return p.partial1 + ((size_t)bb * 2 + (s.rs1[bb] >= d.g0 ? 0 : 1)) * SLOT_FLOATS + d.off;
+}
+
+TSM_DEV void down_loads(const LayerSmem& s, const LayerParams& p, const DownSrc& d, bool use, float (&t)[DV_LOADS]) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int bb = b2 + q;
-      t[q] = 0.f;  // past bl or an empty range: adds nothing
-      if (bb <= bl && s.rs1[bb] != s.rs1[bb + 1])
-        t[q] = ld_cg(p.partial1 + ((size_t)bb * 2 + (s.rs1[bb] >= g0 ? 0 : 1)) * SLOT_FLOATS + off);
+  for (int q = 0; q < DV_LOADS; ++q) {
+    const int bb = d.bf + q;
+    t[q] = 0.f;  // past bl or an empty range: adds nothing
+    if (!use) continue;
+    if (d.bf == d.bl) {
+      if (q == 0) t[q] = ld_cg(d.base);
+    } else if (bb <= d.bl && s.rs1[bb] != s.rs1[bb + 1]) {
+      t[q] = ld_cg(slot_ptr(s, p, d, bb));
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) v += t[q];
   }
+}
+
+TSM_DEV float down_sum(const LayerSmem& s, const LayerParams& p, const DownSrc& d, const float (&t)[DV_LOADS]) {
+  if (d.bf == d.bl) return t[0];
+  float v = 0.f;
+#pragma unroll
+  for (int q = 0; q < DV_LOADS; ++q) v += t[q];
+  for (int bb = d.bf + DV_LOADS; bb <= d.bl; ++bb)  // more contributors than DV_LOADS (small M)
+    if (s.rs1[bb] != s.rs1[bb + 1]) v += ld_cg(slot_ptr(s, p, d, bb));
   return v;
 }
 
@@ -301,125 +397,99 @@ TSM_DEV bool combine_prepare(LayerSmem& s, const LayerParams& p, int NB, int cti
 }
 
 // After the grid barrier: y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared)
-// in slot order over this CTA's slice; resid += y.  The barrier orders the
+// in slot order over this CTA's slice; resid += y.  Two passes, so that the
+// loads of many (output, slot) pairs are in flight together: (1) each pair's
+// down value -- the K slots, then the shared expert -- into the idle weight
+// ring, CB pairs per thread with all of their loads issued before any is
+// used; (2) each output sums its values in slot order.  The barrier orders the
 // owner table written by combine_prepare before its reads here.
 TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid, bool use_tab, float r0) {
+  constexpr int CT = NWC * 32, CB = 2;
   const int K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = p.rp.M * K, nE = s.r.nE;
   const unsigned* tab = reinterpret_cast<const unsigned*>(&s.r.part[0][0][0]);
   int lo, hi;
   combine_range(p, NB, lo, hi);
   const int KP = K + (p.rp.has_shared ? 1 : 0);
-  if ((hi - lo) * KP > 2 * NWC * 32) {
-    // many outputs: one thread per output, its K (+1) values loaded together
-    for (int i = lo + ctid; i < hi; i += NWC * 32) {
-      const int t = i / H, h = i - t * H, grp = h / (gs * 16);
-      float v[MAX_K + 1];
-#pragma unroll
-      for (int k = 0; k < MAX_K; ++k) {
-        v[k] = 0.f;
-        if (k < K) {
-          const int pos = s.r.rpos[t * K + k];
-          const int j = s.r.rj[pos];
-          const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-          v[k] = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
-        }
-      }
-      v[MAX_K] = 0.f;
-      if (p.rp.has_shared) {
-        const int j = s.r.nT;
-        const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-        v[MAX_K] = down_value(s, p, own, grp, gs, j, t, h, MK + t);
-      }
-      float y = 0.f;
-#pragma unroll
-      for (int k = 0; k < MAX_K; ++k)
-        if (k < K) y = fmaf(s.r.w[t * K + k], v[k], y);
-      y += v[MAX_K];
-      if (p.y) p.y[(size_t)t * H + h] = y;
-      if (p.resid) {
-        __nv_bfloat16* r = p.resid + (size_t)t * H + h;
-        *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
-      }
-    }
-    return;
-  }
-  // few outputs (small M): two passes, so the loads of all (output, slot)
-  // pairs are in flight together: (1) each pair's down value -- the K slots,
-  // then the shared expert -- into the idle weight ring; (2) each output sums
-  // its values in slot order (the same operations as above).
   float* vbuf = reinterpret_cast<float*>(&s.w[0][0]);
   const int cap = (int)((sizeof(s.w) + sizeof(s.x)) / sizeof(float)) / KP;  // outputs per batch
   for (int base = lo; base < hi; base += cap) {
-    const int nb = min(cap, hi - base);
-    for (int q = ctid; q < nb * KP; q += NWC * 32) {
-      const int o = q / KP, k = q - o * KP, i = base + o;
-      const int t = i / H, h = i - t * H, grp = h / (gs * 16);
-      float v;
-      if (k < K) {
-        const int pos = s.r.rpos[t * K + k];
-        const int j = s.r.rj[pos];
+    const int nb = min(cap, hi - base), npair = nb * KP;
+    for (int q0 = ctid; q0 < npair; q0 += CT * CB) {
+      DownSrc d[CB];
+      float t[CB][DV_LOADS];
+#pragma unroll
+      for (int u = 0; u < CB; ++u) {
+        const int q = q0 + u * CT;
+        const bool use = q < npair;
+        const int o = use ? q / KP : 0, k = q - o * KP, i = base + o;
+        const int tk = i / H, h = i - tk * H, grp = h / (gs * 16);
+        int j, n, route;
+        if (k < K) {
+          route = s.r.rpos[tk * K + k];
+          j = s.r.rj[route];
+          n = route - s.r.ro[j];
+        } else {
+          j = s.r.nT;
+          n = tk;
+          route = MK + tk;
+        }
         const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-        v = down_value(s, p, own, grp, gs, j, pos - s.r.ro[j], h, pos);
-      } else {
-        const int j = s.r.nT;
-        const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
-        v = down_value(s, p, own, grp, gs, j, t, h, MK + t);
+        d[u] = down_src(s, p, own, grp, gs, j, n, h, route);
+        down_loads(s, p, d[u], use, t[u]);
       }
-      vbuf[q] = v;
+#pragma unroll
+      for (int u = 0; u < CB; ++u) {
+        const int q = q0 + u * CT;
+        if (q < npair) vbuf[q] = down_sum(s, p, d[u], t[u]);
+      }
     }
-    bar_sync(1, NWC * 32);
-    for (int o = ctid; o < nb; o += NWC * 32) {
-      const int i = base + o, t = i / H, h = i - t * H;
+    bar_sync(1, CT);
+    for (int o = ctid; o < nb; o += CT) {
+      const int i = base + o, tk = i / H, h = i - tk * H;
       float y = 0.f;
-      for (int k = 0; k < K; ++k) y = fmaf(s.r.w[t * K + k], vbuf[o * KP + k], y);
+      for (int k = 0; k < K; ++k) y = fmaf(s.r.w[tk * K + k], vbuf[o * KP + k], y);
       if (p.rp.has_shared) y += vbuf[o * KP + K];
-      if (p.y) p.y[(size_t)t * H + h] = y;
+      if (p.y) p.y[(size_t)tk * H + h] = y;
       if (p.resid) {
-        __nv_bfloat16* r = p.resid + (size_t)t * H + h;
+        __nv_bfloat16* r = p.resid + (size_t)tk * H + h;
         *r = __float2bfloat16_rn((i == lo + ctid ? r0 : __bfloat162float(*r)) + y);
       }
     }
-    bar_sync(1, NWC * 32);  // vbuf is rewritten by the next batch
+    bar_sync(1, CT);  // vbuf is rewritten by the next batch
   }
 }
 
 // Grid-wide barrier among the consumer warps of all CTAs (one CTA per SM, all
-// resident).  The arrival counter is never reset: launch number gen0 (read at
-// the start, before any CTA of this launch can arrive) is complete when it
-// reaches (gen0 + 1) * NB, which every CTA polls directly; the last arriver
-// also advances the launch counter for the next launch.  Bounded: a CTA that
-// waits longer than WAIT_LIMIT_NS records ERR_TIMEOUT_GRID and goes on.
+// resident).  The 64-bit arrival counter is never reset, so launch number
+// gen0 = floor(count / NB) read at the start is right even when other CTAs of
+// this launch have already arrived (at most NB - 1 of them can have), and the
+// launch is complete when the count reaches (gen0 + 1) * NB.  Each CTA arrives
+// with a release reduction (nothing to wait for on the way in) and polls with
+// acquire loads.  Bounded: a CTA that waits longer than WAIT_LIMIT_NS records
+// ERR_TIMEOUT_GRID and goes on.
 TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int ctid) {
-  bar_sync(1, NWC * 32);  // orders every consumer's stores before thread 0's gpu-scope fence
+  bar_sync(1, NWC * 32);  // orders every consumer's stores before thread 0's release
   if (ctid == 0) {
-    __threadfence();
-    const unsigned target = (s.gen0 + 1u) * (unsigned)NB;
-    if (atomicAdd(p.grid_cnt, 1u) + 1u == target) {
-      atomicAdd(p.grid_gen, 1u);
-    } else {
-      const unsigned long long t0 = globaltimer();
-      while ((int)(ld_acquire_u32(p.grid_cnt) - target) < 0) {
-        if (globaltimer() - t0 > WAIT_LIMIT_NS) {
-          atomicOr(p.err, ERR_TIMEOUT_GRID);
-          break;
-        }
+    if (!(p.debug_skip_arrival && blockIdx.x == 0)) red_release_add_u64(p.grid_cnt, 1ull);
+    const unsigned long long target = (s.gen0 + 1ull) * (unsigned long long)NB;
+    const unsigned long long t0 = globaltimer();
+    while (ld_acquire_u64(p.grid_cnt) < target) {
+      if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+        atomicOr(p.err, ERR_TIMEOUT_GRID);
+        break;
       }
     }
   }
-  bar_sync(1, NWC * 32);
-  __threadfence();
+  bar_sync(1, NWC * 32);  // thread 0's acquire, then the CTA barrier, orders the other CTAs' writes before our reads
 }
 
 // A warp's share of a finished gate/up group (its tiles' acts written):
 // count it for the entry.  __syncwarp orders the warp's stores before lane
-// 0's gpu-scope fence (cumulative) and increment; an entry is complete when
-// its count reaches ngroups * NWC.
+// 0's release increment (cumulative, so the whole warp's acts are published
+// with it); an entry is complete when its count reaches ngroups * NWC.
 TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int lane) {
   __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    atomicAdd(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
-  }
+  if (lane == 0) red_release_add_u32(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
 }
 
 // Group epilogue with complete sums in acc.
@@ -473,8 +543,9 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
 template <int FMT, int PH, int NT>
 TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int& wi, int& wph, int& xi, int& xph,
                          int warp, int lane, int ctid, int NB) {
-  constexpr int KC = FMT == 1 ? 64 : 32;
+  constexpr int KC = FMT == FMT_MXFP4 ? 64 : 32;
   constexpr int KWC = KW / KC;
+  constexpr int KS = stage_chunks<FMT>(), UB = unit_b<FMT>();
   float acc[RW][NT][4];
 #pragma unroll
   for (int r = 0; r < RW; ++r)
@@ -492,12 +563,12 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
       if (kk == KS && sg.ntg == GS_MAX) {  // whole stage of a whole group: no guards
 #pragma unroll
         for (int q = 0; q < KS; ++q)
-          mma_chunk<FMT, NT, true>(acc, st + q * GS_MAX * UNIT_BYTES, GS_MAX, warp, xw + (k + q - ws) * KC * 2, lane);
+          mma_chunk<FMT, NT, true>(acc, st + q * GS_MAX * UB, GS_MAX, warp, xw + (k + q - ws) * KC * 2, lane);
       } else {
 #pragma unroll
         for (int q = 0; q < KS; ++q)
           if (q < kk)
-            mma_chunk<FMT, NT>(acc, st + q * sg.ntg * UNIT_BYTES, sg.ntg, warp, xw + (k + q - ws) * KC * 2, lane);
+            mma_chunk<FMT, NT>(acc, st + q * sg.ntg * UB, sg.ntg, warp, xw + (k + q - ws) * KC * 2, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.wempty[wi]);
@@ -542,17 +613,18 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
   if (PH == 1) return;  // down partials are combined after the grid barrier
   // gate/up: per warp (its own tiles), the last contributing CTA finishes the
   // group.  __syncwarp orders the warp's partial stores before lane 0's
-  // gpu-scope fence and chunk count; no other warp of the CTA waits.
+  // acquire-release chunk count, which publishes them and, for the last
+  // contributor, makes the others' slots visible; the second __syncwarp
+  // orders the other lanes' reads after it.  No other warp of the CTA waits.
   const unsigned key = ((unsigned)(sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp) * NWC + warp;
   __syncwarp();
   unsigned last = 0;
   if (lane == 0) {
-    __threadfence();
     const unsigned inc = (unsigned)(sg.c1 - sg.c0);
-    last = atomicAdd(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks;
+    last = atom_acq_rel_add_u32(p.cnt_group + key, inc) + inc == (unsigned)sg.chunks;
   }
+  __syncwarp();
   if (!__shfl_sync(0xffffffffu, last, 0)) return;
-  __threadfence();  // the other contributors' slots, published before their counts
 #pragma unroll
   for (int r = 0; r < RW; ++r)
 #pragma unroll
@@ -604,8 +676,9 @@ template <int FMT, int PH>
 TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, long long u1, int& wi, int& wph, int& xi,
                            int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_src,
                            bool xh_wait) {
-  constexpr int KC = FMT == 1 ? 64 : 32;
+  constexpr int KC = FMT == FMT_MXFP4 ? 64 : 32;
   constexpr int KWC = KW / KC;
+  constexpr int KS = stage_chunks<FMT>(), UB = unit_b<FMT>();
   long long u = u0;
   int j = 0;
   Seg sg;
@@ -613,7 +686,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
   while (alive && next_seg<PH>(s, p, u, u1, j, sg)) {
     const uint8_t* mat = PH == 0 ? (sg.sh ? p.wBs : p.wB + (uint64_t)s.r.ex[sg.j] * p.wB_stride)
                                  : (sg.sh ? p.wCs : p.wC + (uint64_t)s.r.ex[sg.j] * p.wC_stride);
-    const uint8_t* gbase = mat + group_offset(sg.gs, sg.chunks, sg.grp);
+    const uint8_t* gbase = mat + group_offset(sg.gs, sg.chunks, sg.grp, UB);  // (a shared expert only with Q8_0)
     const __half* brow = nullptr;
     if (lane < sg.nc) {
       if (PH == 0)
@@ -621,7 +694,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
       else
         brow = sg.sh ? p.acts_sh + (size_t)lane * p.Sp : p.acts + (size_t)(sg.ro + lane) * p.Ip;
     }
-    const unsigned ustride = (unsigned)sg.ntg * UNIT_BYTES;
+    const unsigned ustride = (unsigned)sg.ntg * UB;
     int k_issued = sg.c0;  // first chunk whose weight stage is not yet issued
     for (int ws = sg.c0; alive && ws < sg.c1;) {
       const int we = min(sg.c1, (ws / KWC + 1) * KWC);
@@ -661,9 +734,8 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
         xh_wait = false;
         alive = __shfl_sync(0xffffffffu, alive && !s.dead, 0);
         if (!alive) break;
-        // the data were written through the generic proxy by other CTAs; the
-        // bulk copies below read them through the async proxy
-        __threadfence();
+        // the data were written through the generic proxy by other CTAs and
+        // acquired above; the bulk copies below read them through the async proxy
         fence_proxy_async_global();
       }
       const unsigned xbytes = (unsigned)(we - ws) * KC * 2;
@@ -756,7 +828,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   grid_dep_launch();
   if (tid == 0) {
     if (rcta) slice_issue_x(rp, s.r, rcs, xs);
-    s.gen0 = ld_acquire_u32(p.grid_gen);
+    // floor(count / NB), exact in FP64 for counts below 2^53 (no 64-bit integer division)
+    s.gen0 = (unsigned long long)floor((double)ld_acquire_u64(p.grid_cnt) / (double)NB);
   }
   route_init_smem(s.r, rc, tid);
   __syncthreads();
@@ -773,9 +846,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     else
       slice_gemv<1>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
     if (rj == 0 && tid < rp.M) p.max_pub[rcs * MAX_TOK + tid] = s.r.smax[tid];
-    __threadfence();
     __syncthreads();
-    if (tid == 0) atomicAdd(p.route_cnt, 1u);
+    if (tid == 0) red_release_add_u32(p.route_cnt, 1u);  // publishes the item written by the whole CTA
   }
   // every item published (bounded); then the S items and slice maxima are
   // brought in by two bulk copies when they fit past the item buffers
@@ -828,44 +900,23 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // gate/up B operand: this CTA's slice of x as FP16, published with the count of slices written
   __half* xh_src = p.xh;
   const bool xwriter = rcta && rj == 0;
-  if (xwriter) {
-    slice_xh(rp, s.r, rcs, xs, xh_src, tid, NTHREADS);
-    __threadfence();
-  }
+  if (xwriter) slice_xh(rp, s.r, rcs, xs, xh_src, tid, NTHREADS);
   route_topk(rp, s.r, warp, lane);
   __syncthreads();
-  if (xwriter && tid == 0) atomicAdd(p.xh_cnt, 1u);
+  if (xwriter && tid == 0) red_release_add_u32(p.xh_cnt, 1u);  // after the barrier: the CTA's slice of xh
   route_list(rp, s.r, warp, lane, tid, NTHREADS);
   fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
 
-  // ---- unit prefixes and the per-phase CTA ranges
+  // ---- this CTA's ranges of both phases, in closed form, so the producer
+  // starts at once; the consumer warps tabulate every CTA's range starts (for
+  // the owners of split groups and the combine) while the first stages load
   const int nE = s.r.nE, nT = s.r.nT;
   const bool hs = rp.has_shared != 0;
-  const long long units_b = (long long)p.gB.ngroups * p.gB.chunks;
-  for (int j = tid; j <= nE; j += NTHREADS) {
-    s.upre0[j] = (long long)min(j, nT) * units_b + (j > nT ? (long long)p.gBs.ngroups * p.gBs.chunks : 0);
-    s.cpre1[j] = min(j, nT) * p.gC.chunks + (j > nT ? p.gCs.chunks : 0);
-  }
-  __syncthreads();
-  const long long U0 = s.upre0[nE];
-  const long long U1 = (long long)p.gC.ngroups * s.cpre1[nE];
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
   const int G0 = nT * p.gB.ngroups + (hs ? p.gBs.ngroups : 0);
   const bool aligned = use_aligned(G0, NB);
-  for (int i = tid; i <= NB; i += NTHREADS) {
-    if (aligned && i < NB) {
-      const int g = aligned_group_of(i, G0, NB);
-      const bool shg = g >= nT * p.gB.ngroups;
-      const int j = shg ? nT : g / p.gB.ngroups, grp = shg ? g - nT * p.gB.ngroups : g % p.gB.ngroups;
-      const int ch = shg ? p.gBs.chunks : p.gB.chunks;
-      s.rs0[i] = (unsigned)(s.upre0[j] + (long long)grp * ch + aligned_offset(i, G0, NB, ch));
-    } else {
-      s.rs0[i] = (unsigned)range_start((uint64_t)U0, NB, i);
-    }
-    s.rs1[i] = (unsigned)range_start((uint64_t)U1, NB, i);
-  }
-  __syncthreads();
-  const long long a0 = s.rs0[b], a1 = s.rs0[b + 1], d0 = s.rs1[b], d1 = s.rs1[b + 1];
+  const long long a0 = cta_start<0>(p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0>(p, nT, nE, NB, aligned, G0, b + 1);
+  const long long d0 = cta_start<1>(p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1>(p, nT, nE, NB, aligned, G0, b + 1);
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
@@ -894,6 +945,11 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   }
 
   // ------------------------------------------------------------ consumer warps
+  for (int i = tid; i <= NB; i += NWC * 32) {
+    s.rs0[i] = cta_start<0>(p, nT, nE, NB, aligned, G0, i);
+    s.rs1[i] = cta_start<1>(p, nT, nE, NB, aligned, G0, i);
+  }
+  bar_sync(1, NWC * 32);
   int wi = 0, wph = 0, xi = 0, xph = 0;
   {
     long long u = a0;

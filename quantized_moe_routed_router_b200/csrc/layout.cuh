@@ -5,10 +5,14 @@
 //   0..7) with the same 8 rows of up (tile rows 8..15), so one thread holds
 //   gate and up of the same act row and forms the activation in registers.
 //   Down tiles are 16 consecutive rows of the [H][I] matrix.
-//   K is cut into chunks of KC elements (64 for MXFP4, 32 for Q8_0); one
-//   (tile, chunk) unit is 544 bytes: 512 bytes of quants, lane l of a warp
-//   owning bytes [16 l, 16 l + 16) (its whole A fragment for the chunk),
-//   followed by 32 bytes of block scales, 4 per lane quad.
+//   K is cut into chunks of KC elements (64 for MXFP4, 32 for Q8_0 and
+//   INT4-affine).  One (tile, chunk) unit of Q8_0 or MXFP4 is 544 bytes: 512
+//   bytes of quants, lane l of a warp owning bytes [16 l, 16 l + 16) (its
+//   whole A fragment for the chunk), followed by 32 bytes of block scales, 4
+//   per lane quad.  An INT4-affine unit is 320 bytes: 256 bytes of 4-bit codes
+//   (lane l owns bytes [8 l, 8 l + 8)), then per lane quad g the fp16 scales
+//   and offsets {d(g), d(g+8), m(g), m(g+8)} (8 bytes).  Every format's unit
+//   holds as many bytes as the user blocks it comes from.
 //   Tiles are grouped (GS tiles per group, the last group may be short) and a
 //   group is stored chunk-major: [chunk][tile in group][544 B], so any run of
 //   chunks of one group is one contiguous range -- one bulk copy.
@@ -21,15 +25,19 @@
 
 namespace tsm {
 
-constexpr int UNIT_BYTES = 544;       // one (tile, chunk): 512 B quants + 32 B scales
+constexpr int UNIT_BYTES = 544;       // one Q8_0 / MXFP4 (tile, chunk): 512 B quants + 32 B scales
 constexpr int QUANT_BYTES = 512;
+constexpr int UNIT_BYTES_I4 = 320;    // one INT4-affine (tile, chunk): 256 B codes + 64 B scales and offsets
+constexpr int QUANT_BYTES_I4 = 256;
+enum { FMT_Q8_0 = 0, FMT_MXFP4 = 1, FMT_INT4_AFFINE = 2 };
 constexpr int GS_MAX = 30;            // tiles per group (= consumer warps x tiles per warp)
 constexpr int MAX_TOK = 16;
 constexpr int MAX_K = 8;
 constexpr int MAX_E = 256;
 constexpr int MAX_ENTRIES = MAX_E + 1;  // touched routed experts + the shared pseudo-expert
 
-TSM_HD int chunk_k(int fmt) { return fmt == 1 ? 64 : 32; }  // elements of K per chunk
+TSM_HD int chunk_k(int fmt) { return fmt == FMT_MXFP4 ? 64 : 32; }  // elements of K per chunk
+TSM_HD int unit_bytes(int fmt) { return fmt == FMT_INT4_AFFINE ? UNIT_BYTES_I4 : UNIT_BYTES; }
 TSM_HD int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
 struct MatGeom {
@@ -38,8 +46,9 @@ struct MatGeom {
   int gs;          // tiles per group
   int ngroups;     // groups per expert
   int kdim;        // K (unpadded)
-  int fmt;         // 0 Q8_0, 1 MXFP4
-  uint64_t bytes;  // bytes per expert matrix = tiles * chunks * 544
+  int fmt;         // FMT_*
+  int ub;          // bytes per (tile, chunk) unit
+  uint64_t bytes;  // bytes per expert matrix = tiles * chunks * ub
 };
 
 // Tiles per group: the group is one tile per consumer-warp slot (GS_MAX), so
@@ -68,7 +77,8 @@ inline MatGeom make_geom(int rows_tiles, int kdim, int fmt) {
   m.chunks = (kdim + chunk_k(fmt) - 1) / chunk_k(fmt);
   m.gs = pick_group_size(rows_tiles);
   m.ngroups = (rows_tiles + m.gs - 1) / m.gs;
-  m.bytes = (uint64_t)rows_tiles * m.chunks * UNIT_BYTES;
+  m.ub = unit_bytes(fmt);
+  m.bytes = (uint64_t)rows_tiles * m.chunks * m.ub;
   return m;
 }
 
@@ -81,7 +91,7 @@ inline MatGeom make_router_geom(int num_experts, int kdim) {
   return m;
 }
 
-TSM_HD uint64_t group_offset(int gs, int chunks, int grp) { return (uint64_t)grp * gs * chunks * UNIT_BYTES; }
+TSM_HD uint64_t group_offset(int gs, int chunks, int grp, int ub) { return (uint64_t)grp * gs * chunks * ub; }
 TSM_HD int group_tiles(int tiles, int gs, int grp) {
   int t = tiles - grp * gs;
   return t < gs ? t : gs;
@@ -92,7 +102,11 @@ TSM_HD int group_tiles(int tiles, int gs, int grp) {
 // entry-major order (entry, group, chunk) for gate/up and group-major order
 // (group, entry, chunk) for down -- are split into NB contiguous ranges:
 // block b owns [range_start(b), range_start(b + 1)).
-TSM_HD uint64_t range_start(uint64_t U, int NB, int b) { return (uint64_t)b * U / (uint64_t)NB; }
+// floor(b * U / NB) through FP64: b * U < 2^53 is exact, the quotient is
+// correctly rounded, and a true quotient below an integer stays at least 1/NB
+// below it, far more than the rounding error, so truncation gives the floor.
+// (A 64-bit integer division is a long software sequence on the GPU.)
+TSM_HD uint64_t range_start(uint64_t U, int NB, int b) { return (uint64_t)((double)b * (double)U / (double)NB); }
 
 // The block whose range contains unit u (0 <= u < U): the largest b with
 // range_start(b) <= u, i.e. floor(((u + 1) * NB - 1) / U).
@@ -106,13 +120,14 @@ TSM_HD int partial_slot(uint64_t U, int NB, int b, uint64_t g0) { return range_s
 // floor(i * G / NB) only, and the CTAs of one group split its chunks evenly,
 // so no CTA carries two partial groups (a CTA that did would finish its second
 // group late and, as its last contributor, also pay for its reduction).
-TSM_HD int aligned_group_of(int i, int G, int NB) { return (int)((long long)i * G / NB); }
-TSM_HD int aligned_first_cta(int g, int G, int NB) { return (int)(((long long)g * NB + G - 1) / G); }
+// (32-bit arithmetic: the aligned partition is used only with G <= NB <= 512.)
+TSM_HD int aligned_group_of(int i, int G, int NB) { return i * G / NB; }
+TSM_HD int aligned_first_cta(int g, int G, int NB) { return (g * NB + G - 1) / G; }
 // First unit of CTA i inside its group of `chunks` units.
 TSM_HD int aligned_offset(int i, int G, int NB, int chunks) {
   const int g = aligned_group_of(i, G, NB);
   const int f = aligned_first_cta(g, G, NB), n = aligned_first_cta(g + 1, G, NB) - f;
-  return (int)((long long)chunks * (i - f) / n);
+  return chunks * (i - f) / n;
 }
 // Used when the busiest CTA then does at most 10 % more than the mean
 // (G <= NB and NB <= 1.1 * G * floor(NB / G)); otherwise plain contiguous ranges.

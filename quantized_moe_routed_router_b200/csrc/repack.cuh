@@ -16,13 +16,21 @@
 //   Q8_0 (2 steps, 32 K): per step two words {row g: q(4c), q(4c+1), row g+8:
 //     q(4c), q(4c+1)}, {.. q(4c+2), q(4c+3) ..}, each byte stored as q + 128;
 //     scales per quad g: {d(g), d(g+8)} fp16.
+//   INT4-affine (2 steps, 32 K = one block): per step one word of eight
+//     nibbles, low to high {g: e0, g+8: e0, g: e2, g+8: e2, g: e1, g+8: e1,
+//     g: e3, g+8: e3} (e_i = element 16s + 4c + i), so that masks of nibbles
+//     0/4 and 1/5 (and of the word shifted by 8) land in FP16 mantissas as the
+//     A fragment's register pairs; per quad g {d(g), d(g+8), m(g), m(g+8)}.
 #pragma once
 #include "common.cuh"
 #include "layout.cuh"
 
 namespace tsm {
 
-enum : unsigned { BAD_E8M0_NAN = 1u, BAD_Q8_SCALE = 2u, BAD_ROUTER_SCALE = 4u };
+enum : unsigned { BAD_E8M0_NAN = 1u, BAD_Q8_SCALE = 2u, BAD_ROUTER_SCALE = 4u, BAD_I4_SCALE = 8u };
+
+// Nibble `e` (0..31) of an INT4-affine block's code bytes.
+TSM_DEV uint32_t i4_code(const uint8_t* qs, int e) { return (qs[e >> 1] >> ((e & 1) * 4)) & 0xFu; }
 
 // PHASE 0: tile t rows 0..7 = gate rows 8t..8t+7, rows 8..15 = up rows
 // 8t..8t+7 (matrices [rows][row_bytes]); PHASE 1: tile t rows = rows
@@ -41,7 +49,8 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
     const int t = (int)(u / chunks), ck = (int)(u % chunks);
     const int grp = t / gs, jt = t % gs;
     const int ntg = group_tiles(tiles, gs, grp);
-    uint8_t* unit = dst + group_offset(gs, chunks, grp) + ((uint64_t)ck * ntg + jt) * UNIT_BYTES;
+    constexpr int UB = FMT == FMT_INT4_AFFINE ? UNIT_BYTES_I4 : UNIT_BYTES;
+    uint8_t* unit = dst + group_offset(gs, chunks, grp, UB) + ((uint64_t)ck * ntg + jt) * UB;
     const uint8_t* rg;
     const uint8_t* rg8;
     bool zg = false, zg8 = false;
@@ -55,7 +64,23 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
       rg8 = a + (size_t)(zg8 ? 0 : 16 * t + g + 8) * row_bytes;
     }
     uint32_t w[4];
-    if (FMT == 1) {
+    if (FMT == FMT_INT4_AFFINE) {
+      const uint8_t* qg = rg + ck * 20 + 4;
+      const uint8_t* qg8 = rg8 + ck * 20 + 4;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int e0 = 16 * s + 4 * c;
+        const uint32_t n[8] = {i4_code(qg, e0),     i4_code(qg8, e0),     i4_code(qg, e0 + 2), i4_code(qg8, e0 + 2),
+                               i4_code(qg, e0 + 1), i4_code(qg8, e0 + 1), i4_code(qg, e0 + 3), i4_code(qg8, e0 + 3)};
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v |= n[i] << (4 * i);
+        if (zg) v &= 0xF0F0F0F0u;   // row g nibbles are 0, 2, 4, 6
+        if (zg8) v &= 0x0F0F0F0Fu;                      // row g+8 nibbles are 1, 3, 5, 7
+        w[s] = v;
+      }
+      w[2] = w[3] = 0u;
+    } else if (FMT == FMT_MXFP4) {
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const int blk = 2 * ck + s / 2;
@@ -88,7 +113,10 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
         }
       }
     }
-    *reinterpret_cast<uint4*>(unit + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (FMT == FMT_INT4_AFFINE)
+      *reinterpret_cast<uint2*>(unit + lane * 8) = make_uint2(w[0], w[1]);
+    else
+      *reinterpret_cast<uint4*>(unit + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     if (lane < 8) {
       // scales of the quad of rows (lane, lane + 8)
       const uint8_t* sg;
@@ -104,7 +132,17 @@ __global__ void repack_kernel(const uint8_t* __restrict__ a, const uint8_t* __re
         sg8 = a + (size_t)(zs8 ? 0 : 16 * t + lane + 8) * row_bytes;
       }
       uint32_t sw;
-      if (FMT == 1) {
+      if (FMT == FMT_INT4_AFFINE) {
+        const uint32_t d0 = zs ? 0u : (uint32_t)sg[ck * 20] | ((uint32_t)sg[ck * 20 + 1] << 8);
+        const uint32_t d1 = zs8 ? 0u : (uint32_t)sg8[ck * 20] | ((uint32_t)sg8[ck * 20 + 1] << 8);
+        const uint32_t m0 = zs ? 0u : (uint32_t)sg[ck * 20 + 2] | ((uint32_t)sg[ck * 20 + 3] << 8);
+        const uint32_t m1 = zs8 ? 0u : (uint32_t)sg8[ck * 20 + 2] | ((uint32_t)sg8[ck * 20 + 3] << 8);
+        if ((d0 & 0x7C00u) == 0x7C00u || (d1 & 0x7C00u) == 0x7C00u || (m0 & 0x7C00u) == 0x7C00u ||
+            (m1 & 0x7C00u) == 0x7C00u)
+          mybad |= BAD_I4_SCALE;
+        *reinterpret_cast<uint2*>(unit + QUANT_BYTES_I4 + lane * 8) = make_uint2(d0 | (d1 << 16), m0 | (m1 << 16));
+        continue;
+      } else if (FMT == FMT_MXFP4) {
         uint32_t e[4] = {0, 0, 0, 0};
         if (2 * ck < nblocks) {
           e[0] = sg[(2 * ck) * 17];

@@ -40,7 +40,10 @@ struct LayerDev {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t blob_row_bytes(int fmt, int cols) { return (size_t)(cols / 32) * (fmt == TS_FMT_Q8_0 ? 34 : 17); }
+// Bytes of one user row of `cols` weights: 32-element blocks of 34 (Q8_0), 17 (MXFP4) or 20 (INT4-affine) bytes.
+size_t blob_row_bytes(int fmt, int cols) {
+  return (size_t)(cols / 32) * (fmt == TS_FMT_Q8_0 ? 34 : fmt == TS_FMT_MXFP4 ? 17 : 20);
+}
 
 }  // namespace
 
@@ -75,7 +78,9 @@ struct ts_moe {
   float* partial1 = nullptr;
   unsigned* entry_done = nullptr;
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group, consumer warp) chunk counters
-  unsigned* grid = nullptr;     // {grid barrier arrivals, launches, x slices written, router items published}
+  unsigned long long* arrivals = nullptr;  // grid barrier arrivals (64-bit, never reset while the handle lives)
+  unsigned* grid = nullptr;     // {x slices written, router items published}
+  bool debug_skip_arrival = false;
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
   uint8_t* counters = nullptr;
@@ -120,7 +125,8 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
     return bad("top_k must be in [1, min(8, num_experts)] (the 8-slot phase-2 reduce)");
   if (c->num_layers < 1 || c->num_layers > 1024) return bad("num_layers must be in [1, 1024]");
   if (c->max_tokens < 1 || c->max_tokens > TS_MOE_MAX_PREFILL) return bad("max_tokens must be in [1, 65536]");
-  if (c->expert_fmt != TS_FMT_Q8_0 && c->expert_fmt != TS_FMT_MXFP4) return bad("unknown expert_fmt");
+  if (c->expert_fmt != TS_FMT_Q8_0 && c->expert_fmt != TS_FMT_MXFP4 && c->expert_fmt != TS_FMT_INT4_AFFINE)
+    return bad("unknown expert_fmt");
   if (c->score != TS_SCORE_SOFTMAX_SELECTED && c->score != TS_SCORE_SOFTMAX_ALL_NORENORM &&
       c->score != TS_SCORE_SIGMOID_RENORM)
     return bad("unknown score");
@@ -232,6 +238,7 @@ ts_moe_status set_smem_attrs(ts_moe* h) {
   const int bytes = (int)sizeof(LayerSmem);
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX));
   return TS_MOE_OK;
 }
@@ -244,6 +251,9 @@ void launch_repack(int fmt, const uint8_t* a, const uint8_t* b, int row_bytes, i
   const long long blocks = std::min<long long>((units + 7) / 8, 65535LL * 8);
   if (fmt == TS_FMT_MXFP4)
     repack_kernel<1, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
+                                                                                      g.chunks, g.gs, dst, bad, nrows);
+  else if (fmt == TS_FMT_INT4_AFFINE)
+    repack_kernel<2, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
                                                                                       g.chunks, g.gs, dst, bad, nrows);
   else
     repack_kernel<0, PHASE><<<(int)std::max<long long>(1, blocks), threads, 0, st>>>(a, b, row_bytes, nblocks, g.tiles,
@@ -381,7 +391,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + 4 + 1;  // + grid[4] + error word
+    const size_t n_cnt = 2 + (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + 2 + 1;  // arrivals (u64) + ... + grid[2] + error word
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -408,10 +418,11 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     unsigned* cn = (unsigned*)(h->ws + o_cnt);
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
-    h->cnt_gB = cn;
+    h->arrivals = (unsigned long long*)cn;  // 256-byte aligned: first in the counter block
+    h->cnt_gB = cn + 2;
     h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B * NWC;
-    h->grid = h->entry_done + (E + 1);  // grid barrier arrivals, launches, x slices written, router items published
-    h->err = h->grid + 4;
+    h->grid = h->entry_done + (E + 1);  // x slices written, router items published
+    h->err = h->grid + 2;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
     if (ce != cudaSuccess) {
@@ -428,6 +439,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     int per_sm = 0;
     ce = fmt == TS_FMT_MXFP4
              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<1>, NTHREADS, sizeof(LayerSmem))
+         : fmt == TS_FMT_INT4_AFFINE
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<2>, NTHREADS, sizeof(LayerSmem))
              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<0>, NTHREADS, sizeof(LayerSmem));
     if (ce != cudaSuccess) {
       g_open_error = std::string("occupancy query: ") + cudaGetErrorString(ce);
@@ -534,6 +547,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   if (bad) {
     g_open_error = std::string("refused at open: ") + ((bad & BAD_E8M0_NAN) ? "MXFP4 block scale e8m0 = 255 (NaN); " : "") +
                    ((bad & BAD_Q8_SCALE) ? "non-finite Q8_0 block scale; " : "") +
+                   ((bad & BAD_I4_SCALE) ? "non-finite INT4-affine block scale or offset; " : "") +
                    ((bad & BAD_ROUTER_SCALE) ? "non-finite router block scale; " : "");
     ts_moe_close(h);
     return TS_MOE_EINVAL;
@@ -646,10 +660,11 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   lp.cnt_group = h->cnt_gB;
   lp.ng_max = h->ng_max_B;
   lp.entry_done = h->entry_done;
-  lp.grid_cnt = h->grid;
-  lp.grid_gen = h->grid + 1;
-  lp.xh_cnt = h->grid + 2;
-  lp.route_cnt = h->grid + 3;
+  lp.grid_cnt = h->arrivals;
+  lp.xh_cnt = h->grid;
+  lp.route_cnt = h->grid + 1;
+  lp.debug_skip_arrival = h->debug_skip_arrival ? 1 : 0;
+  h->debug_skip_arrival = false;  // one launch only
   lp.err = h->err;
   lp.act = c.act;
   lp.alpha = c.act_alpha;
@@ -665,6 +680,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
     cudaError_t e;
     if (c.expert_fmt == TS_FMT_MXFP4)
       e = launch_pdl(layer_kernel<1>, h->nb, NTHREADS, smem, st, lp);
+    else if (c.expert_fmt == TS_FMT_INT4_AFFINE)
+      e = launch_pdl(layer_kernel<2>, h->nb, NTHREADS, smem, st, lp);
     else
       e = launch_pdl(layer_kernel<0>, h->nb, NTHREADS, smem, st, lp);
     if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
@@ -860,10 +877,7 @@ ts_moe_status ts_moe_debug_skew_barrier(ts_moe* h, void* stream) {
   if (!h) return TS_MOE_EINVAL;
   TSM_CUDA(h, cudaSetDevice(h->cfg.device));
   TSM_CUDA(h, cudaStreamSynchronize((cudaStream_t)stream));
-  unsigned gen = 0;
-  TSM_CUDA(h, cudaMemcpy(&gen, h->grid + 1, 4, cudaMemcpyDeviceToHost));
-  gen += 2u;  // the next launch waits for (gen + 1) * NB arrivals; only NB more come
-  TSM_CUDA(h, cudaMemcpy(h->grid + 1, &gen, 4, cudaMemcpyHostToDevice));
+  h->debug_skip_arrival = true;  // the next launch's CTA 0 does not arrive: only NB - 1 of NB arrivals come
   return TS_MOE_OK;
 }
 

@@ -51,7 +51,7 @@ import torch
 
 FMT_Q8_0 = 0
 FMT_MXFP4 = 1
-FMT_INT4_AFFINE = 2  # oracle only: the CUDA library refuses it (unknown expert_fmt)
+FMT_INT4_AFFINE = 2
 SCORE_SOFTMAX_SELECTED = 0
 SCORE_SOFTMAX_ALL_NORENORM = 1
 SCORE_SIGMOID_RENORM = 2
@@ -134,6 +134,10 @@ CONFIGS = {
     # sigmoid scoring with a selection-only correction bias (the MiniMax flow), MiniMax-M2-like widths
     7: MoEShape("minimax-m2-shaped-q8_0-sigmoid-4-layer-stack", 3072, 1536, 256, 8, score=SCORE_SIGMOID_RENORM,
                 bias_mode=BIAS_SELECT_ONLY, num_layers=4, cfg_id=7),
+    # INT4-affine experts (the format the gpt-oss state page names for its batched-GEMV seam) on the
+    # gpt-oss-shaped 24-layer stack: 11.9 GB of experts
+    8: MoEShape("gpt-oss-20b-shaped-int4-affine-24-layer-stack", 2880, 2880, 32, 4, expert_fmt=FMT_INT4_AFFINE,
+                bias_mode=BIAS_LOGITS, act=ACT_SWIGLU_CLAMPED, num_layers=24, cfg_id=8),
 }
 
 

@@ -58,7 +58,7 @@ SHAPE = synth.MoEShape("t", 64, 64, 4, 2, cfg_id=77, max_tokens=4)
     (dict(top_k=5), 1, "top_k"),           # > num_experts (4)
     (dict(max_tokens=65537), 1, "max_tokens"),
     (dict(max_tokens=0), 1, "max_tokens"),
-    (dict(expert_fmt=2), 1, "expert_fmt"),      # INT4-affine: defined in the oracle only so far
+    (dict(expert_fmt=3), 1, "expert_fmt"),
     (dict(score=3), 1, "score"),
     (dict(bias_mode=7), 1, "bias_mode"),
     (dict(act=5), 1, "act"),
@@ -101,6 +101,12 @@ def test_bias_and_shared_consistency(B):
     assert st == 2 and "shared" in msg
     ok = SHAPE.replace(shared_inter=64)
     assert B.validate(ok, _small_layers(ok))[0] == 0
+    # INT4-affine experts are accepted, but not with a shared expert (the shared expert is Q8_0)
+    i4 = SHAPE.replace(expert_fmt=synth.FMT_INT4_AFFINE, cfg_id=79)
+    assert B.validate(i4, _small_layers(i4))[0] == 0
+    i4s = i4.replace(shared_inter=64)
+    st, msg = B.validate(i4s, _small_layers(i4s))
+    assert st == 2 and "shared" in msg
 
 
 def test_sigmoid_scoring_takes_a_selection_only_bias(B):
@@ -207,8 +213,8 @@ def _header_constants():
 def test_header_constants_match_the_binding_and_the_generator(B):
     h = _header_constants()
     assert h["TS_MOE_ABI_VERSION"] == B.TS_MOE_ABI_VERSION
-    assert (h["TS_FMT_Q8_0"], h["TS_FMT_MXFP4"]) == (synth.FMT_Q8_0, synth.FMT_MXFP4)
-    assert "TS_FMT_INT4_AFFINE" not in h            # the library does not accept it yet
+    assert (h["TS_FMT_Q8_0"], h["TS_FMT_MXFP4"], h["TS_FMT_INT4_AFFINE"]) == \
+        (synth.FMT_Q8_0, synth.FMT_MXFP4, synth.FMT_INT4_AFFINE)
     assert (h["TS_SCORE_SOFTMAX_SELECTED"], h["TS_SCORE_SOFTMAX_ALL_NORENORM"], h["TS_SCORE_SIGMOID_RENORM"]) == \
         (synth.SCORE_SOFTMAX_SELECTED, synth.SCORE_SOFTMAX_ALL_NORENORM, synth.SCORE_SIGMOID_RENORM)
     assert (h["TS_BIAS_NONE"], h["TS_BIAS_LOGITS"], h["TS_BIAS_SELECT_ONLY"]) == \

@@ -12,7 +12,7 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 S = synth.MoEShape
-Q8, MX = synth.FMT_Q8_0, synth.FMT_MXFP4
+Q8, MX, I4 = synth.FMT_Q8_0, synth.FMT_MXFP4, synth.FMT_INT4_AFFINE
 
 SMALL = {
     # name: shape  (cfg_id only seeds the draws)
@@ -29,6 +29,12 @@ SMALL = {
     "q8_sigmoid_correction_bias": S("sig", 256, 128, 16, 4, score=2, bias_mode=2, cfg_id=111),
     "mx_sigmoid_e256_k8": S("sigmx", 128, 128, 256, 8, expert_fmt=MX, score=2, bias_mode=2, cfg_id=112),
     "q8_sigmoid_no_bias": S("sig0", 64, 64, 8, 2, score=2, cfg_id=113),
+    # INT4-affine experts (d * q + m per 32-block)
+    "i4_sel": S("i4", 256, 160, 8, 2, expert_fmt=I4, cfg_id=114),
+    "i4_odd_blocks_clamped_bias": S("i4c", 96, 224, 5, 3, expert_fmt=I4, bias_mode=1, act=1, cfg_id=115),
+    "i4_sigmoid_e256_k8": S("i4sig", 128, 128, 256, 8, expert_fmt=I4, score=2, bias_mode=2, cfg_id=116),
+    "i4_large_k_window_split": S("i4k", 1088, 96, 4, 2, expert_fmt=I4, cfg_id=117),
+    "i4_wide_inter": S("i4w", 64, 2080, 3, 2, expert_fmt=I4, cfg_id=118),
 }
 
 
@@ -185,9 +191,12 @@ def test_chunked_prefill_gptoss_full_size_sampled():
 
 # cfg 3 at every M of the benchmark's sweep: the router slicing, the read-back
 # of the router items and the gate/up partition all switch with M
-@pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 2), (3, 4), (3, 8), (3, 16), (4, 16)])
+@pytest.mark.parametrize("cfg,M", [(1, 1), (2, 1), (2, 16), (3, 1), (3, 2), (3, 4), (3, 8), (3, 16), (4, 16),
+                                   (8, 1), (8, 16)])
 def test_workload_full_size(cfg, M):
     shape = synth.CONFIGS[cfg]
+    if shape.num_layers > 1:
+        shape = shape.replace(num_layers=1)          # one layer of a stack workload
     if M > shape.max_tokens:
         shape = shape.replace(max_tokens=M)
     rep = parity.check_shape(shape, M)
@@ -197,7 +206,7 @@ def test_workload_full_size(cfg, M):
 # dense FFN on the same kernels (E = 1, K = 1, weight 1): the deepseek2 dense lead
 # layer (hidden 2048, dense width 10944, Q8_0) and a Mixtral-width dense FFN
 @pytest.mark.parametrize("name,H,I,fmt", [("dense_lead_ds2", 2048, 10944, Q8), ("dense_mixtral_width", 4096, 14336, Q8),
-                                          ("dense_mx", 2880, 2880, MX)])
+                                          ("dense_mx", 2880, 2880, MX), ("dense_i4", 2880, 2880, I4)])
 @pytest.mark.parametrize("M", [1, 16])
 def test_dense_ffn(name, H, I, fmt, M):
     shape = S(name, H, I, 1, 1, expert_fmt=fmt, cfg_id=120 + H % 7 + fmt, max_tokens=16)

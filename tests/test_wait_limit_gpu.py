@@ -1,7 +1,7 @@
 """Failure detection on the GPU without a fault: a bounded wait that runs out.
 
 The grid barrier of the layer kernel waits for a count that a test hook has
-made unreachable.  Every CTA gives up after the 2 s limit, records the
+made unreachable (one CTA is told not to arrive).  Every CTA gives up after the 2 s limit, records the
 "grid barrier wait gave up" bit in the device error word and runs to its end.
 The host then reads the error through ts_moe_device_status.  That call re-zeroes
 the handle's counters, and the next call is the same, bit for bit, as one made
