@@ -323,7 +323,7 @@ TSM_DEV unsigned down_owners(const LayerSmem& s, const LayerParams& p, int NB, i
 // else the contributing CTAs' partial slots, to be added in CTA order.
 // down_loads issues the first DV_LOADS of them (predicated, all in flight
 // together) into t and returns how many it covered; down_rest adds the rest.
-constexpr int DV_LOADS = 4;
+constexpr int DV_LOADS = 8;
 
 struct DownSrc {
   const float* base;  // P row, or the partial-slot base of contributor bf

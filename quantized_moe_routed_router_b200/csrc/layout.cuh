@@ -102,11 +102,13 @@ TSM_HD int group_tiles(int tiles, int gs, int grp) {
 // entry-major order (entry, group, chunk) for gate/up and group-major order
 // (group, entry, chunk) for down -- are split into NB contiguous ranges:
 // block b owns [range_start(b), range_start(b + 1)).
-// floor(b * U / NB) through FP64: b * U < 2^53 is exact, the quotient is
-// correctly rounded, and a true quotient below an integer stays at least 1/NB
-// below it, far more than the rounding error, so truncation gives the floor.
-// (A 64-bit integer division is a long software sequence on the GPU.)
-TSM_HD uint64_t range_start(uint64_t U, int NB, int b) { return (uint64_t)((double)b * (double)U / (double)NB); }
+// floor(b * U / NB) in 32-bit arithmetic (U < 2^32, b <= NB <= 512): with
+// U = q NB + r, b U / NB = b q + b r / NB and b r < 2^18.  (A 64-bit integer
+// division is a long software sequence on the GPU.)
+TSM_HD uint64_t range_start(uint64_t U, int NB, int b) {
+  const unsigned u = (unsigned)U, nb = (unsigned)NB, q = u / nb, r = u - q * nb;
+  return (uint64_t)((unsigned)b * q + (unsigned)b * r / nb);
+}
 
 // The block whose range contains unit u (0 <= u < U): the largest b with
 // range_start(b) <= u, i.e. floor(((u + 1) * NB - 1) / U).
