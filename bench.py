@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--M", type=int, default=16)
     ap.add_argument("--cfg", type=int, default=5)
     ap.add_argument("--layers", type=int, default=0, help="override the number of layers (0 = the workload's)")
-    ap.add_argument("--no-sweep", action="store_true", help="skip timing M in {1,2,4,8,16} (key m_sweep) and the chunked M = 64 (key prefill_chunked)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip timing M in {1,2,4,8,16} (key m_sweep) and the one-launch M = 64 prefill (key prefill)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -130,7 +130,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = os.path.join(ROOT, "quantized_moe_routed_router_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "layer_kernel_traffic.json")
-PREFILL_M = 64  # the chunked-prefill point of the sweep: four 16-token launches per layer
+PREFILL_M = 64  # the prefill point of the sweep: one 64-token launch per layer
 
 
 def kernel_sources_sha256() -> str:
@@ -238,20 +238,30 @@ def run_ours(args, rank, world, local):
     rs = torch.stack([synth.make_x(shape, l, Mr, device=dev, master=master, tensor=synth.T_RESID) for l in range(NL)])
     stream = torch.cuda.Stream(device=dev)
 
+    LT = info.launch_tokens  # tokens per layer-kernel launch
+
     def touched_bytes(Mx, src=xs):
-        """Weight bytes one step streams: per layer, per launch of up to 16
-        tokens, the touched experts + router (+ shared)."""
+        """Weight bytes one step streams: per layer, per launch of up to LT
+        tokens, each touched expert once per 16 routes it receives (its
+        entries) + the router (+ the shared expert once per 16 tokens)."""
         idx = torch.empty(Mx, shape.top_k, dtype=torch.int32, device=dev)
         w = torch.empty(Mx, shape.top_k, device=dev)
-        n_touched = []
+        n_entries, n_touched = [], []
         with torch.cuda.stream(stream):
             for l in range(NL):
                 moe.route(l, src[l, :Mx], idx, w, stream=stream)
                 stream.synchronize()
                 ih = idx.cpu().numpy()
-                n_touched.append([len(set(ih[c:c + 16].ravel().tolist())) for c in range(0, Mx, 16)])
-        per_layer = [sum(n * info.expert_bytes + info.router_bytes + info.shared_bytes for n in nl)
-                     for nl in n_touched]
+                ent, tch = [], []
+                for c in range(0, Mx, LT):
+                    cnt = np.bincount(ih[c:c + LT].ravel(), minlength=shape.num_experts)
+                    ent.append(int(((cnt + 15) // 16).sum()))
+                    tch.append(int((cnt > 0).sum()))
+                n_entries.append(ent)
+                n_touched.append(tch)
+        per_layer = [sum(n * info.expert_bytes + info.router_bytes +
+                         -(-min(LT, Mx - i * LT) // 16) * info.shared_bytes for i, n in enumerate(nl))
+                     for nl in n_entries]
         return sum(per_layer), [n for nl in n_touched for n in nl], per_layer
 
     def make_graph(Mx, out, src=xs):
@@ -317,7 +327,7 @@ def run_ours(args, rank, world, local):
     # The headline kernel time: the graph's timed region holds nothing but the
     # layer-kernel launches (PDL-chained), so the events around it divided by
     # the launches give the kernel's average duration inside the step.
-    launches_per_step = NL * ((M + 15) // 16)
+    launches_per_step = NL * ((M + LT - 1) // LT)
     avg_ms = ms_step / launches_per_step
     bytes_per_launch = algo_bytes / launches_per_step
     achieved = bytes_per_launch / (avg_ms * 1e-3) / 1e9
@@ -373,15 +383,16 @@ def run_ours(args, rank, world, local):
                               "frac_of_8TBs": round(b2 / (ms2 * 1e-3) / 8e12, 4),
                               "touched_experts_per_layer": round(sum(nt2) / len(nt2), 2)}
             del g2
-        # chunked prefill: M = 64 tokens per layer run as four 16-token launches
+        # prefill: M = 64 tokens per layer in one launch (each touched expert read once per 16 routes)
         xp = torch.stack([synth.make_x(shape, l, PREFILL_M, device=dev, master=master) for l in range(NL)])
         op = torch.stack([synth.make_x(shape, l, PREFILL_M, device=dev, master=master, tensor=synth.T_RESID)
                           for l in range(NL)])
         gp = make_graph(PREFILL_M, op, xp)
         bp, ntp, _ = touched_bytes(PREFILL_M, xp)
         msp, _ = time_graph(gp, max(20, args.steps // 2), args.warmup)
-        prefill = {"M": PREFILL_M, "launches_per_layer": (PREFILL_M + 15) // 16,
+        prefill = {"M": PREFILL_M, "launches_per_layer": (PREFILL_M + LT - 1) // LT,
                    "tokens_per_s": round(world * PREFILL_M / (msp * 1e-3), 1), "ms_per_step": round(msp, 4),
+                   "streamed_GB_per_step": round(bp / 1e9, 3),
                    "streamed_GB_per_s": round(bp / (msp * 1e-3) / 1e9, 1),
                    "touched_experts_per_launch": round(sum(ntp) / len(ntp), 2)}
         del gp, xp, op
@@ -408,13 +419,13 @@ def run_ours(args, rank, world, local):
             "roofline": roofline,
             "e2e": {"value": round(world * M / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-            "gpu_launches": args.steps * NL * ((M + 15) // 16),
+            "gpu_launches": args.steps * NL * ((M + LT - 1) // LT),
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
         if sweep:
             line["m_sweep"] = sweep
-            line["prefill_chunked"] = prefill
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
     moe.close()
 

@@ -8,9 +8,12 @@
  *   (+ optional shared expert) -> added back to the residual stream.
  * Every step runs in this library's CUDA kernels on the caller's stream; the
  * host does no per-call arithmetic, no allocation and no synchronisation.
- * One kernel launch takes at most TS_MOE_MAX_TOKENS (16) tokens, the pages'
- * micro-batch; a call with more runs as ceil(M / 16) launches over consecutive
- * 16-row blocks (full blocks first), as the pages' chunked-prefill driver does.
+ * Routing works on blocks of TS_MOE_MAX_TOKENS (16) tokens, the pages'
+ * micro-batch.  One ts_moe_forward launch takes up to TS_MOE_MAX_LAUNCH_TOKENS
+ * (64) tokens, four such blocks, and reads each touched expert's weights once
+ * for every 16 routes it receives; a call with more tokens runs as several
+ * launches over consecutive row blocks (full ones first), as the pages'
+ * chunked-prefill driver feeds the routed half block by block.
  *
  * Conventions
  *   - "device" pointers are CUDA device addresses on cfg->device; "host"
@@ -37,8 +40,9 @@ extern "C" {
 #endif
 
 #define TS_MOE_ABI_VERSION 1u
-#define TS_MOE_MAX_TOKENS 16     /* tokens per launch: MAX_PREFILL_BATCH = 16 (llama / gpt-oss state pages) */
-#define TS_MOE_MAX_PREFILL 65536 /* largest max_tokens: calls above 16 tokens run in 16-token chunks */
+#define TS_MOE_MAX_TOKENS 16     /* tokens per routing block: MAX_PREFILL_BATCH = 16 (llama / gpt-oss state pages) */
+#define TS_MOE_MAX_LAUNCH_TOKENS 64 /* tokens per layer launch (four routing blocks), see ts_moe_info.launch_tokens */
+#define TS_MOE_MAX_PREFILL 65536 /* largest max_tokens: calls above one launch run in chunks */
 #define TS_MOE_MAX_TOPK 8    /* PHASE2_FIXED_SLOTS = 8 (deepseek2 state page, `build`) */
 #define TS_MOE_MAX_EXPERTS 256
 
@@ -86,7 +90,7 @@ typedef struct {
   int32_t num_experts;   /* E, 1..256 */
   int32_t top_k;         /* K, 1..min(8, E) */
   int32_t num_layers;    /* layers held by this handle, 1..1024 */
-  int32_t max_tokens;    /* largest M any call will pass, 1..65536 (the workspace holds min(max_tokens, 16)) */
+  int32_t max_tokens;    /* largest M any call will pass, 1..65536 (the workspace holds one launch's tokens) */
   int32_t expert_fmt;    /* TS_FMT_*; router and shared expert are always Q8_0 (a shared expert needs Q8_0 experts) */
   int32_t score;         /* TS_SCORE_* */
   int32_t bias_mode;     /* TS_BIAS_* */
@@ -136,8 +140,9 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
  * selection logit, lower index first on ties); w: device [M][K] float32
  * weights; logits: device [M][E] float32 router logits before any bias, or
  * NULL.  0 <= M <= max_tokens (M = 0 is a no-op; M > 16 runs in 16-token
- * chunks, one launch each).  Asynchronous on `stream` (a cudaStream_t, NULL =
- * legacy default stream). */
+ * chunks, one launch each).  The routing equals the one ts_moe_forward uses
+ * for a call of the same M, bit for bit.  Asynchronous on `stream` (a
+ * cudaStream_t, NULL = legacy default stream). */
 ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
                            void* stream);
 
@@ -145,9 +150,8 @@ ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* 
  * post-attention-norm activations, `moe_x`).  resid: device [M][H] BF16,
  * updated in place to bf16(resid + y), or NULL.  y: device [M][H] float32
  * routed(+shared) sum (`h2`), or NULL.  At least one of resid / y must be
- * non-NULL.  0 <= M <= max_tokens; M > 16 runs as ceil(M / 16) launches of
- * one 16-row block each (the remainder last), each token's result the same as
- * in a call of its own block.  Asynchronous on `stream`; allocates nothing;
+ * non-NULL.  0 <= M <= max_tokens; a call runs as launches of up to
+ * launch_tokens (64) rows (the remainder last).  Asynchronous on `stream`; allocates nothing;
  * calls on one handle must not overlap on the device (they share the
  * handle's workspace). */
 ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream);
@@ -177,6 +181,7 @@ typedef struct {
   uint64_t shared_bytes;
   int32_t num_ctas;
   int32_t sm_count;
+  int32_t launch_tokens;  /* tokens per layer launch: 64, or 16 when the router cannot be cut for four blocks */
 } ts_moe_info;
 ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
 

@@ -45,7 +45,7 @@ class LayerWeights(C.Structure):
 class Info(C.Structure):
     _fields_ = [("arena_bytes", C.c_uint64), ("workspace_bytes", C.c_uint64), ("expert_bytes", C.c_uint64),
                 ("router_bytes", C.c_uint64), ("shared_bytes", C.c_uint64), ("num_ctas", C.c_int32),
-                ("sm_count", C.c_int32)]
+                ("sm_count", C.c_int32), ("launch_tokens", C.c_int32)]
 
 
 def _load():

@@ -59,10 +59,10 @@ static_assert(ROUTE_WARPS <= NWC + 1, "routing uses the first ROUTE_WARPS warps"
 
 struct LayerParams {
   RouteParams rp;           // routing inputs; its output pointers are written by CTA 0 only
-  __half* xh;               // [Mmax][Hp] FP16 x (the gate/up B operand), slice c written by CTA c
+  __half* xh;               // [M][Hp] FP16 x (the gate/up B operand), written by the routing CTAs of tile 0
   unsigned* xh_cnt;         // slices of xh written (reset at the end of each launch)
-  float* part_pub;          // [S][M][item_ld(E)] router items (tile j's 16 experts of slice c by CTA j * S + c)
-  float* max_pub;           // [S][MAX_TOK] |x| max of each slice
+  float* part_pub;          // [S][M][item_ld(E)] router items (block tb, tile j, slice c by CTA (tb T + j) S + c)
+  float* max_pub;           // [S][MAX_LT] |x| max of each slice
   unsigned* route_cnt;      // router items published (reset at the end of each launch)
   const uint8_t* wB;        // gate/up: expert e at wB + e * wB_stride
   uint64_t wB_stride;
@@ -77,9 +77,9 @@ struct LayerParams {
   float* P;                 // [M*K + M][H] down outputs of whole segments
   float* partial0;          // [NB][2][SLOT_FLOATS] gate/up partial slots
   float* partial1;          // [NB][2][SLOT_FLOATS] down partial slots
-  unsigned* cnt_group;      // [(E+1) * ng_max * NWC] gate/up chunk counters per (entry, group, consumer warp)
+  unsigned* cnt_group;      // [MAX_ENTRIES * ng_max * NWC] gate/up chunk counters per (entry, group, consumer warp)
   int ng_max;
-  unsigned* entry_done;     // [E+1] gate/up (group, consumer warp) shares finished per expert (+ shared)
+  unsigned* entry_done;     // [MAX_ENTRIES] gate/up (group, consumer warp) shares finished per entry
   unsigned long long* grid_cnt;  // grid barrier arrivals, never reset: NB per launch (64-bit: never wraps)
   int debug_skip_arrival;   // test hook: CTA 0 does not arrive, so the barrier's bounded wait runs out
   float* y;                 // [M][H] or null
@@ -109,13 +109,17 @@ struct Seg {
   long long g0;   // unit index of the (entry, group)'s first chunk
 };
 
-// First unit of entry j (touched experts, then the shared expert as entry nT):
-// gate/up units are entry-major, so entry j starts at upre0(j); down units are
-// group-major, and inside a group entry j starts at cpre1(j).
+// First unit of entry j (the nT routed entries, then the shared expert's
+// entries from nT on): gate/up units are entry-major, so entry j starts at
+// upre0(j); down units are group-major, and inside a group entry j starts at
+// cpre1(j).
 TSM_DEV long long upre0(const LayerParams& p, int nT, int j) {
-  return (long long)min(j, nT) * p.gB.ngroups * p.gB.chunks + (j > nT ? (long long)p.gBs.ngroups * p.gBs.chunks : 0);
+  return (long long)min(j, nT) * p.gB.ngroups * p.gB.chunks +
+         (j > nT ? (long long)(j - nT) * p.gBs.ngroups * p.gBs.chunks : 0);
 }
-TSM_DEV int cpre1(const LayerParams& p, int nT, int j) { return min(j, nT) * p.gC.chunks + (j > nT ? p.gCs.chunks : 0); }
+TSM_DEV int cpre1(const LayerParams& p, int nT, int j) {
+  return min(j, nT) * p.gC.chunks + (j > nT ? (j - nT) * p.gCs.chunks : 0);
+}
 
 // First unit of CTA b's range in phase PH (b = NB: the total), from the unit
 // counts alone: plain contiguous ranges, or for gate/up with few groups the
@@ -126,7 +130,9 @@ TSM_DEV unsigned cta_start(const LayerParams& p, int nT, int nE, int NB, bool al
   if (!aligned || b >= NB) return (unsigned)range_start((uint64_t)upre0(p, nT, nE), NB, b);
   const int g = aligned_group_of(b, G0, NB);
   const bool shg = g >= nT * p.gB.ngroups;
-  const int j = shg ? nT : g / p.gB.ngroups, grp = shg ? g - nT * p.gB.ngroups : g % p.gB.ngroups;
+  const int gs_ = g - nT * p.gB.ngroups;
+  const int j = shg ? nT + gs_ / p.gBs.ngroups : g / p.gB.ngroups;
+  const int grp = shg ? gs_ % p.gBs.ngroups : g % p.gB.ngroups;
   const int ch = shg ? p.gBs.chunks : p.gB.chunks;
   return (unsigned)(upre0(p, nT, j) + (long long)grp * ch + aligned_offset(b, G0, NB, ch));
 }
@@ -147,13 +153,14 @@ TSM_DEV bool next_seg(const LayerSmem& s, const LayerParams& p, long long& u, lo
     const unsigned upg = (unsigned)cpre1(p, nT, s.r.nE);
     grp = (int)(uu / upg);
     const int r = (int)(uu - (unsigned)grp * upg);
-    j = r < nT * gr.chunks ? r / gr.chunks : nT;
+    j = r < nT * gr.chunks ? r / gr.chunks : nT + (r - nT * gr.chunks) / gsh.chunks;
     c0 = r - cpre1(p, nT, j);
     base = (unsigned)grp * upg + (unsigned)cpre1(p, nT, j);
   } else {
     const unsigned ub = (unsigned)(gr.ngroups * gr.chunks);
-    j = uu < (unsigned)nT * ub ? (int)(uu / ub) : nT;
-    const bool sh = p.rp.has_shared && j == nT;
+    const unsigned ush = (unsigned)(gsh.ngroups * gsh.chunks);
+    j = uu < (unsigned)nT * ub ? (int)(uu / ub) : nT + (int)((uu - (unsigned)nT * ub) / ush);
+    const bool sh = p.rp.has_shared && j >= nT;
     const unsigned chunks = (unsigned)(sh ? gsh.chunks : gr.chunks);
     const unsigned e0 = (unsigned)upre0(p, nT, j);
     grp = (int)((uu - e0) / chunks);
@@ -161,7 +168,7 @@ TSM_DEV bool next_seg(const LayerSmem& s, const LayerParams& p, long long& u, lo
     base = e0 + (unsigned)grp * chunks;
   }
   sg.j = j;
-  sg.sh = p.rp.has_shared && j == s.r.nT;
+  sg.sh = p.rp.has_shared && j >= s.r.nT;
   const MatGeom& g = sg.sh ? gsh : gr;
   sg.chunks = g.chunks;
   sg.tiles = g.tiles;
@@ -312,7 +319,7 @@ TSM_DEV void mma_chunk(float (&acc)[RW][NT][4], const uint8_t* chunk, int ntg, i
 // First / last CTA that worked on the down segment (entry j, row group grp),
 // packed as bf | bl << 16.
 TSM_DEV unsigned down_owners(const LayerSmem& s, const LayerParams& p, int NB, int grp, int j) {
-  const bool sh = p.rp.has_shared && j == s.r.nT;
+  const bool sh = p.rp.has_shared && j >= s.r.nT;
   const unsigned C = (unsigned)(sh ? p.gCs.chunks : p.gC.chunks);
   const unsigned g0 = (unsigned)grp * (unsigned)cpre1(p, s.r.nT, s.r.nE) + (unsigned)cpre1(p, s.r.nT, j);
   return (unsigned)owner_tab(s.rs1, NB, g0) | ((unsigned)owner_tab(s.rs1, NB, g0 + C - 1) << 16);
@@ -403,13 +410,20 @@ TSM_DEV bool combine_prepare(LayerSmem& s, const LayerParams& p, int NB, int cti
 // ring, CB pairs per thread with all of their loads issued before any is
 // used; (2) each output sums its values in slot order.  The barrier orders the
 // owner table written by combine_prepare before its reads here.
+// floor(a / b) for 0 <= a < 2^21 and b >= 1 by a float reciprocal rb = 1 / b:
+// the product's relative error is below 2^-23, so its absolute error is below
+// 2^-23 (a + 0.5) / b < 0.25 / b, while (a + 0.5) / b lies at least 0.5 / b
+// from every integer; the truncation is exact.
+TSM_DEV int fdiv(int a, float rb) { return (int)(((float)a + 0.5f) * rb); }
+
 TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid, bool use_tab, float r0) {
-  constexpr int CT = NWC * 32, CB = 2;
+  constexpr int CT = NWC * 32, CB = 3;
   const int K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = p.rp.M * K, nE = s.r.nE;
   const unsigned* tab = reinterpret_cast<const unsigned*>(&s.r.part[0][0][0]);
   int lo, hi;
   combine_range(p, NB, lo, hi);
   const int KP = K + (p.rp.has_shared ? 1 : 0);
+  const float rKP = 1.f / (float)KP, rH = 1.f / (float)H, rG = 1.f / (float)(gs * 16);
   float* vbuf = reinterpret_cast<float*>(&s.w[0][0]);
   const int cap = (int)((sizeof(s.w) + sizeof(s.x)) / sizeof(float)) / KP;  // outputs per batch
   for (int base = lo; base < hi; base += cap) {
@@ -421,16 +435,16 @@ TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid,
       for (int u = 0; u < CB; ++u) {
         const int q = q0 + u * CT;
         const bool use = q < npair;
-        const int o = use ? q / KP : 0, k = q - o * KP, i = base + o;
-        const int tk = i / H, h = i - tk * H, grp = h / (gs * 16);
+        const int o = use ? fdiv(q, rKP) : 0, k = q - o * KP, i = base + o;
+        const int tk = fdiv(i, rH), h = i - tk * H, grp = fdiv(h, rG);
         int j, n, route;
         if (k < K) {
           route = s.r.rpos[tk * K + k];
           j = s.r.rj[route];
           n = route - s.r.ro[j];
-        } else {
-          j = s.r.nT;
-          n = tk;
+        } else {  // the shared expert: its entries take 16 tokens each
+          j = s.r.nT + tk / MAX_TOK;
+          n = tk % MAX_TOK;
           route = MK + tk;
         }
         const unsigned own = use_tab ? tab[grp * nE + j] : down_owners(s, p, NB, grp, j);
@@ -487,9 +501,9 @@ TSM_DEV void grid_barrier(const LayerSmem& s, const LayerParams& p, int NB, int 
 // count it for the entry.  __syncwarp orders the warp's stores before lane
 // 0's release increment (cumulative, so the whole warp's acts are published
 // with it); an entry is complete when its count reaches ngroups * NWC.
-TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, const LayerSmem& s, int lane) {
+TSM_DEV void entry_warp_done(const LayerParams& p, const Seg& sg, int lane) {
   __syncwarp();
-  if (lane == 0) red_release_add_u32(p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]), 1u);
+  if (lane == 0) red_release_add_u32(p.entry_done + sg.j, 1u);
 }
 
 // Group epilogue with complete sums in acc.
@@ -509,15 +523,15 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
         for (int h = 0; h < 2; ++h) {
           const int n = nt * 8 + 2 * c + h;
           if (n < sg.nc) {
-            const int tk = sg.sh ? n : s.r.tok[sg.ro + n];
+            const int tk = sg.sh ? sg.ro - p.rp.M * p.rp.K + n : s.r.tok[sg.ro + n];
             const float scl = __uint_as_float((uint32_t)(127 - s.r.shift[tk]) << 23);
             const float a = act_fn(p.act, p.alpha, p.limit, acc[r][nt][h] * scl, acc[r][nt][2 + h] * scl);
-            __half* dst = sg.sh ? p.acts_sh + (size_t)n * p.Sp : p.acts + (size_t)(sg.ro + n) * p.Ip;
+            __half* dst = sg.sh ? p.acts_sh + (size_t)tk * p.Sp : p.acts + (size_t)(sg.ro + n) * p.Ip;
             dst[arow] = __float2half_rn(a);
           }
         }
     }
-    entry_warp_done(p, sg, s, lane);
+    entry_warp_done(p, sg, lane);
   } else {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
@@ -530,7 +544,7 @@ TSM_DEV void group_epilogue(const LayerSmem& s, const LayerParams& p, const Seg&
         for (int hh = 0; hh < 2; ++hh) {
           const int n = nt * 8 + 2 * c + hh;
           if (n < sg.nc) {
-            const int route = sg.sh ? p.rp.M * p.rp.K + n : sg.ro + n;
+            const int route = sg.ro + n;  // (shared entries start at M K + their first token)
             float* dst = p.P + (size_t)route * p.rp.H + h0;
             dst[0] = acc[r][nt][hh];
             dst[8] = acc[r][nt][2 + hh];
@@ -616,7 +630,7 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
   // acquire-release chunk count, which publishes them and, for the last
   // contributor, makes the others' slots visible; the second __syncwarp
   // orders the other lanes' reads after it.  No other warp of the CTA waits.
-  const unsigned key = ((unsigned)(sg.sh ? p.rp.E : s.r.ex[sg.j]) * p.ng_max + sg.grp) * NWC + warp;
+  const unsigned key = ((unsigned)sg.j * p.ng_max + sg.grp) * NWC + warp;
   __syncwarp();
   unsigned last = 0;
   if (lane == 0) {
@@ -689,10 +703,11 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
     const uint8_t* gbase = mat + group_offset(sg.gs, sg.chunks, sg.grp, UB);  // (a shared expert only with Q8_0)
     const __half* brow = nullptr;
     if (lane < sg.nc) {
+      const int shtok = sg.ro - p.rp.M * p.rp.K + lane;  // shared entries: the token of column `lane`
       if (PH == 0)
-        brow = xh_src + (size_t)(sg.sh ? lane : s.r.tok[sg.ro + lane]) * p.rp.Hp;
+        brow = xh_src + (size_t)(sg.sh ? shtok : s.r.tok[sg.ro + lane]) * p.rp.Hp;
       else
-        brow = sg.sh ? p.acts_sh + (size_t)lane * p.Sp : p.acts + (size_t)(sg.ro + lane) * p.Ip;
+        brow = sg.sh ? p.acts_sh + (size_t)shtok * p.Sp : p.acts + (size_t)(sg.ro + lane) * p.Ip;
     }
     const unsigned ustride = (unsigned)sg.ntg * UB;
     int k_issued = sg.c0;  // first chunk whose weight stage is not yet issued
@@ -719,8 +734,10 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
           k_issued += kk;
         }
         if (lane == 0 && alive) {
-          const unsigned need = PH == 1 ? (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups) * NWC : (unsigned)p.rp.S;
-          const unsigned* flag = PH == 1 ? p.entry_done + (sg.sh ? p.rp.E : s.r.ex[sg.j]) : p.xh_cnt;
+          // gate/up: every routing block's tile-0 CTAs wrote their slices of xh
+          const unsigned need = PH == 1 ? (unsigned)(sg.sh ? p.gBs.ngroups : p.gB.ngroups) * NWC
+                                        : (unsigned)(p.rp.S * ((p.rp.M + MAX_TOK - 1) / MAX_TOK));
+          const unsigned* flag = PH == 1 ? p.entry_done + sg.j : p.xh_cnt;
           const unsigned long long t0 = globaltimer();
           while (ld_acquire_u32(flag) < need) {
             if (s.dead) break;
@@ -782,11 +799,13 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NB = gridDim.x, b = blockIdx.x;
 
-  // ---- 1. route.  CTA b < T * S computes router item (tile b / S, slice
-  // b % S) exactly as route_kernel does and publishes it with the slice's |x|
-  // max; every CTA then adds the items in slice order, forms the top-k and the
-  // route list itself.  The CTAs of tile 0 (b < S) also write their slice of
-  // the FP16 x that the gate/up phase reads.
+  // ---- 1. route.  The launch's M <= 64 tokens are cut into routing blocks
+  // of 16.  CTA b < T S NTB computes router item (block tb, tile j, slice c)
+  // with b = (tb T + j) S + c, exactly as route_kernel computes it for that
+  // block, and publishes it with the slice's |x| max; every CTA then adds the
+  // items in slice order, forms the top-k and the route list itself.  The
+  // CTAs of tile 0 also write their block's slice of the FP16 x that the
+  // gate/up phase reads.
   RouteParams rp = p.rp;
   rp.logits = nullptr;  // written below by CTA 0 from the summed items
   if (b != 0) {
@@ -797,11 +816,17 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.routes = nullptr;
     rp.rpos = nullptr;
   }
-  const int S = rp.S, nR = rp.rg.tiles * S;
+  const int M = rp.M, NTB = (M + MAX_TOK - 1) / MAX_TOK;
+  const int S = rp.S, TS = rp.rg.tiles * S, nR = TS * NTB;
   const bool rcta = b < nR;
-  const int rj = rcta ? b / S : 0, rcs = rcta ? b % S : 0;
+  const int rtb = rcta ? b / TS : 0, rrem = rcta ? b % TS : 0;
+  const int rj = rrem / S, rcs = rrem % S;
+  const int t0 = rtb * MAX_TOK;
+  RouteParams bp = rp;  // this CTA's routing block: rows t0 .. t0 + mb - 1 of x
+  bp.x = rp.x + (size_t)t0 * rp.H;
+  bp.M = min(MAX_TOK, M - t0);
   // the item's buffers sit in the still idle weight and window rings
-  const SliceSmem L(rp.M, rp.CS, rp.xscale != nullptr);
+  const SliceSmem L(min(M, MAX_TOK), rp.CS, rp.xscale != nullptr);
   uint8_t* ring = &s.w[0][0];
   constexpr size_t ring_bytes = sizeof(s.w) + sizeof(s.x);  // w and x are adjacent
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring + L.xs);
@@ -822,12 +847,12 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     mbar_init(&s.r.pbar, 1);
     fence_barrier_init();
     s.dead = 0;
-    if (rcta) slice_issue_router(rp, s.r, rj, rcs, rt);
+    if (rcta) slice_issue_router(bp, s.r, rj, rcs, rt);
   }
   grid_dep_wait();
   grid_dep_launch();
   if (tid == 0) {
-    if (rcta) slice_issue_x(rp, s.r, rcs, xs);
+    if (rcta) slice_issue_x(bp, s.r, rcs, xs);
     // floor(count / NB), exact in FP64 for counts below 2^53 (no 64-bit integer division)
     s.gen0 = (unsigned long long)floor((double)ld_acquire_u64(p.grid_cnt) / (double)NB);
   }
@@ -835,32 +860,35 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   __syncthreads();
   if (rcta) {
     mbar_wait(&s.r.xbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
-    slice_max(rp, s.r, rcs, xs, warp, lane);
+    slice_max(bp, s.r, rcs, xs, warp, lane);
     __syncthreads();
-    slice_input(rp, s.r, rcs, xs, xin, tid, NTHREADS);
+    slice_input(bp, s.r, rcs, xs, xin, tid, NTHREADS);
     __syncthreads();
     mbar_wait(&s.r.rbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
-    float* pub = p.part_pub + (size_t)rcs * rp.M * item_ld(rp.E);
-    if (rp.M > 8)
-      slice_gemv<2>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
+    float* pub = p.part_pub + ((size_t)rcs * M + t0) * item_ld(rp.E);
+    if (bp.M > 8)
+      slice_gemv<2>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
     else
-      slice_gemv<1>(rp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
-    if (rj == 0 && tid < rp.M) p.max_pub[rcs * MAX_TOK + tid] = s.r.smax[tid];
+      slice_gemv<1>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
+    if (rj == 0 && tid < bp.M) p.max_pub[rcs * MAX_LT + t0 + tid] = s.r.smax[tid];
     __syncthreads();
     if (tid == 0) red_release_add_u32(p.route_cnt, 1u);  // publishes the item written by the whole CTA
   }
   // every item published (bounded); then the S items and slice maxima are
-  // brought in by two bulk copies when they fit past the item buffers
+  // brought in by two bulk copies when they fit past the item buffers (with
+  // the logits after them)
   const int ild = item_ld(rp.E);
-  const unsigned ibytes = (unsigned)((size_t)S * rp.M * ild * 4), mbytes = (unsigned)S * MAX_TOK * 4;
-  const size_t pst = align128(L.total);
-  const bool bulk_items = pst + ibytes + mbytes <= ring_bytes;
+  const unsigned ibytes = (unsigned)((size_t)S * M * ild * 4), mbytes = (unsigned)S * MAX_LT * 4;
+  const size_t pst = align128(L.total), lgbytes = (size_t)M * rp.E * 4;
+  const bool bulk_items = pst + ibytes + mbytes + lgbytes <= ring_bytes;
   const float* items = bulk_items ? reinterpret_cast<const float*>(ring + pst) : p.part_pub;
   const float* maxes = bulk_items ? reinterpret_cast<const float*>(ring + pst + ibytes) : p.max_pub;
+  s.r.lg = reinterpret_cast<float*>(ring + (bulk_items ? pst + ibytes + mbytes : pst));  // fits: checked at open
+  s.r.lgld = rp.E;
   if (tid == 0) {
-    const unsigned long long t0 = globaltimer();
+    const unsigned long long tw = globaltimer();
     while (ld_acquire_u32(p.route_cnt) < (unsigned)nR) {
-      if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      if (globaltimer() - tw > WAIT_LIMIT_NS) {
         s.dead = 1;
         atomicOr(p.err, ERR_TIMEOUT_ROUTE);
         break;
@@ -876,32 +904,32 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   __syncthreads();
   if (bulk_items) mbar_wait(&s.r.pbar, 0, &s.dead, p.err, ERR_TIMEOUT_ROUTE);
   // logits: the items added in slice order; shift from the max of the slice maxima
-  for (int i = tid; i < rp.M * rp.E; i += NTHREADS) {
+  for (int i = tid; i < M * rp.E; i += NTHREADS) {
     const int t = i / rp.E, e = i - t * rp.E;
     float v = 0.f;
 #pragma unroll 8
     for (int c = 0; c < S; ++c) {
-      const float* src = items + ((size_t)c * rp.M + t) * ild + e;
+      const float* src = items + ((size_t)c * M + t) * ild + e;
       v += bulk_items ? *src : ld_cg(src);
     }
-    s.r.lg[t][e] = v;
+    s.r.lg[i] = v;
     if (b == 0 && p.rp.logits) p.rp.logits[i] = v;
   }
-  if (tid < rp.M) {
+  if (tid < M) {
     float m = 0.f;
     for (int c = 0; c < S; ++c) {
-      const float* src = maxes + c * MAX_TOK + tid;
+      const float* src = maxes + c * MAX_LT + tid;
       m = fmaxf(m, bulk_items ? *src : ld_cg(src));
     }
     s.r.shift[tid] = shift_of_max(m);
     if (rp.shift) rp.shift[tid] = s.r.shift[tid];
   }
   __syncthreads();
-  // gate/up B operand: this CTA's slice of x as FP16, published with the count of slices written
+  // gate/up B operand: this CTA's slice of its block's x as FP16, published with the count of slices written
   __half* xh_src = p.xh;
   const bool xwriter = rcta && rj == 0;
-  if (xwriter) slice_xh(rp, s.r, rcs, xs, xh_src, tid, NTHREADS);
-  route_topk(rp, s.r, warp, lane);
+  if (xwriter) slice_xh(bp, s.r, rcs, xs, xh_src, t0, tid, NTHREADS);
+  route_topk(rp, s.r, warp, lane, NTHREADS / 32);
   __syncthreads();
   if (xwriter && tid == 0) red_release_add_u32(p.xh_cnt, 1u);  // after the barrier: the CTA's slice of xh
   route_list(rp, s.r, warp, lane, tid, NTHREADS);
@@ -911,9 +939,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // starts at once; the consumer warps tabulate every CTA's range starts (for
   // the owners of split groups and the combine) while the first stages load
   const int nE = s.r.nE, nT = s.r.nT;
-  const bool hs = rp.has_shared != 0;
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
-  const int G0 = nT * p.gB.ngroups + (hs ? p.gBs.ngroups : 0);
+  const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
   const long long a0 = cta_start<0>(p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0>(p, nT, nE, NB, aligned, G0, b + 1);
   const long long d0 = cta_start<1>(p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1>(p, nT, nE, NB, aligned, G0, b + 1);
@@ -978,7 +1005,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   grid_barrier(s, p, NB, tid);
   final_combine(s, p, NB, tid, use_tab, r0);
   if (b == 0) {  // every readiness wait of this launch is over
-    for (int e = tid; e <= rp.E; e += NWC * 32) p.entry_done[e] = 0u;
+    for (int j = tid; j < nE; j += NWC * 32) p.entry_done[j] = 0u;
     if (tid == 0) {
       *p.route_cnt = 0u;
       *p.xh_cnt = 0u;

@@ -31,10 +31,14 @@ constexpr int UNIT_BYTES_I4 = 320;    // one INT4-affine (tile, chunk): 256 B co
 constexpr int QUANT_BYTES_I4 = 256;
 enum { FMT_Q8_0 = 0, FMT_MXFP4 = 1, FMT_INT4_AFFINE = 2 };
 constexpr int GS_MAX = 30;            // tiles per group (= consumer warps x tiles per warp)
-constexpr int MAX_TOK = 16;
+constexpr int MAX_TOK = 16;           // tokens of one routing block (a router item's columns; an entry's routes)
+constexpr int MAX_LT = 64;            // tokens of one layer-kernel launch (up to four routing blocks)
 constexpr int MAX_K = 8;
 constexpr int MAX_E = 256;
-constexpr int MAX_ENTRIES = MAX_E + 1;  // touched routed experts + the shared pseudo-expert
+// Entries: every touched expert's routes in blocks of at most 16 (so an expert
+// with r routes is ceil(r / 16) entries), then the shared expert in blocks of
+// 16 tokens.  M <= 64 tokens x K <= 8 routes give at most E + 32 routed entries.
+constexpr int MAX_ENTRIES = MAX_E + MAX_LT * MAX_K / MAX_TOK + MAX_LT / MAX_TOK;
 
 TSM_HD int chunk_k(int fmt) { return fmt == FMT_MXFP4 ? 64 : 32; }  // elements of K per chunk
 TSM_HD int unit_bytes(int fmt) { return fmt == FMT_INT4_AFFINE ? UNIT_BYTES_I4 : UNIT_BYTES; }

@@ -33,9 +33,9 @@
 // reading the logits back; here it never leaves the device.
 //
 // The (token, slot) pairs are then grouped by expert into the route list the
-// expert phases walk: per touched expert its first route and count, routes
-// sorted by (expert, token) -- each expert's weights are then streamed once
-// per micro-batch.  The pages' route list is a host-written 16-byte record
+// expert phases walk: routes sorted by (expert, token), cut into entries of at
+// most 16 routes (an expert's weights are streamed once per entry: once per
+// micro-batch for up to 16 routes, once per 16 routes beyond).  The pages' route list is a host-written 16-byte record
 // per route (gpt-oss state page, `batch_routes`); ours is built on the device.
 //
 // The gate/up B operand is x as FP16 scaled by a per-token power of two taken
@@ -63,7 +63,7 @@ constexpr int MAX_SLICES = 64;   // router slices along K
 
 struct RouteParams {
   const __nv_bfloat16* x;  // [M][H]
-  int M, H, Hp, E, K;
+  int M, H, Hp, E, K;      // M: tokens of the launch (layer kernel <= 64, route kernel <= 16)
   int S, CS;               // router slices: S slices of CS chunks (32 K each), the last may be shorter
   const uint8_t* rw;       // router, repacked Q8_0 fragment tiles, tile-major (rows padded to 16)
   MatGeom rg;              // its geometry
@@ -88,23 +88,24 @@ struct RouteParams {
 
 // Routing results, in the shared memory of the kernel that routes.
 struct RouteState {
-  float part[ROUTE_WARPS][16][16];        // per-warp partial logits [row][token]
-  float lg[MAX_TOK][MAX_E];               // logits (before bias)
-  int shift[MAX_TOK];                     // per-token power-of-two scale of x (whole row)
-  float smax[MAX_TOK];                    // |x| max of the current slice
+  float part[ROUTE_WARPS][16][16];        // per-warp partial logits [row][token] of one router item
+  float* lg;                              // logits (before bias) [M][lgld], in the caller's scratch
+  int lgld;
+  int shift[MAX_LT];                      // per-token power-of-two scale of x (whole row)
+  float smax[MAX_TOK];                    // |x| max of the current slice (one routing block)
   int sshift[MAX_TOK];                    // its power-of-two scale
   float gmax[MAX_TOK];                    // running |x| max over the slices (route_kernel)
-  int idx[MAX_TOK * MAX_K];               // selected experts, slot order
-  float w[MAX_TOK * MAX_K];               // their weights
+  int idx[MAX_LT * MAX_K];                // selected experts, slot order
+  float w[MAX_LT * MAX_K];                // their weights
   int off[MAX_E];                         // first route position of each expert
-  int eslot[MAX_E];                       // entry index of each touched expert
-  unsigned tmask[MAX_E];                  // tokens that selected each expert (bit t)
+  int eslot[MAX_E];                       // first entry index of each touched expert
+  unsigned long long tmask[MAX_E];        // tokens that selected each expert (bit t)
   float bias[MAX_E], pes[MAX_E];          // router bias and per-expert scale (read before the dependency wait)
-  int ex[MAX_ENTRIES], ro[MAX_ENTRIES], nc[MAX_ENTRIES];  // touched experts (+ shared entry)
-  int tok[MAX_TOK * MAX_K];               // token of each route position
-  int rpos[MAX_TOK * MAX_K];              // route position of each (token, slot)
-  int rj[MAX_TOK * MAX_K];                // entry index of each route position
-  int nT, nE;
+  int ex[MAX_ENTRIES], ro[MAX_ENTRIES], nc[MAX_ENTRIES];  // entries: expert, first route, routes (<= 16)
+  int tok[MAX_LT * MAX_K];                // token of each route position
+  int rpos[MAX_LT * MAX_K];               // route position of each (token, slot)
+  int rj[MAX_LT * MAX_K];                 // entry index of each route position
+  int nT, nE;                             // routed entries; routed + shared entries
   uint64_t xbar;                          // completion of the bulk copy of an x slice
   uint64_t rbar;                          // completion of the bulk copy of an item's router units
   uint64_t pbar;                          // completion of the bulk copy of the published items
@@ -155,7 +156,7 @@ TSM_DEV void route_init_smem(RouteState& s, const RouteConst& c, int tid) {
   if (tid < MAX_E) {
     s.bias[tid] = c.b;
     s.pes[tid] = c.s;
-    s.tmask[tid] = 0u;
+    s.tmask[tid] = 0ull;
   }
 }
 
@@ -262,16 +263,17 @@ TSM_DEV void slice_input(const RouteParams& p, const RouteState& s, int c, const
   }
 }
 
-// x slice c -> FP16 * 2^shift[t] (whole-row scale) into xh [M][Hp].
-TSM_DEV void slice_xh(const RouteParams& p, const RouteState& s, int c, const __nv_bfloat16* xs, __half* xh,
+// x slice c of a routing block (p.M <= 16 rows, the launch's tokens t0 ..)
+// -> FP16 * 2^shift[t0 + t] (whole-row scale) into rows t0 + t of xh [.][Hp].
+TSM_DEV void slice_xh(const RouteParams& p, const RouteState& s, int c, const __nv_bfloat16* xs, __half* xh, int t0,
                       int tid, int nthr) {
   const int lo = slice_lo(p.CS, c), per_row = (slice_hi(p.CS, p.rg.chunks, c) - lo) * 4;
   for (int i = tid; i < p.M * per_row; i += nthr) {
     const int t = i / per_row, k = (i - t * per_row) * 8;
     const uint4 raw = *reinterpret_cast<const uint4*>(xs + (size_t)t * p.CS * 32 + k);
     uint4 hx, hh, hl;
-    convert8(p, raw, lo * 32 + k, pow2f(s.shift[t]), false, hx, hh, hl);
-    *reinterpret_cast<uint4*>(xh + (size_t)t * p.Hp + lo * 32 + k) = hx;
+    convert8(p, raw, lo * 32 + k, pow2f(s.shift[t0 + t]), false, hx, hh, hl);
+    *reinterpret_cast<uint4*>(xh + (size_t)(t0 + t) * p.Hp + lo * 32 + k) = hx;
   }
 }
 
@@ -345,7 +347,7 @@ TSM_DEV void slice_gemv(const RouteParams& p, RouteState& s, int j, int c, const
     if (pub)
       pub[(size_t)t * item_ld(p.E) + e] = v;
     else
-      s.lg[t][e] += v;
+      s.lg[t * s.lgld + e] += v;
   }
   __syncthreads();
 }
@@ -359,194 +361,191 @@ TSM_DEV unsigned order_key(float f) {
 }
 TSM_DEV float key_value(unsigned k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k); }
 
-// Top-k and weights: warp t handles token t (lane holds experts lane,
-// lane + 32, ...; PER = ceil(E / 32)).  The selection order is (selection
-// logit desc, expert index asc): each step takes the largest key over the
-// warp, then the smallest index holding it.  Each selected (token, expert)
-// also sets the token's bit in the expert's token mask.
+// Top-k and weights: warp w handles tokens w, w + nwarps, ... (lane holds
+// experts lane, lane + 32, ...; PER = ceil(E / 32)).  The selection order is
+// (selection logit desc, expert index asc): each step takes the largest key
+// over the warp, then the smallest index holding it.  Each selected (token,
+// expert) also sets the token's bit in the expert's token mask.
 template <int PER>
-TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lane) {
-  if (warp >= p.M) return;
-  const int t = warp;
+TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lane, int nwarps) {
   const bool biased = p.bias && p.bias_mode != 0;
   const bool score_biased = p.bias && p.bias_mode == 1;
   const bool sig = p.score == 2;  // sigmoid scores; the bias is a selection-only correction
-  unsigned key[PER];
-  float vsc[PER];
+  for (int t = warp; t < p.M; t += nwarps) {
+    const float* lgt = s.lg + (size_t)t * s.lgld;
+    unsigned key[PER];
+    float vsc[PER];
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane + 32 * i;
-    const float l = e < p.E ? s.lg[t][e] : -INFINITY;
-    const float base = sig ? 1.f / (1.f + expf(-l)) : l;
-    const float ls = (e < p.E && biased) ? base + s.bias[e] : base;
-    key[i] = e < p.E ? order_key(ls) : 0u;
-    vsc[i] = score_biased ? ls : l;
-    if (e < p.E) {
-      if (p.logits) p.logits[(size_t)t * p.E + e] = l;
-      if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
-    }
-  }
-  int selk = 0;  // lane k: the k-th selected expert
-  for (int k = 0; k < p.K; ++k) {
-    unsigned bk = 0u;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (key[i] > bk) {  // strict: the lowest index wins among this lane's equal keys
-        bk = key[i];
-        be = lane + 32 * i;
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      const float l = e < p.E ? lgt[e] : -INFINITY;
+      const float base = sig ? 1.f / (1.f + expf(-l)) : l;
+      const float ls = (e < p.E && biased) ? base + s.bias[e] : base;
+      key[i] = e < p.E ? order_key(ls) : 0u;
+      vsc[i] = score_biased ? ls : l;
+      if (e < p.E) {
+        if (p.logits) p.logits[(size_t)t * p.E + e] = l;
+        if (p.logits_out) p.logits_out[(size_t)t * p.E + e] = l;
       }
-    const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
-    int bi = (int)__reduce_min_sync(0xffffffffu, bk == kmax && kmax != 0u ? (unsigned)be : 0x7fffffffu);
-    if (kmax == 0u || bi >= p.E) {  // no candidate left: only with NaN logits
-      if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
-      bi = 0;
     }
+    int selk = 0;  // lane k: the k-th selected expert
+    for (int k = 0; k < p.K; ++k) {
+      unsigned bk = 0u;
+      int be = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (lane + 32 * i == bi) key[i] = 0u;
-    if (lane == k) selk = bi;
-  }
-  const bool act = lane < p.K;
-  if (sig) {  // weights: the selected sigmoid scores renormalised to sum 1
-    const float sk = act ? 1.f / (1.f + expf(-s.lg[t][selk])) : 0.f;
-    float den = sk;
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      for (int i = 0; i < PER; ++i)
+        if (key[i] > bk) {  // strict: the lowest index wins among this lane's equal keys
+          bk = key[i];
+          be = lane + 32 * i;
+        }
+      const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
+      int bi = (int)__reduce_min_sync(0xffffffffu, bk == kmax && kmax != 0u ? (unsigned)be : 0x7fffffffu);
+      if (kmax == 0u || bi >= p.E) {  // no candidate left: only with NaN logits
+        if (lane == 0) atomicOr(p.err, ERR_BAD_INDEX);
+        bi = 0;
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (lane + 32 * i == bi) key[i] = 0u;
+      if (lane == k) selk = bi;
+    }
+    const bool act = lane < p.K;
+    float wv = 0.f;
+    if (sig) {  // weights: the selected sigmoid scores renormalised to sum 1
+      const float sk = act ? 1.f / (1.f + expf(-lgt[selk])) : 0.f;
+      float den = sk;
+      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      wv = act ? sk / den * s.pes[selk] : 0.f;
+    } else {
+      // score logit of the selected expert, recomputed exactly as above
+      float sck = -INFINITY;
+      if (act) {
+        const float l = lgt[selk];
+        sck = score_biased ? l + s.bias[selk] : l;
+      }
+      unsigned mk = act ? order_key(sck) : 0u;
+      if (p.score != 0) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+          if (lane + 32 * i < p.E) mk = max(mk, order_key(vsc[i]));
+      }
+      const float m = key_value(__reduce_max_sync(0xffffffffu, mk));
+      float den = 0.f;
+      if (p.score == 0) {
+        den = act ? expf(sck - m) : 0.f;
+      } else {
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+          if (lane + 32 * i < p.E) den += expf(vsc[i] - m);
+      }
+      for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (act) wv = expf(sck - m) / den * s.pes[selk];
+    }
     if (act) {
-      const float wv = sk / den * s.pes[selk];
       s.idx[t * p.K + lane] = selk;
       s.w[t * p.K + lane] = wv;
-      atomicOr(&s.tmask[selk], 1u << t);
+      atomicOr(&s.tmask[selk], 1ull << t);
       if (p.idx) p.idx[t * p.K + lane] = selk;
       if (p.w) p.w[t * p.K + lane] = wv;
       if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
       if (p.w_out) p.w_out[t * p.K + lane] = wv;
     }
-    return;
-  }
-  // score logit of the selected expert, recomputed exactly as above
-  float sck = -INFINITY;
-  if (act) {
-    const float l = s.lg[t][selk];
-    sck = score_biased ? l + s.bias[selk] : l;
-  }
-  unsigned mk = act ? order_key(sck) : 0u;
-  if (p.score != 0) {
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (lane + 32 * i < p.E) mk = max(mk, order_key(vsc[i]));
-  }
-  const float m = key_value(__reduce_max_sync(0xffffffffu, mk));
-  float den = 0.f;
-  if (p.score == 0) {
-    den = act ? expf(sck - m) : 0.f;
-  } else {
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (lane + 32 * i < p.E) den += expf(vsc[i] - m);
-  }
-  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  if (act) {
-    const float wv = expf(sck - m) / den * s.pes[selk];
-    s.idx[t * p.K + lane] = selk;
-    s.w[t * p.K + lane] = wv;
-    atomicOr(&s.tmask[selk], 1u << t);
-    if (p.idx) p.idx[t * p.K + lane] = selk;
-    if (p.w) p.w[t * p.K + lane] = wv;
-    if (p.idx_out) p.idx_out[t * p.K + lane] = selk;
-    if (p.w_out) p.w_out[t * p.K + lane] = wv;
   }
 }
 
-TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane) {
+TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane, int nwarps) {
   if (p.E <= 32)
-    route_topk_t<1>(p, s, warp, lane);
+    route_topk_t<1>(p, s, warp, lane, nwarps);
   else if (p.E <= 64)
-    route_topk_t<2>(p, s, warp, lane);
+    route_topk_t<2>(p, s, warp, lane, nwarps);
   else if (p.E <= 128)
-    route_topk_t<4>(p, s, warp, lane);
+    route_topk_t<4>(p, s, warp, lane, nwarps);
   else
-    route_topk_t<8>(p, s, warp, lane);
+    route_topk_t<8>(p, s, warp, lane, nwarps);
 }
 
 // Route list: the (token, slot) pairs grouped by expert (touched experts in
-// ascending order, tokens ascending), plus the shared expert as the last
-// entry with all M tokens.  A token selects an expert at most once, so the
-// expert's route count is the popcount of its token mask (set by
-// route_topk) and a token's rank among them the popcount of the mask's lower
-// bits.  Needs s.tmask cleared (route_init_smem) and a CTA barrier after
-// route_topk; ends with one.
+// ascending order, tokens ascending), cut into entries of at most 16 routes,
+// then the shared expert's entries (all M tokens, 16 per entry).  A token
+// selects an expert at most once, so the expert's route count is the
+// popcount of its token mask (set by route_topk) and a token's rank among
+// them the popcount of the mask's lower bits.  A shared entry's routes are
+// M K + its tokens, so every entry's route r of column n is ro + n.  Needs
+// s.tmask cleared (route_init_smem) and a CTA barrier after route_topk; ends
+// with one.
 TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
   const int MK = p.M * p.K;
   if (warp == 0) {
     constexpr int PER = MAX_E / 32;
-    int cl[PER], tot = 0, nz = 0;
+    int cl[PER], tot = 0, ne = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane * PER + i;
-      cl[i] = e < p.E ? __popc(s.tmask[e]) : 0;
+      cl[i] = e < p.E ? __popcll(s.tmask[e]) : 0;
       tot += cl[i];
-      nz += cl[i] > 0;
+      ne += (cl[i] + MAX_TOK - 1) / MAX_TOK;
     }
-    int incl = tot, nzincl = nz;
+    int incl = tot, neincl = ne;
     for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o), w = __shfl_up_sync(0xffffffffu, nzincl, o);
+      const int v = __shfl_up_sync(0xffffffffu, incl, o), w = __shfl_up_sync(0xffffffffu, neincl, o);
       if (lane >= o) {
         incl += v;
-        nzincl += w;
+        neincl += w;
       }
     }
-    int run = incl - tot, slot = nzincl - nz;
+    int run = incl - tot, slot = neincl - ne;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int e = lane * PER + i;
       if (e < p.E) {
         s.off[e] = run;
-        if (cl[i]) {
-          s.eslot[e] = slot;
+        s.eslot[e] = slot;
+        for (int q = 0; q < cl[i]; q += MAX_TOK, ++slot) {
           s.ex[slot] = e;
-          s.ro[slot] = run;
-          s.nc[slot] = cl[i];
+          s.ro[slot] = run + q;
+          s.nc[slot] = min(MAX_TOK, cl[i] - q);
           if (p.meta) {
             p.meta[META_EX + slot] = e;
-            p.meta[META_RO + slot] = run;
-            p.meta[META_NC + slot] = cl[i];
+            p.meta[META_RO + slot] = run + q;
+            p.meta[META_NC + slot] = min(MAX_TOK, cl[i] - q);
           }
-          ++slot;
         }
         run += cl[i];
       }
     }
-    const int nT = __shfl_sync(0xffffffffu, nzincl, 31);
+    const int nT = __shfl_sync(0xffffffffu, neincl, 31);
+    const int nsh = p.has_shared ? (p.M + MAX_TOK - 1) / MAX_TOK : 0;
+    if (lane < nsh) {
+      const int j = nT + lane, n = min(MAX_TOK, p.M - MAX_TOK * lane);
+      s.ex[j] = p.E;
+      s.ro[j] = MK + MAX_TOK * lane;
+      s.nc[j] = n;
+      if (p.meta) {
+        p.meta[META_EX + j] = p.E;
+        p.meta[META_RO + j] = MK + MAX_TOK * lane;
+        p.meta[META_NC + j] = n;
+      }
+    }
     if (lane == 0) {
       s.nT = nT;
-      s.nE = nT + (p.has_shared ? 1 : 0);
-      if (p.has_shared) {
-        s.ex[nT] = p.E;
-        s.ro[nT] = MK;
-        s.nc[nT] = p.M;
-      }
+      s.nE = nT + nsh;
       if (p.meta) {
-        if (p.has_shared) {
-          p.meta[META_EX + nT] = p.E;
-          p.meta[META_RO + nT] = MK;
-          p.meta[META_NC + nT] = p.M;
-        }
         p.meta[META_M] = p.M;
         p.meta[META_NT] = nT;
         p.meta[META_MK] = MK;
         p.meta[META_HAS_SHARED] = p.has_shared;
-        p.meta[META_NE] = s.nE;
+        p.meta[META_NE] = nT + nsh;
       }
     }
   }
   __syncthreads();
   for (int i = tid; i < MK; i += nthr) {
     const int e = s.idx[i], tk = i / p.K;
-    const int pos = s.off[e] + __popc(s.tmask[e] & ((1u << tk) - 1u));  // tokens before tk that chose e
+    const int rank = __popcll(s.tmask[e] & ((1ull << tk) - 1ull));  // tokens before tk that chose e
+    const int pos = s.off[e] + rank;
     s.tok[pos] = tk;
     s.rpos[i] = pos;
-    s.rj[pos] = s.eslot[e];
+    s.rj[pos] = s.eslot[e] + rank / MAX_TOK;
     if (p.routes) {
       Route r;
       r.token = tk;
@@ -590,6 +589,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
   __half* xin = reinterpret_cast<__half*>(sbuf + L.xin);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const RouteConst rc = route_const_load(p, tid);
+  s.lg = reinterpret_cast<float*>(sbuf + align128(L.total));  // [M][E]
+  s.lgld = p.E;
   if (tid == 0) {
     mbar_init(&s.xbar, 1);
     fence_barrier_init();
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
   // the bias and per-expert scale are device inputs here: a non-finite one is an error of the call
   if (tid < p.E && !(isfinite(rc.b) && isfinite(rc.s))) atomicOr(p.err, ERR_BAD_ROUTER_INPUT);
   route_init_smem(s, rc, tid);
-  for (int i = tid; i < p.M * MAX_E; i += ROUTE_THREADS) s.lg[i / MAX_E][i % MAX_E] = 0.f;
+  for (int i = tid; i < p.M * p.E; i += ROUTE_THREADS) s.lg[i] = 0.f;
   if (tid < MAX_TOK) s.gmax[tid] = 0.f;
   __syncthreads();
   for (int c = 0; c < p.S; ++c) {
@@ -626,7 +627,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
     if (p.shift) p.shift[tid] = s.shift[tid];
   }
   __syncthreads();
-  route_topk(p, s, warp, lane);
+  route_topk(p, s, warp, lane, ROUTE_WARPS);
   __syncthreads();
   route_list(p, s, warp, lane, tid, ROUTE_THREADS);
   if (p.sentinel) route_sentinel(p, tid);

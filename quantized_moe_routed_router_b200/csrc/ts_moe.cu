@@ -50,7 +50,9 @@ size_t blob_row_bytes(int fmt, int cols) {
 struct ts_moe {
   ts_moe_config cfg{};
   int sm_count = 0, nb = 0;
-  int slices[MAX_TOK + 1] = {};  // router slices per token count
+  int slices[MAX_TOK + 1] = {};  // router slices per token count (calls of at most 16 tokens)
+  int lt = 0;                    // tokens per layer-kernel launch: 64, or 16 when no slicing fits four blocks
+  int s_chunk = 0;               // router slices of every launch of a call with more than 16 tokens
   int Hp = 0, Ip = 0, Sp = 0;
   MatGeom gR{}, gB{}, gC{}, gBs{}, gCs{};
   int ng_max_B = 0;
@@ -167,28 +169,31 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
   return TS_MOE_OK;
 }
 
-// Dynamic shared memory of route_kernel: RouteState, then one item's slice buffers.
+// Dynamic shared memory of route_kernel: RouteState, one item's slice buffers, the logits.
 constexpr int ROUTE_SMEM_MAX = 220 * 1024;
 size_t route_smem(const RouteParams& rp) {
-  return align128(sizeof(RouteState)) + SliceSmem(rp.M, rp.CS, rp.xscale != nullptr).total;
+  return align128(sizeof(RouteState)) + align128(SliceSmem(rp.M, rp.CS, rp.xscale != nullptr).total) +
+         (size_t)rp.M * rp.E * 4;
 }
 
-// Router slices for M tokens: the count S (CS = ceil(C / S) chunks each) that
-// balances the bytes a routing CTA loads (its x slice and CS router units)
-// against the bytes every CTA reads back (S items of M x E logits), with the
-// T * S routing CTAs within the grid and one item's buffers within the
-// layer kernel's weight and window rings.  Returns 0 when no S fits.
+// Router slices for a launch of `ml` tokens cut into `ntb` routing blocks of
+// at most M tokens: the count S (CS = ceil(C / S) chunks each) that balances
+// the bytes a routing CTA loads (its block's x slice and CS router units)
+// against the bytes every CTA reads back (S items of ml x E logits), with the
+// T * S * ntb routing CTAs within the grid and one item's buffers plus the
+// launch's logits within the layer kernel's weight and window rings.
+// Returns 0 when no S fits.
 constexpr size_t RING_BYTES = sizeof(LayerSmem::w) + sizeof(LayerSmem::x);
-int choose_slices(int M, int C, int T, int E, int nb, bool split) {
+int choose_slices(int M, int C, int T, int E, int nb, bool split, int ntb, int ml) {
   int best = 0;
   double best_cost = 0.0;
-  const int smax = std::min({C, MAX_SLICES, nb / std::max(T, 1)});
+  const int smax = std::min({C, MAX_SLICES, nb / std::max(T * ntb, 1)});
   for (int S = 1; S <= smax; ++S) {
     const int CS = (C + S - 1) / S;
     if ((C + CS - 1) / CS != S) continue;  // S must be the slice count CS gives
-    if (SliceSmem(M, CS, split).total > RING_BYTES) continue;
+    if (align128(SliceSmem(M, CS, split).total) + (size_t)ml * E * 4 > RING_BYTES) continue;
     const double load = (double)M * CS * 64 + (double)CS * UNIT_BYTES;
-    const double read = (double)S * (M * item_ld(E) + MAX_TOK) * 4;
+    const double read = (double)S * (ml * item_ld(E) + MAX_LT) * 4;
     const double cost = std::max(load, read);
     if (best == 0 || cost < best_cost) {
       best = S;
@@ -206,7 +211,7 @@ int layer_ctas(int sm_count) { return std::min(sm_count, MAX_NB); }
 // the same router and SM count both sum a logit's partial products in the same
 // order (the allocation-free path matches a handle opened without an x-scale).
 bool router_slicing(int M, const MatGeom& gR, int E, int nb, bool split, int& S, int& CS) {
-  const int s = choose_slices(M, gR.chunks, gR.tiles, E, nb, split);
+  const int s = choose_slices(M, gR.chunks, gR.tiles, E, nb, split, 1, M);
   if (s == 0) return false;
   CS = (gR.chunks + s - 1) / s;
   S = (gR.chunks + CS - 1) / CS;
@@ -288,22 +293,11 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   h->cfg = *cfg;
   const ts_moe_config& c = h->cfg;
   const int H = c.hidden, I = c.moe_inter, E = c.num_experts, K = c.top_k, S = c.shared_inter;
-  // The workspace holds one launch's tokens: a call with more runs in chunks.
-  const int Mx = std::min(c.max_tokens, TS_MOE_MAX_TOKENS);
-  const int fmt = c.expert_fmt;
-  h->sm_count = prop.multiProcessorCount;
-  h->nb = layer_ctas(h->sm_count);
-  h->Hp = round_up(H, 64);
-  h->Ip = round_up(I, 64);
-  h->Sp = S ? round_up(S, 64) : 0;
+  // Calls above 16 tokens run in launches of up to 64 tokens (four routing
+  // blocks) when a router slicing fits that, else of 16; the workspace holds
+  // one launch's tokens.
+  h->nb = layer_ctas(prop.multiProcessorCount);
   h->gR = make_router_geom(E, H);
-  h->gB = make_geom(I / 8, H, fmt);
-  h->gC = make_geom(H / 16, I, fmt);
-  if (S) {
-    h->gBs = make_geom(S / 8, H, TS_FMT_Q8_0);
-    h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
-  }
-  h->ng_max_B = std::max(h->gB.ngroups, S ? h->gBs.ngroups : 0);
   for (int l = 0; l < c.num_layers && !h->any_xscale; ++l)
     if (layers[l].router_xscale)
       for (int n = 0; n < H; ++n)
@@ -311,7 +305,28 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
           h->any_xscale = true;
           break;
         }
-  for (int m = 1; m <= Mx; ++m) {
+  h->s_chunk = choose_slices(MAX_TOK, h->gR.chunks, h->gR.tiles, E, h->nb, h->any_xscale, MAX_LT / MAX_TOK, MAX_LT);
+  h->lt = h->s_chunk ? MAX_LT : MAX_TOK;
+  if (!h->s_chunk) h->s_chunk = choose_slices(MAX_TOK, h->gR.chunks, h->gR.tiles, E, h->nb, h->any_xscale, 1, MAX_TOK);
+  const int Mx = std::min(c.max_tokens, h->lt);
+  const int fmt = c.expert_fmt;
+  h->sm_count = prop.multiProcessorCount;
+  h->Hp = round_up(H, 64);
+  h->Ip = round_up(I, 64);
+  h->Sp = S ? round_up(S, 64) : 0;
+  h->gB = make_geom(I / 8, H, fmt);
+  h->gC = make_geom(H / 16, I, fmt);
+  if (S) {
+    h->gBs = make_geom(S / 8, H, TS_FMT_Q8_0);
+    h->gCs = make_geom(H / 16, S, TS_FMT_Q8_0);
+  }
+  h->ng_max_B = std::max(h->gB.ngroups, S ? h->gBs.ngroups : 0);
+  if (c.max_tokens > MAX_TOK && h->s_chunk == 0) {
+    g_open_error = "no router slicing fits these sizes (too many experts for the SM count, or hidden too large)";
+    ts_moe_close(h);
+    return TS_MOE_EUNSUPPORTED;
+  }
+  for (int m = 1; m <= std::min(Mx, MAX_TOK); ++m) {
     int S_m = 0, CS_m = 0;
     h->slices[m] = router_slicing(m, h->gR, E, h->nb, h->any_xscale, S_m, CS_m) ? S_m : 0;
     if (h->slices[m] == 0) {
@@ -384,14 +399,14 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_routes = slot((size_t)Mx * K * sizeof(Route));
     const size_t o_xh = slot((size_t)Mx * h->Hp * 2);
     const size_t o_part = slot((size_t)MAX_SLICES * Mx * item_ld(E) * 4);
-    const size_t o_max = slot((size_t)MAX_SLICES * MAX_TOK * 4);
+    const size_t o_max = slot((size_t)MAX_SLICES * MAX_LT * 4);
     const size_t o_acts = slot((size_t)Mx * K * h->Ip * 2);
     const size_t o_acts_sh = slot((size_t)Mx * std::max(h->Sp, 64) * 2);
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_cnt = off;
-    const size_t n_cnt = 2 + (size_t)(E + 1) * h->ng_max_B * NWC + (E + 1) + 2 + 1;  // arrivals (u64) + ... + grid[2] + error word
+    const size_t n_cnt = 2 + (size_t)MAX_ENTRIES * h->ng_max_B * NWC + MAX_ENTRIES + 2 + 1;  // arrivals (u64) + ... + grid[2] + error word
     slot(n_cnt * 4);
     h->ws_bytes = off;
     ce = cudaMalloc(&h->ws, h->ws_bytes);
@@ -420,8 +435,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->counters_bytes = n_cnt * 4;
     h->arrivals = (unsigned long long*)cn;  // 256-byte aligned: first in the counter block
     h->cnt_gB = cn + 2;
-    h->entry_done = h->cnt_gB + (size_t)(E + 1) * h->ng_max_B * NWC;
-    h->grid = h->entry_done + (E + 1);  // x slices written, router items published
+    h->entry_done = h->cnt_gB + (size_t)MAX_ENTRIES * h->ng_max_B * NWC;
+    h->grid = h->entry_done + MAX_ENTRIES;  // x slices written, router items published
     h->err = h->grid + 2;
     // zeros: counters, error word, and the padding columns of x / acts
     ce = cudaMemset(h->ws, 0, h->ws_bytes);
@@ -556,7 +571,11 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   return TS_MOE_OK;
 }
 
-static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
+// A launch of M tokens within a call of call_m tokens: calls of at most 16
+// tokens take the slicing chosen for their M, every launch of a longer call
+// the one chosen for chunks, so that ts_moe_route and ts_moe_forward on the
+// same call sum each logit's partial products in the same order.
+static RouteParams route_params(ts_moe* h, int layer, const void* x, int M, int call_m) {
   const ts_moe_config& c = h->cfg;
   const LayerDev& d = h->layers[layer];
   RouteParams rp;
@@ -579,7 +598,12 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M) {
   rp.idx = h->idx;
   rp.w = h->w;
   rp.shift = h->shift;
-  router_slicing(M, h->gR, rp.E, h->nb, h->any_xscale, rp.S, rp.CS);  // fits: checked at open
+  if (call_m > MAX_TOK) {
+    rp.CS = (h->gR.chunks + h->s_chunk - 1) / h->s_chunk;
+    rp.S = (h->gR.chunks + rp.CS - 1) / rp.CS;
+  } else {
+    router_slicing(M, h->gR, rp.E, h->nb, h->any_xscale, rp.S, rp.CS);  // fits: checked at open
+  }
   rp.meta = h->meta;
   rp.routes = h->routes;
   rp.rpos = h->rpos;
@@ -602,12 +626,14 @@ static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t
   return TS_MOE_OK;
 }
 
-// A call of M tokens runs as ceil(M / 16) launches over consecutive row blocks:
-// full 16-token chunks first, the remainder last.  Tokens are independent in
-// the routed half, so the chunking changes no token's route or its math (the
-// chunked-prefill driver of the gpt-oss state page, `BatchedRoutedScratch`,
-// feeds the routed half MAX_PREFILL_BATCH rows at a time the same way).
-static inline int chunk_rows(int M, int m0) { return std::min(TS_MOE_MAX_TOKENS, M - m0); }
+// A call of M tokens runs as launches over consecutive row blocks, full ones
+// first: ts_moe_forward in launches of h->lt (64) tokens, each of which reads
+// every touched expert's weights once per 16 routes; ts_moe_route in launches
+// of 16.  Tokens are independent in the routed half, so the chunking changes
+// no token's route (the chunked-prefill driver of the gpt-oss state page,
+// `BatchedRoutedScratch`, feeds the routed half MAX_PREFILL_BATCH = 16 rows
+// at a time; here a launch takes up to four such blocks).
+static inline int chunk_rows(int M, int m0, int n) { return std::min(n, M - m0); }
 
 ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
                            void* stream) {
@@ -616,8 +642,8 @@ ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* 
   if (M == 0) return TS_MOE_OK;
   if (!idx || !w) return fail(h, TS_MOE_EINVAL, "idx and w must be non-NULL");
   const int H = h->cfg.hidden, E = h->cfg.num_experts, K = h->cfg.top_k;
-  for (int m0 = 0; m0 < M; m0 += TS_MOE_MAX_TOKENS) {
-    RouteParams rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0));
+  for (int m0 = 0; m0 < M; m0 += MAX_TOK) {
+    RouteParams rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, MAX_TOK), M);
     rp.idx_out = idx + (size_t)m0 * K;
     rp.w_out = w + (size_t)m0 * K;
     rp.logits_out = logits ? logits + (size_t)m0 * E : nullptr;
@@ -673,8 +699,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   const size_t smem = sizeof(LayerSmem);
   const int H = c.hidden;
   if (h->timing) cudaEventRecord(h->ev[0], st);
-  for (int m0 = 0; m0 < M; m0 += TS_MOE_MAX_TOKENS) {
-    lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0));
+  for (int m0 = 0; m0 < M; m0 += h->lt) {
+    lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, h->lt), M);
     lp.y = y ? y + (size_t)m0 * H : nullptr;
     lp.resid = resid ? (__nv_bfloat16*)resid + (size_t)m0 * H : nullptr;
     cudaError_t e;
@@ -715,6 +741,7 @@ ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info) {
   info->shared_bytes = h->shared_bytes;
   info->num_ctas = h->nb;
   info->sm_count = h->sm_count;
+  info->launch_tokens = h->lt;
   return TS_MOE_OK;
 }
 

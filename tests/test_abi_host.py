@@ -221,6 +221,7 @@ def test_header_constants_match_the_binding_and_the_generator(B):
         (synth.BIAS_NONE, synth.BIAS_LOGITS, synth.BIAS_SELECT_ONLY)
     assert (h["TS_ACT_SWIGLU"], h["TS_ACT_SWIGLU_CLAMPED"]) == (synth.ACT_SWIGLU, synth.ACT_SWIGLU_CLAMPED)
     assert (h["TS_MOE_MAX_TOKENS"], h["TS_MOE_MAX_TOPK"], h["TS_MOE_MAX_EXPERTS"]) == (16, 8, 256)
+    assert h["TS_MOE_MAX_LAUNCH_TOKENS"] == 64
     assert h["TS_MOE_OK"] == 0 and h["TS_MOE_EDEVICE"] == 5
 
 
