@@ -817,7 +817,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.rpos = nullptr;
   }
   const int M = rp.M, NTB = (M + MAX_TOK - 1) / MAX_TOK;
-  const int S = rp.S, TS = rp.rg.tiles * S, nR = TS * NTB;
+  const int S = rp.S, TS = rp.rg.tiles * S, nR = rp.whole ? 0 : TS * NTB;
   const bool rcta = b < nR;
   const int rtb = rcta ? b / TS : 0, rrem = rcta ? b % TS : 0;
   const int rj = rrem / S, rcs = rrem % S;
@@ -825,8 +825,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   RouteParams bp = rp;  // this CTA's routing block: rows t0 .. t0 + mb - 1 of x
   bp.x = rp.x + (size_t)t0 * rp.H;
   bp.M = min(MAX_TOK, M - t0);
-  // the item's buffers sit in the still idle weight and window rings
+  // the routing buffers sit in the still idle weight and window rings
   const SliceSmem L(min(M, MAX_TOK), rp.CS, rp.xscale != nullptr);
+  const WholeSmem WS(M, rp.H, rp.rg.tiles, rp.rg.chunks, S, rp.CS, rp.E, rp.xscale != nullptr);
   uint8_t* ring = &s.w[0][0];
   constexpr size_t ring_bytes = sizeof(s.w) + sizeof(s.x);  // w and x are adjacent
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(ring + L.xs);
@@ -847,88 +848,109 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     mbar_init(&s.r.pbar, 1);
     fence_barrier_init();
     s.dead = 0;
-    if (rcta) slice_issue_router(bp, s.r, rj, rcs, rt);
+    if (rp.whole) {  // the router is a weight: fetched before the dependency wait
+      const unsigned rbytes = (unsigned)rp.rg.tiles * rp.rg.chunks * UNIT_BYTES;
+      mbar_arrive_expect_tx(&s.r.rbar, rbytes);
+      bulk_g2s(ring + WS.rt, rp.rw, rbytes, &s.r.rbar);
+    } else if (rcta) {
+      slice_issue_router(bp, s.r, rj, rcs, rt);
+    }
   }
   grid_dep_wait();
   grid_dep_launch();
   if (tid == 0) {
-    if (rcta) slice_issue_x(bp, s.r, rcs, xs);
+    if (rp.whole) {
+      const unsigned xbytes = (unsigned)M * rp.H * 2;
+      mbar_arrive_expect_tx(&s.r.xbar, xbytes);
+      bulk_g2s(ring + WS.x, rp.x, xbytes, &s.r.xbar);
+    } else if (rcta) {
+      slice_issue_x(bp, s.r, rcs, xs);
+    }
     // floor(count / NB), exact in FP64 for counts below 2^53 (no 64-bit integer division)
     s.gen0 = (unsigned long long)floor((double)ld_acquire_u64(p.grid_cnt) / (double)NB);
   }
   route_init_smem(s.r, rc, tid);
   __syncthreads();
-  if (rcta) {
-    mbar_wait(&s.r.xbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
-    slice_max(bp, s.r, rcs, xs, warp, lane);
-    __syncthreads();
-    slice_input(bp, s.r, rcs, xs, xin, tid, NTHREADS);
-    __syncthreads();
-    mbar_wait(&s.r.rbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
-    float* pub = p.part_pub + ((size_t)rcs * M + t0) * item_ld(rp.E);
-    if (bp.M > 8)
-      slice_gemv<2>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
-    else
-      slice_gemv<1>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
-    if (rj == 0 && tid < bp.M) p.max_pub[rcs * MAX_LT + t0 + tid] = s.r.smax[tid];
-    __syncthreads();
-    if (tid == 0) red_release_add_u32(p.route_cnt, 1u);  // publishes the item written by the whole CTA
-  }
-  // every item published (bounded); then the S items and slice maxima are
-  // brought in by two bulk copies when they fit past the item buffers (with
-  // the logits after them)
-  const int ild = item_ld(rp.E);
-  const unsigned ibytes = (unsigned)((size_t)S * M * ild * 4), mbytes = (unsigned)S * MAX_LT * 4;
-  const size_t pst = align128(L.total), lgbytes = (size_t)M * rp.E * 4;
-  const bool bulk_items = pst + ibytes + mbytes + lgbytes <= ring_bytes;
-  const float* items = bulk_items ? reinterpret_cast<const float*>(ring + pst) : p.part_pub;
-  const float* maxes = bulk_items ? reinterpret_cast<const float*>(ring + pst + ibytes) : p.max_pub;
-  s.r.lg = reinterpret_cast<float*>(ring + (bulk_items ? pst + ibytes + mbytes : pst));  // fits: checked at open
-  s.r.lgld = rp.E;
-  if (tid == 0) {
-    const unsigned long long tw = globaltimer();
-    while (ld_acquire_u32(p.route_cnt) < (unsigned)nR) {
-      if (globaltimer() - tw > WAIT_LIMIT_NS) {
-        s.dead = 1;
-        atomicOr(p.err, ERR_TIMEOUT_ROUTE);
-        break;
+  __half* xh_src = p.xh;
+  bool xwriter = false;
+  if (rp.whole) {
+    // few tokens, small router: every CTA routes by itself (and writes the whole xh)
+    route_whole(rp, s.r, ring, WS, xh_src, &s.dead, warp, lane, tid, NTHREADS);
+    for (int i = tid; i < M * rp.E; i += NTHREADS)
+      if (b == 0 && p.rp.logits) p.rp.logits[i] = s.r.lg[i];
+    if (tid < M && rp.shift) rp.shift[tid] = s.r.shift[tid];
+  } else {
+    if (rcta) {
+      mbar_wait(&s.r.xbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+      slice_max(bp, s.r, rcs, xs, warp, lane);
+      __syncthreads();
+      slice_input(bp, s.r, rcs, xs, xin, tid, NTHREADS);
+      __syncthreads();
+      mbar_wait(&s.r.rbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+      float* pub = p.part_pub + ((size_t)rcs * M + t0) * item_ld(rp.E);
+      if (bp.M > 8)
+        slice_gemv<2>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
+      else
+        slice_gemv<1>(bp, s.r, rj, rcs, xin, rt, warp, lane, tid, NTHREADS, pub);
+      if (rj == 0 && tid < bp.M) p.max_pub[rcs * MAX_LT + t0 + tid] = s.r.smax[tid];
+      __syncthreads();
+      if (tid == 0) red_release_add_u32(p.route_cnt, 1u);  // publishes the item written by the whole CTA
+    }
+    // every item published (bounded); then the S items and slice maxima are
+    // brought in by two bulk copies when they fit past the item buffers (with
+    // the logits after them)
+    const int ild = item_ld(rp.E);
+    const unsigned ibytes = (unsigned)((size_t)S * M * ild * 4), mbytes = (unsigned)S * MAX_LT * 4;
+    const size_t pst = align128(L.total), lgbytes = (size_t)M * rp.E * 4;
+    const bool bulk_items = pst + ibytes + mbytes + lgbytes <= ring_bytes;
+    const float* items = bulk_items ? reinterpret_cast<const float*>(ring + pst) : p.part_pub;
+    const float* maxes = bulk_items ? reinterpret_cast<const float*>(ring + pst + ibytes) : p.max_pub;
+    s.r.lg = reinterpret_cast<float*>(ring + (bulk_items ? pst + ibytes + mbytes : pst));  // fits: checked at open
+    s.r.lgld = rp.E;
+    if (tid == 0) {
+      const unsigned long long tw = globaltimer();
+      while (ld_acquire_u32(p.route_cnt) < (unsigned)nR) {
+        if (globaltimer() - tw > WAIT_LIMIT_NS) {
+          s.dead = 1;
+          atomicOr(p.err, ERR_TIMEOUT_ROUTE);
+          break;
+        }
+      }
+      if (bulk_items && !s.dead) {  // (no copy left in flight when the wait gave up)
+        fence_proxy_async_global();  // written by other CTAs' generic stores, read by bulk copies
+        mbar_arrive_expect_tx(&s.r.pbar, ibytes + mbytes);
+        bulk_g2s(ring + pst, p.part_pub, ibytes, &s.r.pbar);
+        bulk_g2s(ring + pst + ibytes, p.max_pub, mbytes, &s.r.pbar);
       }
     }
-    if (bulk_items && !s.dead) {  // (no copy left in flight when the wait gave up)
-      fence_proxy_async_global();  // written by other CTAs' generic stores, read by bulk copies
-      mbar_arrive_expect_tx(&s.r.pbar, ibytes + mbytes);
-      bulk_g2s(ring + pst, p.part_pub, ibytes, &s.r.pbar);
-      bulk_g2s(ring + pst + ibytes, p.max_pub, mbytes, &s.r.pbar);
+    __syncthreads();
+    if (bulk_items) mbar_wait(&s.r.pbar, 0, &s.dead, p.err, ERR_TIMEOUT_ROUTE);
+    // logits: the items added in slice order; shift from the max of the slice maxima
+    for (int i = tid; i < M * rp.E; i += NTHREADS) {
+      const int t = i / rp.E, e = i - t * rp.E;
+      float v = 0.f;
+  #pragma unroll 8
+      for (int c = 0; c < S; ++c) {
+        const float* src = items + ((size_t)c * M + t) * ild + e;
+        v += bulk_items ? *src : ld_cg(src);
+      }
+      s.r.lg[i] = v;
+      if (b == 0 && p.rp.logits) p.rp.logits[i] = v;
     }
-  }
-  __syncthreads();
-  if (bulk_items) mbar_wait(&s.r.pbar, 0, &s.dead, p.err, ERR_TIMEOUT_ROUTE);
-  // logits: the items added in slice order; shift from the max of the slice maxima
-  for (int i = tid; i < M * rp.E; i += NTHREADS) {
-    const int t = i / rp.E, e = i - t * rp.E;
-    float v = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < S; ++c) {
-      const float* src = items + ((size_t)c * M + t) * ild + e;
-      v += bulk_items ? *src : ld_cg(src);
+    if (tid < M) {
+      float m = 0.f;
+      for (int c = 0; c < S; ++c) {
+        const float* src = maxes + c * MAX_LT + tid;
+        m = fmaxf(m, bulk_items ? *src : ld_cg(src));
+      }
+      s.r.shift[tid] = shift_of_max(m);
+      if (rp.shift) rp.shift[tid] = s.r.shift[tid];
     }
-    s.r.lg[i] = v;
-    if (b == 0 && p.rp.logits) p.rp.logits[i] = v;
+    __syncthreads();
+    // gate/up B operand: this CTA's slice of its block's x as FP16, published with the count of slices written
+    xwriter = rcta && rj == 0;
+    if (xwriter) slice_xh(bp, s.r, rcs, xs, xh_src, t0, tid, NTHREADS);
   }
-  if (tid < M) {
-    float m = 0.f;
-    for (int c = 0; c < S; ++c) {
-      const float* src = maxes + c * MAX_LT + tid;
-      m = fmaxf(m, bulk_items ? *src : ld_cg(src));
-    }
-    s.r.shift[tid] = shift_of_max(m);
-    if (rp.shift) rp.shift[tid] = s.r.shift[tid];
-  }
-  __syncthreads();
-  // gate/up B operand: this CTA's slice of its block's x as FP16, published with the count of slices written
-  __half* xh_src = p.xh;
-  const bool xwriter = rcta && rj == 0;
-  if (xwriter) slice_xh(bp, s.r, rcs, xs, xh_src, t0, tid, NTHREADS);
   route_topk(rp, s.r, warp, lane, NTHREADS / 32);
   __syncthreads();
   if (xwriter && tid == 0) red_release_add_u32(p.xh_cnt, 1u);  // after the barrier: the CTA's slice of xh
@@ -952,8 +974,11 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     int wuse[NSW], xuse[NSX];
     for (int i = 0; i < NSW; ++i) wuse[i] = 0;
     for (int i = 0; i < NSX; ++i) xuse[i] = 0;
-    // gate/up reads x written by the slice CTAs: wait for all S slices
-    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, true);
+    // gate/up reads x written by the routing CTAs: wait for all their slices;
+    // routed with the whole router, this CTA wrote all of x itself, before the
+    // barriers above (its generic writes, read by the window bulk copies)
+    if (rp.whole) fence_proxy_async_global();
+    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, !rp.whole);
     if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, false);
     // Copies still in flight must land before the CTA can exit (only matters
     // when a wait gave up): wait, bounded, for each slot's last issued phase.

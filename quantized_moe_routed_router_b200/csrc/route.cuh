@@ -84,6 +84,7 @@ struct RouteParams {
   float* logits_out;
   const unsigned* pre_err; // route_kernel only: a word an earlier kernel of the same call set on bad input, or null
   int sentinel;            // route_kernel only: on any error, overwrite idx_out / w_out with -1 / 0
+  int whole;               // 1: every routing CTA holds the whole router and x (route_whole), 0: router items
 };
 
 // Routing results, in the shared memory of the kernel that routes.
@@ -133,6 +134,24 @@ struct SliceSmem {
     xin = align128((size_t)M * CS * 64);
     rt = xin + align128((size_t)(split ? 2 : 1) * M * slice_ld(CS) * 2);
     total = rt + align128((size_t)CS * UNIT_BYTES);
+  }
+};
+
+// Shared memory of route_whole: the whole repacked router [T][C] units, x
+// [M][H] BF16, the router input of every slice [S][halves][M][slice_ld(CS)]
+// FP16, the slice maxima and shifts [M][S], the items [T][S][16][M] FP32 and
+// the logits [M][E] FP32.
+struct WholeSmem {
+  size_t rt, x, xin, smx, ssh, item, lg, total;
+  TSM_HD WholeSmem(int M, int H, int T, int C, int S, int CS, int E, bool split) {
+    rt = 0;
+    x = align128((size_t)T * C * UNIT_BYTES);
+    xin = x + align128((size_t)M * H * 2);
+    smx = xin + align128((size_t)S * (split ? 2 : 1) * M * slice_ld(CS) * 2);
+    ssh = smx + align128((size_t)M * S * 4);
+    item = ssh + align128((size_t)M * S * 4);
+    lg = item + align128((size_t)T * S * 16 * M * 4);
+    total = lg + align128((size_t)M * E * 4);
   }
 };
 
@@ -559,6 +578,117 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
   __syncthreads();
 }
 
+// ---------------------------------------------------------------------------- routing with the whole router
+// For a few tokens and a router that fits in shared memory, a CTA can compute
+// all logits by itself with four CTA barriers: (1) the |x| max of every
+// (token, slice), (2) x (* xscale) as FP16 scaled per (token, slice) as in
+// slice_input, and the gate/up operand xh (scaled per token) to global
+// memory, (3) warp w computes the items (tile j, slice c) = w, w + nwarps, ...
+// -- the slice's units in order, one accumulator -- unscaled into `item`, (4)
+// the logits, each the sum of its S items in slice order.  The router must be
+// in smem at w.rt and x at w.x (bulk copies issued by the caller, completing
+// on s.rbar and s.xbar).  Every CTA that runs it, and route_kernel for the
+// same call, gets the same bits.  Leaves the logits in s.lg (= smem + w.lg)
+// and the per-token shifts in s.shift; ends with a CTA barrier.
+TSM_DEV void route_whole(const RouteParams& p, RouteState& s, uint8_t* smem, const WholeSmem& ws, __half* xh,
+                         volatile int* dead, int warp, int lane, int tid, int nthr) {
+  const int M = p.M, H = p.H, S = p.S, CS = p.CS, C = p.rg.chunks, T = p.rg.tiles, E = p.E;
+  const bool split = p.xscale != nullptr;
+  const int ld = slice_ld(CS), halves = split ? 2 : 1, nwarps = nthr / 32;
+  const __nv_bfloat16* xr = reinterpret_cast<const __nv_bfloat16*>(smem + ws.x);
+  __half* xin = reinterpret_cast<__half*>(smem + ws.xin);
+  float* smx = reinterpret_cast<float*>(smem + ws.smx);
+  int* ssh = reinterpret_cast<int*>(smem + ws.ssh);
+  float* item = reinterpret_cast<float*>(smem + ws.item);
+  const uint8_t* rt = smem + ws.rt;
+  s.lg = reinterpret_cast<float*>(smem + ws.lg);
+  s.lgld = E;
+  mbar_wait(&s.xbar, 0, dead, p.err, ERR_TIMEOUT_XSTAGE);
+  mbar_wait(&s.rbar, 0, dead, p.err, ERR_TIMEOUT_XSTAGE);
+  // (1) slice maxima, one warp per (token, slice)
+  for (int q = warp; q < M * S; q += nwarps) {
+    const int t = q / S, c = q - t * S, lo = slice_lo(CS, c), n = (slice_hi(CS, C, c) - lo) * 32;
+    const __nv_bfloat16* row = xr + (size_t)t * H + lo * 32;
+    float m = 0.f;
+    for (int k = lane * 8; k < n; k += 256) m = absmax8(p, *reinterpret_cast<const uint4*>(row + k), lo * 32 + k, m);
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) {
+      smx[t * S + c] = m;
+      ssh[t * S + c] = shift_of_max(m);
+    }
+  }
+  __syncthreads();
+  if (tid < M) {
+    float m = 0.f;
+    for (int c = 0; c < S; ++c) m = fmaxf(m, smx[tid * S + c]);
+    s.shift[tid] = shift_of_max(m);
+  }
+  // (2) router input per (slice, token) and the gate/up operand xh
+  for (int i = tid; i < M * (H / 8); i += nthr) {
+    const int t = i / (H / 8), k = (i - t * (H / 8)) * 8, c = k / (CS * 32), kk = k - c * CS * 32;
+    const uint4 raw = *reinterpret_cast<const uint4*>(xr + (size_t)t * H + k);
+    uint4 hx, hh, hl;
+    convert8(p, raw, k, pow2f(ssh[t * S + c]), split, hx, hh, hl);
+    __half* dst = xin + ((size_t)c * halves * M + t) * ld + kk;
+    *reinterpret_cast<uint4*>(dst) = split ? hh : hx;
+    if (split) *reinterpret_cast<uint4*>(dst + (size_t)M * ld) = hl;
+  }
+  if (xh) {
+    __syncthreads();  // s.shift
+    for (int i = tid; i < M * (H / 8); i += nthr) {
+      const int t = i / (H / 8), k = (i - t * (H / 8)) * 8;
+      const uint4 raw = *reinterpret_cast<const uint4*>(xr + (size_t)t * H + k);
+      uint4 hx, hh, hl;
+      convert8(p, raw, k, pow2f(s.shift[t]), false, hx, hh, hl);
+      *reinterpret_cast<uint4*>(xh + (size_t)t * p.Hp + k) = hx;
+    }
+  }
+  __syncthreads();
+  // (3) items: warp w takes (tile j, slice c) pairs w, w + nwarps, ...; the
+  // slice's units in order into one accumulator, unscaled per token
+  for (int q = warp; q < T * S; q += nwarps) {
+    const int j = q / S, c = q - j * S, lo = slice_lo(CS, c), nck = slice_hi(CS, C, c) - lo;
+    const __half* xc = xin + (size_t)c * halves * M * ld;
+    float acc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int u = 0; u < nck; ++u) {
+      const uint8_t* un = rt + ((size_t)j * C + lo + u) * UNIT_BYTES;
+      const uint4 qw = *reinterpret_cast<const uint4*>(un + lane * 16);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(un + QUANT_BYTES + (lane >> 2) * 4);
+      for (int h = 0; h < halves; ++h) {
+        if (M > 8)
+          router_unit<2>(acc, qw, sc, xc + (size_t)h * M * ld + u * 32, ld, M, lane);
+        else
+          router_unit<1>(reinterpret_cast<float(&)[1][4]>(acc[0]), qw, sc, xc + (size_t)h * M * ld + u * 32, ld, M,
+                         lane);
+      }
+    }
+    const int gq = lane >> 2, cq = lane & 3;
+    float* it = item + (size_t)q * 16 * M;  // [row][token]
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = nt * 8 + 2 * cq + hh;
+        if (t < M) {
+          const float sc = pow2f(-ssh[t * S + c]);
+          it[gq * M + t] = acc[nt][hh] * sc;
+          it[(gq + 8) * M + t] = acc[nt][2 + hh] * sc;
+        }
+      }
+  }
+  __syncthreads();
+  // (4) logits: each the sum of its items in slice order
+  for (int i = tid; i < M * E; i += nthr) {
+    const int t = i / E, e = i - t * E, j = e >> 4, r = e & 15;
+    float v = 0.f;
+    for (int c = 0; c < S; ++c) v += item[((size_t)(j * S + c) * 16 + r) * M + t];
+    s.lg[i] = v;
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------------------- standalone route kernel
 constexpr int ROUTE_THREADS = ROUTE_WARPS * 32;
 
@@ -584,6 +714,38 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
   extern __shared__ __align__(128) uint8_t route_smem_raw[];
   RouteState& s = *reinterpret_cast<RouteState*>(route_smem_raw);
   uint8_t* sbuf = route_smem_raw + align128(sizeof(RouteState));
+  if (p.whole) {
+    // the whole-router algorithm, exactly as the layer kernel runs it
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const WholeSmem ws(p.M, p.H, p.rg.tiles, p.rg.chunks, p.S, p.CS, p.E, p.xscale != nullptr);
+    const RouteConst rc = route_const_load(p, tid);
+    if (tid == 0) {
+      mbar_init(&s.xbar, 1);
+      mbar_init(&s.rbar, 1);
+      fence_barrier_init();
+      s.xdead = 0;
+      const unsigned rbytes = (unsigned)p.rg.tiles * p.rg.chunks * UNIT_BYTES;
+      mbar_arrive_expect_tx(&s.rbar, rbytes);
+      bulk_g2s(sbuf + ws.rt, p.rw, rbytes, &s.rbar);
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    if (tid == 0) {
+      const unsigned xbytes = (unsigned)p.M * p.H * 2;
+      mbar_arrive_expect_tx(&s.xbar, xbytes);
+      bulk_g2s(sbuf + ws.x, p.x, xbytes, &s.xbar);
+    }
+    if (tid < p.E && !(isfinite(rc.b) && isfinite(rc.s))) atomicOr(p.err, ERR_BAD_ROUTER_INPUT);
+    route_init_smem(s, rc, tid);
+    __syncthreads();
+    route_whole(p, s, sbuf, ws, nullptr, &s.xdead, warp, lane, tid, ROUTE_THREADS);
+    if (tid < p.M && p.shift) p.shift[tid] = s.shift[tid];
+    route_topk(p, s, warp, lane, ROUTE_WARPS);
+    __syncthreads();
+    route_list(p, s, warp, lane, tid, ROUTE_THREADS);
+    if (p.sentinel) route_sentinel(p, tid);
+    return;
+  }
   const SliceSmem L(p.M, p.CS, p.xscale != nullptr);
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sbuf + L.xs);
   __half* xin = reinterpret_cast<__half*>(sbuf + L.xin);

@@ -172,6 +172,9 @@ ts_moe_status validate(const ts_moe_config* c, const ts_moe_layer_weights* L) {
 // Dynamic shared memory of route_kernel: RouteState, one item's slice buffers, the logits.
 constexpr int ROUTE_SMEM_MAX = 220 * 1024;
 size_t route_smem(const RouteParams& rp) {
+  if (rp.whole)
+    return align128(sizeof(RouteState)) +
+           WholeSmem(rp.M, rp.H, rp.rg.tiles, rp.rg.chunks, rp.S, rp.CS, rp.E, rp.xscale != nullptr).total;
   return align128(sizeof(RouteState)) + align128(SliceSmem(rp.M, rp.CS, rp.xscale != nullptr).total) +
          (size_t)rp.M * rp.E * 4;
 }
@@ -201,6 +204,24 @@ int choose_slices(int M, int C, int T, int E, int nb, bool split, int ntb, int m
     }
   }
   return best;
+}
+
+// Calls of at most WHOLE_MAX_M tokens whose router and routing buffers fit in
+// the rings route with the whole router in every CTA (route_whole): S and CS
+// give every warp of a CTA about one (tile, slice) item.  Both the handle path
+// and the allocation-free entry point decide here.
+#ifndef TSM_WHOLE_MAX_M
+#define TSM_WHOLE_MAX_M 1
+#endif
+constexpr int WHOLE_MAX_M = TSM_WHOLE_MAX_M;
+bool whole_slicing(int M, const MatGeom& gR, int E, int H, bool split, int& S, int& CS) {
+  if (M > WHOLE_MAX_M) return false;
+  const int C = gR.chunks, T = gR.tiles;
+  int s = std::max(1, std::min(C, (ROUTE_WARPS + T - 1) / T));
+  CS = (C + s - 1) / s;
+  S = (C + CS - 1) / CS;
+  const size_t need = WholeSmem(M, H, T, C, S, CS, E, split).total;
+  return need <= RING_BYTES && align128(sizeof(RouteState)) + need <= (size_t)ROUTE_SMEM_MAX;
 }
 
 // CTAs of one layer-kernel launch on a device with `sm_count` SMs: one per SM.
@@ -601,6 +622,8 @@ static RouteParams route_params(ts_moe* h, int layer, const void* x, int M, int 
   if (call_m > MAX_TOK) {
     rp.CS = (h->gR.chunks + h->s_chunk - 1) / h->s_chunk;
     rp.S = (h->gR.chunks + rp.CS - 1) / rp.CS;
+  } else if (whole_slicing(M, h->gR, rp.E, rp.H, h->any_xscale, rp.S, rp.CS)) {
+    rp.whole = 1;
   } else {
     router_slicing(M, h->gR, rp.E, h->nb, h->any_xscale, rp.S, rp.CS);  // fits: checked at open
   }
@@ -881,7 +904,9 @@ ts_moe_status ts_moe_route_noalloc(const void* router, const float* router_bias,
   int nsm = 0;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
-  if (!router_slicing(M, gR, E, layer_ctas(nsm), false, rp.S, rp.CS))
+  if (whole_slicing(M, gR, E, H, false, rp.S, rp.CS))
+    rp.whole = 1;
+  else if (!router_slicing(M, gR, E, layer_ctas(nsm), false, rp.S, rp.CS))
     return fail(nullptr, TS_MOE_EUNSUPPORTED, "no router slicing fits these sizes");
   e = launch_pdl(route_kernel, 1, ROUTE_THREADS, route_smem(rp), s, rp);
   if (e != cudaSuccess) return fail(nullptr, TS_MOE_ECUDA, std::string("route_kernel launch: ") + cudaGetErrorString(e));
