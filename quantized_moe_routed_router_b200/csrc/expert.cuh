@@ -94,6 +94,8 @@ struct __align__(128) LayerSmem {
   uint8_t x[NSX][XWIN];
   uint64_t wfull[NSW], wempty[NSW], xfull[NSX], xempty[NSX];
   RouteState r;
+  unsigned cp0[MAX_ENTRIES + 1];     // gate/up: cost of the entries before entry j (units x weight)
+  unsigned cq1[MAX_ENTRIES + 1];     // down: cost of the entries before entry j within one group
   unsigned rs0[MAX_NB + 1];          // gate/up: first unit of each CTA's range
   unsigned rs1[MAX_NB + 1];          // down: first unit of each CTA's range
   int dead;
@@ -121,13 +123,94 @@ TSM_DEV int cpre1(const LayerParams& p, int nT, int j) {
   return min(j, nT) * p.gC.chunks + (j > nT ? (j - nT) * p.gCs.chunks : 0);
 }
 
-// First unit of CTA b's range in phase PH (b = NB: the total), from the unit
-// counts alone: plain contiguous ranges, or for gate/up with few groups the
-// group-aligned partition (aligned_* in layout.cuh).
-template <int PH>
-TSM_DEV unsigned cta_start(const LayerParams& p, int nT, int nE, int NB, bool aligned, int G0, int b) {
-  if (PH == 1) return (unsigned)range_start((uint64_t)p.gC.ngroups * cpre1(p, nT, nE), NB, b);
-  if (!aligned || b >= NB) return (unsigned)range_start((uint64_t)upre0(p, nT, nE), NB, b);
+// Relative cost of a unit of an entry with nc columns: with more than 8
+// columns the consumers run two n8 MMA tiles per fragment, and the MXFP4 and
+// INT4-affine consumers, bound by their conversion issue, then take about
+// 1.4x the time per unit.  (Q8_0 stays within its memory time either way, so
+// its ranges stay equal in units.)
+TSM_DEV unsigned unit_weight(int nc) { return nc > 8 ? 7u : 5u; }
+
+// Warp 0: the cost prefixes of the entries (gate/up: units x weight, entry
+// major; down: chunks x weight within a group), so that CTA ranges are equal
+// in cost, not in units.  With equal weights the ranges are the same as by
+// units (floor(floor(b U w / NB) / w) = floor(b U / NB)).
+TSM_DEV void cost_tables(LayerSmem& s, const LayerParams& p, int lane) {
+  const int nE = s.r.nE, nT = s.r.nT;
+  const int per = (nE + 31) / 32, j0 = lane * per;
+  unsigned c0[MAX_ENTRIES / 32 + 1], c1[MAX_ENTRIES / 32 + 1], t0 = 0, t1 = 0;
+#pragma unroll
+  for (int i = 0; i < MAX_ENTRIES / 32 + 1; ++i) {
+    const int j = j0 + i;
+    c0[i] = c1[i] = 0u;
+    if (i < per && j < nE) {
+      const bool sh = j >= nT;
+      const unsigned w = unit_weight(s.r.nc[j]);
+      c0[i] = (unsigned)(sh ? p.gBs.ngroups * p.gBs.chunks : p.gB.ngroups * p.gB.chunks) * w;
+      c1[i] = (unsigned)(sh ? p.gCs.chunks : p.gC.chunks) * w;
+    }
+    t0 += c0[i];
+    t1 += c1[i];
+  }
+  unsigned i0 = t0, i1 = t1;
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned a = __shfl_up_sync(0xffffffffu, i0, o), b2 = __shfl_up_sync(0xffffffffu, i1, o);
+    if (lane >= o) {
+      i0 += a;
+      i1 += b2;
+    }
+  }
+  unsigned r0 = i0 - t0, r1 = i1 - t1;
+#pragma unroll
+  for (int i = 0; i < MAX_ENTRIES / 32 + 1; ++i) {
+    const int j = j0 + i;
+    if (i < per && j <= nE) {
+      s.cp0[j] = r0;
+      s.cq1[j] = r1;
+    }
+    r0 += c0[i];
+    r1 += c1[i];
+  }
+  if (lane == 31) {  // totals (the last lane's inclusive sums)
+    s.cp0[nE] = i0;
+    s.cq1[nE] = i1;
+  }
+}
+
+// Largest j in [0, n] with tab[j] <= c (tab non-decreasing, tab[0] = 0 <= c).
+TSM_DEV int last_le(const unsigned* tab, int n, unsigned c) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab[mid] <= c)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+// First unit of CTA b's range in phase PH (b = NB: the total): ranges equal
+// in units, or with COST equal in cost (cost_tables), or for gate/up with few
+// groups the group-aligned partition (aligned_* in layout.cuh).
+template <int PH, bool COST>
+TSM_DEV unsigned cta_start(const LayerSmem& s, const LayerParams& p, int nT, int nE, int NB, bool aligned, int G0,
+                           int b) {
+  if (PH == 1 && !COST) return (unsigned)range_start((uint64_t)p.gC.ngroups * cpre1(p, nT, nE), NB, b);
+  if (PH == 0 && !COST && (!aligned || b >= NB)) return (unsigned)range_start((uint64_t)upre0(p, nT, nE), NB, b);
+  if (PH == 1) {
+    const unsigned upg = (unsigned)cpre1(p, nT, nE), W1 = s.cq1[nE];
+    if (b >= NB) return (unsigned)p.gC.ngroups * upg;
+    const unsigned c = (unsigned)range_start((uint64_t)p.gC.ngroups * W1, NB, b);
+    const unsigned grp = c / W1, r = c - grp * W1;
+    const int j = min(last_le(s.cq1, nE, r), nE - 1);
+    return grp * upg + (unsigned)cpre1(p, nT, j) + (r - s.cq1[j]) / unit_weight(s.r.nc[j]);
+  }
+  if (b >= NB) return (unsigned)upre0(p, nT, nE);
+  if (!aligned) {
+    const unsigned c = (unsigned)range_start((uint64_t)s.cp0[nE], NB, b);
+    const int j = min(last_le(s.cp0, nE, c), nE - 1);
+    return (unsigned)upre0(p, nT, j) + (c - s.cp0[j]) / unit_weight(s.r.nc[j]);
+  }
   const int g = aligned_group_of(b, G0, NB);
   const bool shg = g >= nT * p.gB.ngroups;
   const int gs_ = g - nT * p.gB.ngroups;
@@ -403,21 +486,23 @@ TSM_DEV bool combine_prepare(LayerSmem& s, const LayerParams& p, int NB, int cti
   return use_tab;
 }
 
-// After the grid barrier: y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared)
-// in slot order over this CTA's slice; resid += y.  Two passes, so that the
-// loads of many (output, slot) pairs are in flight together: (1) each pair's
-// down value -- the K slots, then the shared expert -- into the idle weight
-// ring, CB pairs per thread with all of their loads issued before any is
-// used; (2) each output sums its values in slot order.  The barrier orders the
-// owner table written by combine_prepare before its reads here.
 // floor(a / b) for 0 <= a < 2^21 and b >= 1 by a float reciprocal rb = 1 / b:
 // the product's relative error is below 2^-23, so its absolute error is below
 // 2^-23 (a + 0.5) / b < 0.25 / b, while (a + 0.5) / b lies at least 0.5 / b
 // from every integer; the truncation is exact.
 TSM_DEV int fdiv(int a, float rb) { return (int)(((float)a + 0.5f) * rb); }
 
+// After the grid barrier: y[t][h] = sum_k w[t][k] * down_k[t][h] (+ shared)
+// in slot order over this CTA's slice; resid += y.  Two passes, so that the
+// loads of many (output, slot) pairs are in flight together: (1) each pair's
+// down value -- the K slots, then the shared expert -- into the idle weight
+// ring, CB pairs per thread with all of their loads issued before any is
+// used; (2) each output sums its values in slot order.  The barrier orders the
+// owner table written by combine_prepare before its reads here.  CB = 2 for
+// a decode launch, where a thread has at most a few pairs; 3 for more tokens.
+template <int CB>
 TSM_DEV void final_combine(LayerSmem& s, const LayerParams& p, int NB, int ctid, bool use_tab, float r0) {
-  constexpr int CT = NWC * 32, CB = 3;
+  constexpr int CT = NWC * 32;
   const int K = p.rp.K, H = p.rp.H, gs = p.gC.gs, MK = p.rp.M * K, nE = s.r.nE;
   const unsigned* tab = reinterpret_cast<const unsigned*>(&s.r.part[0][0][0]);
   int lo, hi;
@@ -792,7 +877,9 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
   return alive;
 }
 
-template <int FMT>
+// BIG: a launch of more than 16 tokens (several routing blocks, experts cut
+// into entries of 16 routes); the other instance is the decode launch.
+template <int FMT, bool BIG>
 __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   LayerSmem& s = *reinterpret_cast<LayerSmem*>(smem_raw);
@@ -816,7 +903,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.routes = nullptr;
     rp.rpos = nullptr;
   }
-  const int M = rp.M, NTB = (M + MAX_TOK - 1) / MAX_TOK;
+  const int M = rp.M, NTB = BIG ? (M + MAX_TOK - 1) / MAX_TOK : 1;
   const int S = rp.S, TS = rp.rg.tiles * S, nR = rp.whole ? 0 : TS * NTB;
   const bool rcta = b < nR;
   const int rtb = rcta ? b / TS : 0, rrem = rcta ? b % TS : 0;
@@ -951,11 +1038,18 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     xwriter = rcta && rj == 0;
     if (xwriter) slice_xh(bp, s.r, rcs, xs, xh_src, t0, tid, NTHREADS);
   }
-  route_topk(rp, s.r, warp, lane, NTHREADS / 32);
+  route_topk<BIG>(rp, s.r, warp, lane, NTHREADS / 32);
   __syncthreads();
   if (xwriter && tid == 0) red_release_add_u32(p.xh_cnt, 1u);  // after the barrier: the CTA's slice of xh
-  route_list(rp, s.r, warp, lane, tid, NTHREADS);
+  route_list<BIG>(rp, s.r, warp, lane, tid, NTHREADS);
   fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
+  // Cost-weighted ranges where units differ in cost: a launch of more than
+  // 16 tokens cuts experts into entries of up to 16 columns.
+  constexpr bool COST = BIG && FMT != FMT_Q8_0;
+  if (COST) {
+    if (warp == 0) cost_tables(s, p, lane);
+    __syncthreads();
+  }
 
   // ---- this CTA's ranges of both phases, in closed form, so the producer
   // starts at once; the consumer warps tabulate every CTA's range starts (for
@@ -964,8 +1058,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
   const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
-  const long long a0 = cta_start<0>(p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0>(p, nT, nE, NB, aligned, G0, b + 1);
-  const long long d0 = cta_start<1>(p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1>(p, nT, nE, NB, aligned, G0, b + 1);
+  const long long a0 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
+  const long long d0 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
@@ -998,8 +1092,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
 
   // ------------------------------------------------------------ consumer warps
   for (int i = tid; i <= NB; i += NWC * 32) {
-    s.rs0[i] = cta_start<0>(p, nT, nE, NB, aligned, G0, i);
-    s.rs1[i] = cta_start<1>(p, nT, nE, NB, aligned, G0, i);
+    s.rs0[i] = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, i);
+    s.rs1[i] = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, i);
   }
   bar_sync(1, NWC * 32);
   int wi = 0, wph = 0, xi = 0, xph = 0;
@@ -1028,7 +1122,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   float r0;
   const bool use_tab = combine_prepare(s, p, NB, tid, r0);
   grid_barrier(s, p, NB, tid);
-  final_combine(s, p, NB, tid, use_tab, r0);
+  final_combine<BIG ? 3 : 2>(s, p, NB, tid, use_tab, r0);
   if (b == 0) {  // every readiness wait of this launch is over
     for (int j = tid; j < nE; j += NWC * 32) p.entry_done[j] = 0u;
     if (tid == 0) {

@@ -380,17 +380,18 @@ TSM_DEV unsigned order_key(float f) {
 }
 TSM_DEV float key_value(unsigned k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k); }
 
-// Top-k and weights: warp w handles tokens w, w + nwarps, ... (lane holds
+// Top-k and weights: warp w handles tokens w, w + nwarps, ... (MULTI; else
+// the launch has at most 16 tokens and warp w handles token w; lane holds
 // experts lane, lane + 32, ...; PER = ceil(E / 32)).  The selection order is
 // (selection logit desc, expert index asc): each step takes the largest key
 // over the warp, then the smallest index holding it.  Each selected (token,
 // expert) also sets the token's bit in the expert's token mask.
-template <int PER>
+template <int PER, bool MULTI>
 TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lane, int nwarps) {
   const bool biased = p.bias && p.bias_mode != 0;
   const bool score_biased = p.bias && p.bias_mode == 1;
   const bool sig = p.score == 2;  // sigmoid scores; the bias is a selection-only correction
-  for (int t = warp; t < p.M; t += nwarps) {
+  for (int t = warp; t < p.M; t += MULTI ? nwarps : p.M) {
     const float* lgt = s.lg + (size_t)t * s.lgld;
     unsigned key[PER];
     float vsc[PER];
@@ -472,15 +473,16 @@ TSM_DEV void route_topk_t(const RouteParams& p, RouteState& s, int warp, int lan
   }
 }
 
+template <bool MULTI>
 TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane, int nwarps) {
   if (p.E <= 32)
-    route_topk_t<1>(p, s, warp, lane, nwarps);
+    route_topk_t<1, MULTI>(p, s, warp, lane, nwarps);
   else if (p.E <= 64)
-    route_topk_t<2>(p, s, warp, lane, nwarps);
+    route_topk_t<2, MULTI>(p, s, warp, lane, nwarps);
   else if (p.E <= 128)
-    route_topk_t<4>(p, s, warp, lane, nwarps);
+    route_topk_t<4, MULTI>(p, s, warp, lane, nwarps);
   else
-    route_topk_t<8>(p, s, warp, lane, nwarps);
+    route_topk_t<8, MULTI>(p, s, warp, lane, nwarps);
 }
 
 // Route list: the (token, slot) pairs grouped by expert (touched experts in
@@ -489,9 +491,11 @@ TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane,
 // selects an expert at most once, so the expert's route count is the
 // popcount of its token mask (set by route_topk) and a token's rank among
 // them the popcount of the mask's lower bits.  A shared entry's routes are
-// M K + its tokens, so every entry's route r of column n is ro + n.  Needs
-// s.tmask cleared (route_init_smem) and a CTA barrier after route_topk; ends
-// with one.
+// M K + its tokens, so every entry's route r of column n is ro + n.  Without
+// MULTI the launch has at most 16 tokens: one entry per touched expert.
+// Needs s.tmask cleared (route_init_smem) and a CTA barrier after
+// route_topk; ends with one.
+template <bool MULTI>
 TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
   const int MK = p.M * p.K;
   if (warp == 0) {
@@ -502,7 +506,7 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
       const int e = lane * PER + i;
       cl[i] = e < p.E ? __popcll(s.tmask[e]) : 0;
       tot += cl[i];
-      ne += (cl[i] + MAX_TOK - 1) / MAX_TOK;
+      ne += MULTI ? (cl[i] + MAX_TOK - 1) / MAX_TOK : (cl[i] > 0);
     }
     int incl = tot, neincl = ne;
     for (int o = 1; o < 32; o <<= 1) {
@@ -528,12 +532,16 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
             p.meta[META_RO + slot] = run + q;
             p.meta[META_NC + slot] = min(MAX_TOK, cl[i] - q);
           }
+          if (!MULTI) {
+            ++slot;
+            break;
+          }
         }
         run += cl[i];
       }
     }
     const int nT = __shfl_sync(0xffffffffu, neincl, 31);
-    const int nsh = p.has_shared ? (p.M + MAX_TOK - 1) / MAX_TOK : 0;
+    const int nsh = p.has_shared ? (MULTI ? (p.M + MAX_TOK - 1) / MAX_TOK : 1) : 0;
     if (lane < nsh) {
       const int j = nT + lane, n = min(MAX_TOK, p.M - MAX_TOK * lane);
       s.ex[j] = p.E;
@@ -564,7 +572,7 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
     const int pos = s.off[e] + rank;
     s.tok[pos] = tk;
     s.rpos[i] = pos;
-    s.rj[pos] = s.eslot[e] + rank / MAX_TOK;
+    s.rj[pos] = s.eslot[e] + (MULTI ? rank / MAX_TOK : 0);
     if (p.routes) {
       Route r;
       r.token = tk;
@@ -740,9 +748,9 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
     __syncthreads();
     route_whole(p, s, sbuf, ws, nullptr, &s.xdead, warp, lane, tid, ROUTE_THREADS);
     if (tid < p.M && p.shift) p.shift[tid] = s.shift[tid];
-    route_topk(p, s, warp, lane, ROUTE_WARPS);
+    route_topk<false>(p, s, warp, lane, ROUTE_WARPS);
     __syncthreads();
-    route_list(p, s, warp, lane, tid, ROUTE_THREADS);
+    route_list<false>(p, s, warp, lane, tid, ROUTE_THREADS);
     if (p.sentinel) route_sentinel(p, tid);
     return;
   }
@@ -789,9 +797,9 @@ __global__ void __launch_bounds__(ROUTE_THREADS, 1) route_kernel(const RoutePara
     if (p.shift) p.shift[tid] = s.shift[tid];
   }
   __syncthreads();
-  route_topk(p, s, warp, lane, ROUTE_WARPS);
+  route_topk<false>(p, s, warp, lane, ROUTE_WARPS);
   __syncthreads();
-  route_list(p, s, warp, lane, tid, ROUTE_THREADS);
+  route_list<false>(p, s, warp, lane, tid, ROUTE_THREADS);
   if (p.sentinel) route_sentinel(p, tid);
 }
 

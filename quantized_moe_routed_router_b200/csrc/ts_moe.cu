@@ -262,9 +262,12 @@ cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cud
 
 ts_moe_status set_smem_attrs(ts_moe* h) {
   const int bytes = (int)sizeof(LayerSmem);
-  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX));
   return TS_MOE_OK;
 }
@@ -474,10 +477,10 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     // every CTA of a layer launch must be resident at once (grid barrier)
     int per_sm = 0;
     ce = fmt == TS_FMT_MXFP4
-             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<1>, NTHREADS, sizeof(LayerSmem))
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<1, false>, NTHREADS, sizeof(LayerSmem))
          : fmt == TS_FMT_INT4_AFFINE
-             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<2>, NTHREADS, sizeof(LayerSmem))
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<0>, NTHREADS, sizeof(LayerSmem));
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<2, false>, NTHREADS, sizeof(LayerSmem))
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layer_kernel<0, false>, NTHREADS, sizeof(LayerSmem));
     if (ce != cudaSuccess) {
       g_open_error = std::string("occupancy query: ") + cudaGetErrorString(ce);
       return cleanup(TS_MOE_ECUDA);
@@ -727,12 +730,13 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
     lp.y = y ? y + (size_t)m0 * H : nullptr;
     lp.resid = resid ? (__nv_bfloat16*)resid + (size_t)m0 * H : nullptr;
     cudaError_t e;
+    const bool big = lp.rp.M > MAX_TOK;  // a prefill launch: several routing blocks
     if (c.expert_fmt == TS_FMT_MXFP4)
-      e = launch_pdl(layer_kernel<1>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(big ? layer_kernel<1, true> : layer_kernel<1, false>, h->nb, NTHREADS, smem, st, lp);
     else if (c.expert_fmt == TS_FMT_INT4_AFFINE)
-      e = launch_pdl(layer_kernel<2>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(big ? layer_kernel<2, true> : layer_kernel<2, false>, h->nb, NTHREADS, smem, st, lp);
     else
-      e = launch_pdl(layer_kernel<0>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(big ? layer_kernel<0, true> : layer_kernel<0, false>, h->nb, NTHREADS, smem, st, lp);
     if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
   }
   if (h->timing) cudaEventRecord(h->ev[1], st);
