@@ -463,10 +463,11 @@ TSM_DEV float down_sum(const LayerSmem& s, const LayerParams& p, const DownSrc& 
 }
 
 // This CTA's 1/NB slice [lo, hi) of the M x H outputs.
+// (32-bit: M H <= 64 x 16384 = 2^20 and NB <= 512.)
 TSM_DEV void combine_range(const LayerParams& p, int NB, int& lo, int& hi) {
-  const long long MH = (long long)p.rp.M * p.rp.H;
-  lo = (int)(MH * blockIdx.x / NB);
-  hi = (int)(MH * (blockIdx.x + 1) / NB);
+  const unsigned MH = (unsigned)p.rp.M * (unsigned)p.rp.H, nb = (unsigned)NB, b = blockIdx.x;
+  lo = (int)(MH * b / nb);
+  hi = (int)(MH * (b + 1) / nb);
 }
 
 // Before the grid barrier (nothing here depends on other CTAs' down work):
@@ -1051,18 +1052,24 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     __syncthreads();
   }
 
-  // ---- this CTA's ranges of both phases, in closed form, so the producer
-  // starts at once; the consumer warps tabulate every CTA's range starts (for
-  // the owners of split groups and the combine) while the first stages load
+  // ---- this CTA's ranges of both phases, in closed form: the producer's four
+  // bounds one per lane, so that it starts at once; the consumer warps
+  // tabulate every CTA's range starts (for the owners of split groups and the
+  // combine) while the first stages load
   const int nE = s.r.nE, nT = s.r.nT;
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
   const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
-  const long long a0 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
-  const long long d0 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
+    unsigned bound = 0;
+    if (lane < 2)
+      bound = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + lane);
+    else if (lane < 4)
+      bound = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + lane - 2);
+    const long long a0 = __shfl_sync(0xffffffffu, bound, 0), a1 = __shfl_sync(0xffffffffu, bound, 1);
+    const long long d0 = __shfl_sync(0xffffffffu, bound, 2), d1 = __shfl_sync(0xffffffffu, bound, 3);
     const uint64_t pol = policy_evict_first();
     int wi = 0, wph = 0, xi = 0, xph = 0;
     int wuse[NSW], xuse[NSX];
@@ -1091,10 +1098,14 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   }
 
   // ------------------------------------------------------------ consumer warps
-  for (int i = tid; i <= NB; i += NWC * 32) {
-    s.rs0[i] = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, i);
-    s.rs1[i] = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, i);
+  for (int i = tid; i < 2 * (NB + 1); i += NWC * 32) {
+    if (i <= NB)
+      s.rs0[i] = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, i);
+    else
+      s.rs1[i - NB - 1] = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, i - NB - 1);
   }
+  const long long a0 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
+  const long long d0 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
   bar_sync(1, NWC * 32);
   int wi = 0, wph = 0, xi = 0, xph = 0;
   {

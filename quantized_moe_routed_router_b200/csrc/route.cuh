@@ -493,13 +493,13 @@ TSM_DEV void route_topk(const RouteParams& p, RouteState& s, int warp, int lane,
 // them the popcount of the mask's lower bits.  A shared entry's routes are
 // M K + its tokens, so every entry's route r of column n is ro + n.  Without
 // MULTI the launch has at most 16 tokens: one entry per touched expert.
-// Needs s.tmask cleared (route_init_smem) and a CTA barrier after
-// route_topk; ends with one.
-template <bool MULTI>
-TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
+// Warp 0 counts the routes, lane l holding experts l PER .. l PER + PER - 1
+// (PER: the power of two at or above E / 32).  Needs s.tmask cleared
+// (route_init_smem) and a CTA barrier after route_topk; ends with one.
+template <int PER, bool MULTI>
+TSM_DEV void route_list_t(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
   const int MK = p.M * p.K;
   if (warp == 0) {
-    constexpr int PER = MAX_E / 32;
     int cl[PER], tot = 0, ne = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
@@ -584,6 +584,18 @@ TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane,
     if (p.rpos) p.rpos[i] = pos;
   }
   __syncthreads();
+}
+
+template <bool MULTI>
+TSM_DEV void route_list(const RouteParams& p, RouteState& s, int warp, int lane, int tid, int nthr) {
+  if (p.E <= 32)
+    route_list_t<1, MULTI>(p, s, warp, lane, tid, nthr);
+  else if (p.E <= 64)
+    route_list_t<2, MULTI>(p, s, warp, lane, tid, nthr);
+  else if (p.E <= 128)
+    route_list_t<4, MULTI>(p, s, warp, lane, tid, nthr);
+  else
+    route_list_t<8, MULTI>(p, s, warp, lane, tid, nthr);
 }
 
 // ---------------------------------------------------------------------------- routing with the whole router
