@@ -331,7 +331,9 @@ def run_ours(args, rank, world, local):
     avg_ms = ms_step / launches_per_step
     bytes_per_launch = algo_bytes / launches_per_step
     achieved = bytes_per_launch / (avg_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": f"layer_kernel<{'MXFP4' if shape.expert_fmt else 'Q8_0'}> (route + gate/up + down + combine)",
+    fmt_name = {synth.FMT_Q8_0: "Q8_0", synth.FMT_MXFP4: "MXFP4", synth.FMT_INT4_AFFINE: "INT4-affine"}[shape.expert_fmt]
+    instance = "prefill" if M > 16 else "decode"
+    roofline = {"bound": "hbm", "kernel": f"layer_kernel<{fmt_name}, {instance}> (route + gate/up + down + combine)",
                 "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} HBM copy bandwidth",
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(bytes_per_launch),
                 "avg_launch_us": round(avg_ms * 1e3, 2), "algorithmic_bytes_per_launch": int(bytes_per_launch),
