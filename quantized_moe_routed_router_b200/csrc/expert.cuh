@@ -82,12 +82,22 @@ struct LayerParams {
   unsigned* entry_done;     // [MAX_ENTRIES] gate/up (group, consumer warp) shares finished per entry
   unsigned long long* grid_cnt;  // grid barrier arrivals, never reset: NB per launch (64-bit: never wraps)
   int debug_skip_arrival;   // test hook: CTA 0 does not arrive, so the barrier's bounded wait runs out
+  // one-token launches routed with the whole router: the range tables (gate/up
+  // then down, part_stride(NB) entries each) for part_nT routed entries,
+  // computed at open (a token selects K distinct experts); null otherwise
+  const unsigned* part_tab;
+  int part_nT;
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
   unsigned* err;
   int act;
   float alpha, limit;
 };
+
+// Range tables of NB + 1 entries, padded to whole 16-byte rows (a table of
+// part_stride entries is one bulk copy).
+constexpr int RS_LEN = (MAX_NB + 1 + 3) / 4 * 4;
+TSM_HD int part_stride(int NB) { return (NB + 1 + 3) / 4 * 4; }
 
 struct __align__(128) LayerSmem {
   uint8_t w[NSW][WSTAGE];
@@ -96,8 +106,8 @@ struct __align__(128) LayerSmem {
   RouteState r;
   unsigned cp0[MAX_ENTRIES + 1];     // gate/up: cost of the entries before entry j (units x weight)
   unsigned cq1[MAX_ENTRIES + 1];     // down: cost of the entries before entry j within one group
-  unsigned rs0[MAX_NB + 1];          // gate/up: first unit of each CTA's range
-  unsigned rs1[MAX_NB + 1];          // down: first unit of each CTA's range
+  __align__(16) unsigned rs0[RS_LEN];  // gate/up: first unit of each CTA's range
+  __align__(16) unsigned rs1[RS_LEN];  // down: first unit of each CTA's range
   int dead;
   unsigned long long gen0;  // launches completed before this one
 };
@@ -193,11 +203,12 @@ TSM_DEV int last_le(const unsigned* tab, int n, unsigned c) {
 // in units, or with COST equal in cost (cost_tables), or for gate/up with few
 // groups the group-aligned partition (aligned_* in layout.cuh).
 template <int PH, bool COST>
-TSM_DEV unsigned cta_start(const LayerSmem& s, const LayerParams& p, int nT, int nE, int NB, bool aligned, int G0,
+TSM_DEV unsigned cta_start(const LayerSmem* sp, const LayerParams& p, int nT, int nE, int NB, bool aligned, int G0,
                            int b) {
   if (PH == 1 && !COST) return (unsigned)range_start((uint64_t)p.gC.ngroups * cpre1(p, nT, nE), NB, b);
   if (PH == 0 && !COST && (!aligned || b >= NB)) return (unsigned)range_start((uint64_t)upre0(p, nT, nE), NB, b);
-  if (PH == 1) {
+  if (PH == 1) {  // (COST only from here on: the cost tables in *sp)
+    const LayerSmem& s = *sp;
     const unsigned upg = (unsigned)cpre1(p, nT, nE), W1 = s.cq1[nE];
     if (b >= NB) return (unsigned)p.gC.ngroups * upg;
     const unsigned c = (unsigned)range_start((uint64_t)p.gC.ngroups * W1, NB, b);
@@ -207,6 +218,7 @@ TSM_DEV unsigned cta_start(const LayerSmem& s, const LayerParams& p, int nT, int
   }
   if (b >= NB) return (unsigned)upre0(p, nT, nE);
   if (!aligned) {
+    const LayerSmem& s = *sp;
     const unsigned c = (unsigned)range_start((uint64_t)s.cp0[nE], NB, b);
     const int j = min(last_le(s.cp0, nE, c), nE - 1);
     return (unsigned)upre0(p, nT, j) + (c - s.cp0[j]) / unit_weight(s.r.nc[j]);
@@ -218,6 +230,18 @@ TSM_DEV unsigned cta_start(const LayerSmem& s, const LayerParams& p, int nT, int
   const int grp = shg ? gs_ % p.gBs.ngroups : g % p.gB.ngroups;
   const int ch = shg ? p.gBs.chunks : p.gB.chunks;
   return (unsigned)(upre0(p, nT, j) + (long long)grp * ch + aligned_offset(b, G0, NB, ch));
+}
+
+// The unit-equal range tables of a launch with nT routed and nE entries in
+// all: out[b] = gate/up start of CTA b, out[stride + b] = down start (b <= NB).
+// Computed once at open for one-token launches (nT = K), with cta_start.
+__global__ void partition_table_kernel(const LayerParams p, int nT, int nE, int NB, int stride, unsigned* out) {
+  const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
+  const bool aligned = use_aligned(G0, NB);
+  for (int i = threadIdx.x; i <= NB; i += blockDim.x) {
+    out[i] = cta_start<0, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
+    out[stride + i] = cta_start<1, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
+  }
 }
 
 // Next segment (one entry's group, a run of its chunks) of [u, u1) of phase PH
@@ -774,7 +798,7 @@ TSM_DEV void consume_seg(LayerSmem& s, const LayerParams& p, const Seg& sg, int&
 // x is soon ready), then waits (bounded) for the data to be published.
 template <int FMT, int PH>
 TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, long long u1, int& wi, int& wph, int& xi,
-                           int& xph, int* wuse, int* xuse, uint64_t pol, int lane, const __half* xh_src,
+                           int& xph, int& wcount, int& xcount, uint64_t pol, int lane, const __half* xh_src,
                            bool xh_wait) {
   constexpr int KC = FMT == FMT_MXFP4 ? 64 : 32;
   constexpr int KWC = KW / KC;
@@ -812,7 +836,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
             }
           }
           alive = __shfl_sync(0xffffffffu, alive, 0);
-          ++wuse[wi];
+          ++wcount;
           if (++wi == NSW) {
             wi = 0;
             wph ^= 1;
@@ -849,7 +873,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
       alive = __shfl_sync(0xffffffffu, alive, 0);
       if (!alive) break;
       if (lane < sg.nc) bulk_g2s(s.x[xi] + lane * XROW, brow + (size_t)ws * KC, xbytes, &s.xfull[xi]);
-      ++xuse[xi];
+      ++xcount;
       if (++xi == NSX) {
         xi = 0;
         xph ^= 1;
@@ -865,7 +889,7 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
         }
         alive = __shfl_sync(0xffffffffu, alive, 0);
         if (!alive) break;
-        ++wuse[wi];
+        ++wcount;
         if (++wi == NSW) {
           wi = 0;
           wph ^= 1;
@@ -938,8 +962,13 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     s.dead = 0;
     if (rp.whole) {  // the router is a weight: fetched before the dependency wait
       const unsigned rbytes = (unsigned)rp.rg.tiles * rp.rg.chunks * UNIT_BYTES;
-      mbar_arrive_expect_tx(&s.r.rbar, rbytes);
+      const unsigned tbytes = p.part_tab ? (unsigned)part_stride(NB) * 4u : 0u;  // and the range tables
+      mbar_arrive_expect_tx(&s.r.rbar, rbytes + 2 * tbytes);
       bulk_g2s(ring + WS.rt, rp.rw, rbytes, &s.r.rbar);
+      if (p.part_tab) {
+        bulk_g2s(s.rs0, p.part_tab, tbytes, &s.r.rbar);
+        bulk_g2s(s.rs1, p.part_tab + part_stride(NB), tbytes, &s.r.rbar);
+      }
     } else if (rcta) {
       slice_issue_router(bp, s.r, rj, rcs, rt);
     }
@@ -1060,56 +1089,64 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
   const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
+  // one-token launches: the tables loaded with the router hold every range
+  // (unless NaN logits made the token select fewer than K experts)
+  const bool tab = p.part_tab && rp.whole && nT == p.part_nT;
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
     unsigned bound = 0;
-    if (lane < 2)
-      bound = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + lane);
+    if (tab)
+      bound = lane < 2 ? s.rs0[b + lane] : s.rs1[b + (lane & 1)];
+    else if (lane < 2)
+      bound = cta_start<0, COST>(&s, p, nT, nE, NB, aligned, G0, b + lane);
     else if (lane < 4)
-      bound = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + lane - 2);
+      bound = cta_start<1, COST>(&s, p, nT, nE, NB, aligned, G0, b + lane - 2);
     const long long a0 = __shfl_sync(0xffffffffu, bound, 0), a1 = __shfl_sync(0xffffffffu, bound, 1);
     const long long d0 = __shfl_sync(0xffffffffu, bound, 2), d1 = __shfl_sync(0xffffffffu, bound, 3);
     const uint64_t pol = policy_evict_first();
     int wi = 0, wph = 0, xi = 0, xph = 0;
-    int wuse[NSW], xuse[NSX];
-    for (int i = 0; i < NSW; ++i) wuse[i] = 0;
-    for (int i = 0; i < NSX; ++i) xuse[i] = 0;
+    int wcount = 0, xcount = 0;  // copies issued into the weight / window rings (round robin)
     // gate/up reads x written by the routing CTAs: wait for all their slices;
     // routed with the whole router, this CTA wrote all of x itself, before the
     // barriers above (its generic writes, read by the window bulk copies)
     if (rp.whole) fence_proxy_async_global();
-    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, !rp.whole);
-    if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wuse, xuse, pol, lane, xh_src, false);
+    bool alive = produce_phase<FMT, 0>(s, p, a0, a1, wi, wph, xi, xph, wcount, xcount, pol, lane, xh_src, !rp.whole);
+    if (alive) produce_phase<FMT, 1>(s, p, d0, d1, wi, wph, xi, xph, wcount, xcount, pol, lane, xh_src, false);
     // Copies still in flight must land before the CTA can exit (only matters
     // when a wait gave up): wait, bounded, for each slot's last issued phase.
     if (lane == 0 && s.dead) {
       const unsigned long long t0 = globaltimer();
-      for (int i = 0; i < NSW; ++i)
-        if (wuse[i])
-          while (!mbar_try_wait(&s.wfull[i], (wuse[i] - 1) & 1) && globaltimer() - t0 < WAIT_LIMIT_NS) {
+      // slot i of a ring of n was used count / n + (i < count % n) times
+      for (int i = 0; i < NSW; ++i) {
+        const int uses = wcount / NSW + (i < wcount % NSW ? 1 : 0);
+        if (uses)
+          while (!mbar_try_wait(&s.wfull[i], (uses - 1) & 1) && globaltimer() - t0 < WAIT_LIMIT_NS) {
           }
-      for (int i = 0; i < NSX; ++i)
-        if (xuse[i])
-          while (!mbar_try_wait(&s.xfull[i], (xuse[i] - 1) & 1) && globaltimer() - t0 < WAIT_LIMIT_NS) {
+      }
+      for (int i = 0; i < NSX; ++i) {
+        const int uses = xcount / NSX + (i < xcount % NSX ? 1 : 0);
+        if (uses)
+          while (!mbar_try_wait(&s.xfull[i], (uses - 1) & 1) && globaltimer() - t0 < WAIT_LIMIT_NS) {
           }
+      }
     }
     return;
   }
 
   // ------------------------------------------------------------ consumer warps
-  for (int i = tid; i < 2 * (NB + 1); i += NWC * 32) {
-    if (i <= NB)
-      s.rs0[i] = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, i);
-    else
-      s.rs1[i - NB - 1] = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, i - NB - 1);
-  }
-  const long long a0 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b), a1 = cta_start<0, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
-  const long long d0 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b), d1 = cta_start<1, COST>(s, p, nT, nE, NB, aligned, G0, b + 1);
+  if (!tab)
+    for (int i = tid; i < 2 * (NB + 1); i += NWC * 32) {
+      if (i <= NB)
+        s.rs0[i] = cta_start<0, COST>(&s, p, nT, nE, NB, aligned, G0, i);
+      else
+        s.rs1[i - NB - 1] = cta_start<1, COST>(&s, p, nT, nE, NB, aligned, G0, i - NB - 1);
+    }
   bar_sync(1, NWC * 32);
   int wi = 0, wph = 0, xi = 0, xph = 0;
   {
-    long long u = a0;
+    long long u = s.rs0[b];
+    const long long a1 = s.rs0[b + 1];
     int j = 0;
     Seg sg;
     while (next_seg<0>(s, p, u, a1, j, sg)) {
@@ -1120,7 +1157,8 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     }
   }
   {
-    long long u = d0;
+    long long u = s.rs1[b];
+    const long long d1 = s.rs1[b + 1];
     int j = 0;
     Seg sg;
     while (next_seg<1>(s, p, u, d1, j, sg)) {

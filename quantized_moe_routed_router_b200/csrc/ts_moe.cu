@@ -82,6 +82,8 @@ struct ts_moe {
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group, consumer warp) chunk counters
   unsigned long long* arrivals = nullptr;  // grid barrier arrivals (64-bit, never reset while the handle lives)
   unsigned* grid = nullptr;     // {x slices written, router items published}
+  unsigned* part_m1 = nullptr;  // range tables of one-token launches (K routed entries), computed at open
+  int part_m1_nT = 0;
   bool debug_skip_arrival = false;
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
@@ -429,6 +431,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
+    const size_t o_tab = slot((size_t)2 * part_stride(h->nb) * 4);
     const size_t o_cnt = off;
     const size_t n_cnt = 2 + (size_t)MAX_ENTRIES * h->ng_max_B * NWC + MAX_ENTRIES + 2 + 1;  // arrivals (u64) + ... + grid[2] + error word
     slot(n_cnt * 4);
@@ -454,6 +457,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->P = (float*)(h->ws + o_P);
     h->partial0 = (float*)(h->ws + o_part0);
     h->partial1 = (float*)(h->ws + o_part1);
+    h->part_m1 = (unsigned*)(h->ws + o_tab);
     unsigned* cn = (unsigned*)(h->ws + o_cnt);
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
@@ -472,6 +476,25 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
   if ((st = set_smem_attrs(h)) != TS_MOE_OK) {
     g_open_error = h->error;
     return cleanup(st);
+  }
+  {
+    // one token selects K distinct experts: the range tables of its launches
+    // are fixed by the geometry, so they are computed once here
+    LayerParams lp;
+    std::memset(&lp, 0, sizeof(lp));
+    lp.gB = h->gB;
+    lp.gBs = h->gBs;
+    lp.gC = h->gC;
+    lp.gCs = h->gCs;
+    lp.rp.has_shared = c.shared_inter > 0;
+    h->part_m1_nT = K;
+    partition_table_kernel<<<1, 256>>>(lp, K, K + (lp.rp.has_shared ? 1 : 0), h->nb, part_stride(h->nb), h->part_m1);
+    ce = cudaGetLastError();
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(nullptr);
+    if (ce != cudaSuccess) {
+      g_open_error = std::string("partition tables: ") + cudaGetErrorString(ce);
+      return cleanup(TS_MOE_ECUDA);
+    }
   }
   {
     // every CTA of a layer launch must be resident at once (grid barrier)
@@ -529,7 +552,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const uint8_t* r = src(w.router, router_b, 0);
     if (ce != cudaSuccess) break;
     launch_repack<1>(TS_FMT_Q8_0, r, nullptr, (int)blob_row_bytes(TS_FMT_Q8_0, H), H / 32, h->gR, d.rw, d_bad, st0, E);
-    if (ce == cudaSuccess) ce = cudaDeviceSynchronize();  // the staging buffer is reused next
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(nullptr);  // the staging buffer is reused next
     if (w.router_bias && ce == cudaSuccess) ce = cudaMemcpy(d.bias, w.router_bias, E * 4, cudaMemcpyHostToDevice);
     if (ce == cudaSuccess)
       ce = cudaMemcpy(d.pes, w.per_expert_scale ? w.per_expert_scale : ones.data(), E * 4, cudaMemcpyHostToDevice);
@@ -729,6 +752,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
     lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, h->lt), M);
     lp.y = y ? y + (size_t)m0 * H : nullptr;
     lp.resid = resid ? (__nv_bfloat16*)resid + (size_t)m0 * H : nullptr;
+    lp.part_tab = lp.rp.M == 1 && lp.rp.whole ? h->part_m1 : nullptr;  // whole-router one-token launches
+    lp.part_nT = h->part_m1_nT;
     cudaError_t e;
     const bool big = lp.rp.M > MAX_TOK;  // a prefill launch: several routing blocks
     if (c.expert_fmt == TS_FMT_MXFP4)
