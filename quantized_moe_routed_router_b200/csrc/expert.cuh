@@ -82,11 +82,12 @@ struct LayerParams {
   unsigned* entry_done;     // [MAX_ENTRIES] gate/up (group, consumer warp) shares finished per entry
   unsigned long long* grid_cnt;  // grid barrier arrivals, never reset: NB per launch (64-bit: never wraps)
   int debug_skip_arrival;   // test hook: CTA 0 does not arrive, so the barrier's bounded wait runs out
-  // one-token launches routed with the whole router: the range tables (gate/up
-  // then down, part_stride(NB) entries each) for part_nT routed entries,
-  // computed at open (a token selects K distinct experts); null otherwise
-  const unsigned* part_tab;
-  int part_nT;
+  // decode launches: the unit-equal range tables (gate/up then down,
+  // part_stride(NB) entries each) for every count nT = 1 .. part_nmax of
+  // routed entries, table nT - 1 at part_all + (nT - 1) 2 part_stride(NB),
+  // computed at open; null for prefill launches
+  const unsigned* part_all;
+  int part_nmax;
   float* y;                 // [M][H] or null
   __nv_bfloat16* resid;     // [M][H] in/out or null
   unsigned* err;
@@ -109,6 +110,8 @@ struct __align__(128) LayerSmem {
   __align__(16) unsigned rs0[RS_LEN];  // gate/up: first unit of each CTA's range
   __align__(16) unsigned rs1[RS_LEN];  // down: first unit of each CTA's range
   int dead;
+  int tab_nT;               // routed entries whose range tables were fetched after the top-k (0: none)
+  uint64_t tbar;            // completion of that fetch
   unsigned long long gen0;  // launches completed before this one
 };
 
@@ -232,15 +235,18 @@ TSM_DEV unsigned cta_start(const LayerSmem* sp, const LayerParams& p, int nT, in
   return (unsigned)(upre0(p, nT, j) + (long long)grp * ch + aligned_offset(b, G0, NB, ch));
 }
 
-// The unit-equal range tables of a launch with nT routed and nE entries in
-// all: out[b] = gate/up start of CTA b, out[stride + b] = down start (b <= NB).
-// Computed once at open for one-token launches (nT = K), with cta_start.
-__global__ void partition_table_kernel(const LayerParams p, int nT, int nE, int NB, int stride, unsigned* out) {
-  const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
+// The unit-equal range tables of decode launches, computed once at open with
+// cta_start: block t for nT = t + 1 routed entries (and nsh shared ones) writes
+// out[2 t stride + b] = gate/up start of CTA b, out[(2 t + 1) stride + b] =
+// down start (b <= NB).
+__global__ void partition_table_kernel(const LayerParams p, int nsh, int NB, int stride, unsigned* out) {
+  const int nT = blockIdx.x + 1, nE = nT + nsh;
+  const int G0 = nT * p.gB.ngroups + nsh * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
+  unsigned* o = out + (size_t)blockIdx.x * 2 * stride;
   for (int i = threadIdx.x; i <= NB; i += blockDim.x) {
-    out[i] = cta_start<0, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
-    out[stride + i] = cta_start<1, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
+    o[i] = cta_start<0, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
+    o[stride + i] = cta_start<1, false>(nullptr, p, nT, nE, NB, aligned, G0, i);
   }
 }
 
@@ -929,6 +935,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.rpos = nullptr;
   }
   const int M = rp.M, NTB = BIG ? (M + MAX_TOK - 1) / MAX_TOK : 1;
+  // A token selects K distinct experts: a one-token launch routed with the
+  // whole router fetches its range tables (nT = K) with the router.
+  const bool tab_pro = !BIG && p.part_all && rp.whole && M == 1;
   const int S = rp.S, TS = rp.rg.tiles * S, nR = rp.whole ? 0 : TS * NTB;
   const bool rcta = b < nR;
   const int rtb = rcta ? b / TS : 0, rrem = rcta ? b % TS : 0;
@@ -958,16 +967,19 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     mbar_init(&s.r.xbar, 1);
     mbar_init(&s.r.rbar, 1);
     mbar_init(&s.r.pbar, 1);
+    mbar_init(&s.tbar, 1);
     fence_barrier_init();
     s.dead = 0;
+    s.tab_nT = 0;
     if (rp.whole) {  // the router is a weight: fetched before the dependency wait
       const unsigned rbytes = (unsigned)rp.rg.tiles * rp.rg.chunks * UNIT_BYTES;
-      const unsigned tbytes = p.part_tab ? (unsigned)part_stride(NB) * 4u : 0u;  // and the range tables
+      const unsigned tbytes = tab_pro ? (unsigned)part_stride(NB) * 4u : 0u;  // and the one-token range tables
       mbar_arrive_expect_tx(&s.r.rbar, rbytes + 2 * tbytes);
       bulk_g2s(ring + WS.rt, rp.rw, rbytes, &s.r.rbar);
-      if (p.part_tab) {
-        bulk_g2s(s.rs0, p.part_tab, tbytes, &s.r.rbar);
-        bulk_g2s(s.rs1, p.part_tab + part_stride(NB), tbytes, &s.r.rbar);
+      if (tab_pro) {
+        const unsigned* t = p.part_all + (size_t)(rp.K - 1) * 2 * part_stride(NB);
+        bulk_g2s(s.rs0, t, tbytes, &s.r.rbar);
+        bulk_g2s(s.rs1, t + part_stride(NB), tbytes, &s.r.rbar);
       }
     } else if (rcta) {
       slice_issue_router(bp, s.r, rj, rcs, rt);
@@ -1071,6 +1083,22 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   route_topk<BIG>(rp, s.r, warp, lane, NTHREADS / 32);
   __syncthreads();
   if (xwriter && tid == 0) red_release_add_u32(p.xh_cnt, 1u);  // after the barrier: the CTA's slice of xh
+  if (!BIG && p.part_all && !tab_pro && warp == NWC) {
+    // other decode launches: the routed-entry count is known from the token
+    // masks now, so the producer fetches its tables while the list is built
+    const int nw = (rp.E + 31) / 32;
+    int cnt = 0;
+    for (int w = 0; w < nw; ++w)
+      cnt += __popc(__ballot_sync(0xffffffffu, lane + 32 * w < rp.E && s.r.tmask[lane + 32 * w] != 0ull));
+    if (lane == 0 && cnt >= 1 && cnt <= p.part_nmax) {
+      const unsigned tbytes = (unsigned)part_stride(NB) * 4u;
+      const unsigned* t = p.part_all + (size_t)(cnt - 1) * 2 * part_stride(NB);
+      s.tab_nT = cnt;  // published by the route list's first barrier
+      mbar_arrive_expect_tx(&s.tbar, 2 * tbytes);
+      bulk_g2s(s.rs0, t, tbytes, &s.tbar);
+      bulk_g2s(s.rs1, t + part_stride(NB), tbytes, &s.tbar);
+    }
+  }
   route_list<BIG>(rp, s.r, warp, lane, tid, NTHREADS);
   fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
   // Cost-weighted ranges where units differ in cost: a launch of more than
@@ -1089,13 +1117,16 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   // gate/up: with few groups, each CTA stays inside one group (aligned_* in layout.cuh)
   const int G0 = nT * p.gB.ngroups + (nE - nT) * p.gBs.ngroups;
   const bool aligned = use_aligned(G0, NB);
-  // one-token launches: the tables loaded with the router hold every range
-  // (unless NaN logits made the token select fewer than K experts)
-  const bool tab = p.part_tab && rp.whole && nT == p.part_nT;
+  // decode launches: the tables fetched with the router (one token, unless
+  // NaN logits made it select fewer than K experts) or after the top-k hold
+  // every range
+  const bool tab_post = s.tab_nT != 0 && s.tab_nT == nT;
+  const bool tab = (tab_pro && nT == rp.K) || tab_post;
 
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
     unsigned bound = 0;
+    if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
     if (tab)
       bound = lane < 2 ? s.rs0[b + lane] : s.rs1[b + (lane & 1)];
     else if (lane < 2)
@@ -1117,6 +1148,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     // when a wait gave up): wait, bounded, for each slot's last issued phase.
     if (lane == 0 && s.dead) {
       const unsigned long long t0 = globaltimer();
+      if (s.tab_nT)
+        while (!mbar_try_wait(&s.tbar, 0) && globaltimer() - t0 < WAIT_LIMIT_NS) {
+        }
       // slot i of a ring of n was used count / n + (i < count % n) times
       for (int i = 0; i < NSW; ++i) {
         const int uses = wcount / NSW + (i < wcount % NSW ? 1 : 0);
@@ -1135,6 +1169,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   }
 
   // ------------------------------------------------------------ consumer warps
+  if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
   if (!tab)
     for (int i = tid; i < 2 * (NB + 1); i += NWC * 32) {
       if (i <= NB)

@@ -82,8 +82,8 @@ struct ts_moe {
   unsigned* cnt_gB = nullptr;   // gate/up: per (expert, group, consumer warp) chunk counters
   unsigned long long* arrivals = nullptr;  // grid barrier arrivals (64-bit, never reset while the handle lives)
   unsigned* grid = nullptr;     // {x slices written, router items published}
-  unsigned* part_m1 = nullptr;  // range tables of one-token launches (K routed entries), computed at open
-  int part_m1_nT = 0;
+  unsigned* part_all = nullptr;  // decode launches' range tables for 1 .. part_nmax routed entries, computed at open
+  int part_nmax = 0;
   bool debug_skip_arrival = false;
   unsigned* err = nullptr;
   size_t counters_bytes = 0;
@@ -431,7 +431,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     const size_t o_P = slot((size_t)(Mx * K + Mx) * H * 4);
     const size_t o_part0 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
     const size_t o_part1 = slot((size_t)h->nb * 2 * SLOT_FLOATS * 4);
-    const size_t o_tab = slot((size_t)2 * part_stride(h->nb) * 4);
+    h->part_nmax = std::min(E, MAX_TOK * K);  // routed entries of a decode launch
+    const size_t o_tab = slot((size_t)h->part_nmax * 2 * part_stride(h->nb) * 4);
     const size_t o_cnt = off;
     const size_t n_cnt = 2 + (size_t)MAX_ENTRIES * h->ng_max_B * NWC + MAX_ENTRIES + 2 + 1;  // arrivals (u64) + ... + grid[2] + error word
     slot(n_cnt * 4);
@@ -457,7 +458,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     h->P = (float*)(h->ws + o_P);
     h->partial0 = (float*)(h->ws + o_part0);
     h->partial1 = (float*)(h->ws + o_part1);
-    h->part_m1 = (unsigned*)(h->ws + o_tab);
+    h->part_all = (unsigned*)(h->ws + o_tab);
     unsigned* cn = (unsigned*)(h->ws + o_cnt);
     h->counters = (uint8_t*)cn;
     h->counters_bytes = n_cnt * 4;
@@ -478,8 +479,8 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     return cleanup(st);
   }
   {
-    // one token selects K distinct experts: the range tables of its launches
-    // are fixed by the geometry, so they are computed once here
+    // a decode launch's unit-equal range tables depend only on the geometry and
+    // its count of routed entries: computed once here for every count
     LayerParams lp;
     std::memset(&lp, 0, sizeof(lp));
     lp.gB = h->gB;
@@ -487,8 +488,7 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
     lp.gC = h->gC;
     lp.gCs = h->gCs;
     lp.rp.has_shared = c.shared_inter > 0;
-    h->part_m1_nT = K;
-    partition_table_kernel<<<1, 256>>>(lp, K, K + (lp.rp.has_shared ? 1 : 0), h->nb, part_stride(h->nb), h->part_m1);
+    partition_table_kernel<<<h->part_nmax, 256>>>(lp, lp.rp.has_shared ? 1 : 0, h->nb, part_stride(h->nb), h->part_all);
     ce = cudaGetLastError();
     if (ce == cudaSuccess) ce = cudaStreamSynchronize(nullptr);
     if (ce != cudaSuccess) {
@@ -752,8 +752,8 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
     lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, h->lt), M);
     lp.y = y ? y + (size_t)m0 * H : nullptr;
     lp.resid = resid ? (__nv_bfloat16*)resid + (size_t)m0 * H : nullptr;
-    lp.part_tab = lp.rp.M == 1 && lp.rp.whole ? h->part_m1 : nullptr;  // whole-router one-token launches
-    lp.part_nT = h->part_m1_nT;
+    lp.part_all = lp.rp.M <= MAX_TOK ? h->part_all : nullptr;  // decode launches
+    lp.part_nmax = h->part_nmax;
     cudaError_t e;
     const bool big = lp.rp.M > MAX_TOK;  // a prefill launch: several routing blocks
     if (c.expert_fmt == TS_FMT_MXFP4)
