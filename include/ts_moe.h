@@ -128,8 +128,9 @@ typedef struct ts_moe ts_moe;
  * items that fit the SM count and shared memory with TS_MOE_EUNSUPPORTED), then on
  * cfg->device allocates the repacked weight arena and the per-call workspace
  * (sized once for max_tokens) and repacks every layer.  All refusals happen
- * before any device memory exists (deepseek2 state page: errors at open, "not
- * at token 1").  *out is set only on TS_MOE_OK.  Synchronises the device. */
+ * before any device memory exists (deepseek2 state page: a bad model is
+ * refused when it is loaded, never at the first token).  *out is set only on
+ * TS_MOE_OK.  Synchronises the device. */
 ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* layers, ts_moe** out);
 
 /* Router GEMV + top-k only: the int8 router GEMV to FP32 logits with the
@@ -139,10 +140,12 @@ ts_moe_status ts_moe_open(const ts_moe_config* cfg, const ts_moe_layer_weights* 
  * idx: device [M][K] int32 selected experts in slot order (descending
  * selection logit, lower index first on ties); w: device [M][K] float32
  * weights; logits: device [M][E] float32 router logits before any bias, or
- * NULL.  0 <= M <= max_tokens (M = 0 is a no-op; M > 16 runs in 16-token
- * chunks, one launch each).  The routing equals the one ts_moe_forward uses
- * for a call of the same M, bit for bit.  Asynchronous on `stream` (a
- * cudaStream_t, NULL = legacy default stream). */
+ * NULL.  0 <= M <= max_tokens (M = 0 is a no-op).  Runs the routing part of
+ * ts_moe_forward's launches alone (one launch per 64 tokens, on every SM), so
+ * the routing equals the one ts_moe_forward uses for a call of the same M,
+ * bit for bit.  Shares the handle's workspace with ts_moe_forward: calls on
+ * one handle must be ordered.  Asynchronous on `stream` (a cudaStream_t,
+ * NULL = legacy default stream). */
 ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
                            void* stream);
 

@@ -910,7 +910,9 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
 
 // BIG: a launch of more than 16 tokens (several routing blocks, experts cut
 // into entries of 16 routes); the other instance is the decode launch.
-template <int FMT, bool BIG>
+// RONLY: the routing of such a launch alone (ts_moe_route), then a grid
+// barrier so that the item counters can be reset; FMT does not matter there.
+template <int FMT, bool BIG, bool RONLY = false>
 __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   LayerSmem& s = *reinterpret_cast<LayerSmem*>(smem_raw);
@@ -927,6 +929,9 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   RouteParams rp = p.rp;
   rp.logits = nullptr;  // written below by CTA 0 from the summed items
   if (b != 0) {
+    rp.idx_out = nullptr;
+    rp.w_out = nullptr;
+    rp.logits_out = nullptr;
     rp.idx = nullptr;
     rp.w = nullptr;
     rp.shift = nullptr;
@@ -1100,6 +1105,16 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     }
   }
   route_list<BIG>(rp, s.r, warp, lane, tid, NTHREADS);
+  if constexpr (RONLY) {
+    // every CTA has read the router items once all are past the barrier
+    if (warp == NWC) return;
+    grid_barrier(s, p, NB, tid);
+    if (b == 0 && tid == 0) {
+      *p.route_cnt = 0u;
+      *p.xh_cnt = 0u;
+    }
+    return;
+  }
   fence_proxy_async_smem();  // the rings are rewritten by bulk copies from here on
   // Cost-weighted ranges where units differ in cost: a launch of more than
   // 16 tokens cuts experts into entries of up to 16 columns.

@@ -270,6 +270,8 @@ ts_moe_status set_smem_attrs(ts_moe* h) {
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX));
   return TS_MOE_OK;
 }
@@ -669,45 +671,17 @@ static ts_moe_status check_call(ts_moe* h, int layer, const void* x, int M) {
   return TS_MOE_OK;
 }
 
-static ts_moe_status launch_route(ts_moe* h, const RouteParams& rp, cudaStream_t st) {
-  cudaError_t e = launch_pdl(route_kernel, 1, ROUTE_THREADS, route_smem(rp), st, rp);
-  if (e != cudaSuccess) return cuda_fail(h, e, "route_kernel launch");
-  return TS_MOE_OK;
-}
-
 // A call of M tokens runs as launches over consecutive row blocks, full ones
-// first: ts_moe_forward in launches of h->lt (64) tokens, each of which reads
-// every touched expert's weights once per 16 routes; ts_moe_route in launches
-// of 16.  Tokens are independent in the routed half, so the chunking changes
+// first: ts_moe_forward and ts_moe_route in launches of h->lt (64) tokens,
+// each forward launch reading every touched expert's weights once per 16
+// routes.  Tokens are independent in the routed half, so the chunking changes
 // no token's route (the chunked-prefill driver of the gpt-oss state page,
 // `BatchedRoutedScratch`, feeds the routed half MAX_PREFILL_BATCH = 16 rows
 // at a time; here a launch takes up to four such blocks).
 static inline int chunk_rows(int M, int m0, int n) { return std::min(n, M - m0); }
 
-ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
-                           void* stream) {
-  ts_moe_status s = check_call(h, layer, x, M);
-  if (s != TS_MOE_OK) return s;
-  if (M == 0) return TS_MOE_OK;
-  if (!idx || !w) return fail(h, TS_MOE_EINVAL, "idx and w must be non-NULL");
-  const int H = h->cfg.hidden, E = h->cfg.num_experts, K = h->cfg.top_k;
-  for (int m0 = 0; m0 < M; m0 += MAX_TOK) {
-    RouteParams rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, MAX_TOK), M);
-    rp.idx_out = idx + (size_t)m0 * K;
-    rp.w_out = w + (size_t)m0 * K;
-    rp.logits_out = logits ? logits + (size_t)m0 * E : nullptr;
-    s = launch_route(h, rp, (cudaStream_t)stream);
-    if (s != TS_MOE_OK) return s;
-  }
-  return TS_MOE_OK;
-}
-
-ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream) {
-  ts_moe_status s = check_call(h, layer, x, M);
-  if (s != TS_MOE_OK) return s;
-  if (!resid && !y) return fail(h, TS_MOE_EINVAL, "resid and y are both NULL");
-  if (M == 0) return TS_MOE_OK;
-  cudaStream_t st = (cudaStream_t)stream;
+// The launch parameters of a layer, without the per-launch routing and outputs.
+static LayerParams layer_params(ts_moe* h, int layer) {
   const ts_moe_config& c = h->cfg;
   const LayerDev& d = h->layers[layer];
   LayerParams lp;
@@ -738,13 +712,45 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
   lp.grid_cnt = h->arrivals;
   lp.xh_cnt = h->grid;
   lp.route_cnt = h->grid + 1;
-  lp.debug_skip_arrival = h->debug_skip_arrival ? 1 : 0;
-  h->debug_skip_arrival = false;  // one launch only
   lp.err = h->err;
   lp.act = c.act;
   lp.alpha = c.act_alpha;
   lp.limit = c.act_limit;
+  return lp;
+}
 
+// ts_moe_route runs the routing of ts_moe_forward's launches alone (the same
+// launches, so every token's logits, experts and weights are the forward's).
+ts_moe_status ts_moe_route(ts_moe* h, int layer, const void* x, int M, int32_t* idx, float* w, float* logits,
+                           void* stream) {
+  ts_moe_status s = check_call(h, layer, x, M);
+  if (s != TS_MOE_OK) return s;
+  if (M == 0) return TS_MOE_OK;
+  if (!idx || !w) return fail(h, TS_MOE_EINVAL, "idx and w must be non-NULL");
+  const int H = h->cfg.hidden, E = h->cfg.num_experts, K = h->cfg.top_k;
+  LayerParams lp = layer_params(h, layer);
+  for (int m0 = 0; m0 < M; m0 += h->lt) {
+    lp.rp = route_params(h, layer, (const __nv_bfloat16*)x + (size_t)m0 * H, chunk_rows(M, m0, h->lt), M);
+    lp.rp.idx_out = idx + (size_t)m0 * K;
+    lp.rp.w_out = w + (size_t)m0 * K;
+    lp.rp.logits_out = logits ? logits + (size_t)m0 * E : nullptr;
+    const cudaError_t e = launch_pdl(lp.rp.M > MAX_TOK ? layer_kernel<0, true, true> : layer_kernel<0, false, true>,
+                                     h->nb, NTHREADS, sizeof(LayerSmem), (cudaStream_t)stream, lp);
+    if (e != cudaSuccess) return cuda_fail(h, e, "routing launch");
+  }
+  return TS_MOE_OK;
+}
+
+ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* resid, float* y, void* stream) {
+  ts_moe_status s = check_call(h, layer, x, M);
+  if (s != TS_MOE_OK) return s;
+  if (!resid && !y) return fail(h, TS_MOE_EINVAL, "resid and y are both NULL");
+  if (M == 0) return TS_MOE_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const ts_moe_config& c = h->cfg;
+  LayerParams lp = layer_params(h, layer);
+  lp.debug_skip_arrival = h->debug_skip_arrival ? 1 : 0;
+  h->debug_skip_arrival = false;  // the next forward launch only
   const size_t smem = sizeof(LayerSmem);
   const int H = c.hidden;
   if (h->timing) cudaEventRecord(h->ev[0], st);
