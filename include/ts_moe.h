@@ -72,8 +72,8 @@ enum {
                                         w = s over S renormalised to sum 1 (llama state page, MiniMax flow:
                                         router_scoring_func "sigmoid", e_score_correction_bias) */
 };
-/* Router bias (gpt-oss state page, `router_bias`: added to the logits BEFORE
- * top-k).  LOGITS: selection and weights both use l + b.  SELECT_ONLY: l + b
+/* Router bias (gpt-oss state page, `router_bias`: it joins the logits ahead of
+ * the top-k).  LOGITS: selection and weights both use l + b.  SELECT_ONLY: l + b
  * selects, the weights use the unbiased l. */
 enum { TS_BIAS_NONE = 0, TS_BIAS_LOGITS = 1, TS_BIAS_SELECT_ONLY = 2 };
 /* SWIGLU: silu(g) * u.  SWIGLU_CLAMPED (gpt-oss state page header, "clamped

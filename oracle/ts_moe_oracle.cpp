@@ -20,7 +20,7 @@
 //      `router_logits_f32` buffer is                 [llama state: router_ones,
 //                                                     router_logits_f32]
 //   3. selection logits l'[e] = l[e] + b[e] (FP32 add) when a router bias is
-//      present; the bias is added BEFORE top-k          [gpt-oss state:
+//      present; the bias joins the logits ahead of top-k  [gpt-oss state:
 //                                                        router_bias]
 //   4. S = top-K of l' by (value desc, index asc) (sigmoid scoring: of s + b, below)
 //   5. weights: softmax over the selected experts (SOFTMAX_WEIGHT, norm_w

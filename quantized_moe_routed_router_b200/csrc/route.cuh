@@ -22,7 +22,7 @@
 //
 // One warp per token then selects the top K by (selection logit desc, index
 // asc), where the selection logit is l + b when a router bias is present
-// (gpt-oss state page, `router_bias`: added BEFORE the top-k), and forms the
+// (gpt-oss state page, `router_bias`: the bias enters ahead of the top-k), and forms the
 // weights: softmax over the selected (`per_expert_ones`: with unit per-expert
 // scales the weights are exactly that softmax), or the full softmax over all experts taken at
 // the selected indices without renormalisation (deepseek2 layer sketch), or --

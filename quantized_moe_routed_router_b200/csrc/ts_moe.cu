@@ -272,7 +272,6 @@ ts_moe_status set_smem_attrs(ts_moe* h) {
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  TSM_CUDA(h, cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_SMEM_MAX));
   return TS_MOE_OK;
 }
 
