@@ -25,6 +25,7 @@ enum : unsigned {
   ERR_TIMEOUT_XH = 1u << 9,      // a producer gave up waiting for the shared FP16 x
   ERR_TIMEOUT_ROUTE = 1u << 10,  // a CTA gave up waiting for the published router logits
   ERR_BAD_ROUTER_INPUT = 1u << 11,  // a router bias or per-expert scale read by the route kernel was not finite
+  ERR_TIMEOUT_TABLES = 1u << 12,    // a decode launch gave up waiting for its precomputed range tables
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.

@@ -1141,7 +1141,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   if (warp == NWC) {
     // ------------------------------------------------------------ producer warp
     unsigned bound = 0;
-    if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+    if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_TABLES);
     if (tab)
       bound = lane < 2 ? s.rs0[b + lane] : s.rs1[b + (lane & 1)];
     else if (lane < 2)
@@ -1184,7 +1184,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
   }
 
   // ------------------------------------------------------------ consumer warps
-  if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_XSTAGE);
+  if (tab_post) mbar_wait(&s.tbar, 0, &s.dead, p.err, ERR_TIMEOUT_TABLES);
   if (!tab)
     for (int i = tid; i < 2 * (NB + 1); i += NWC * 32) {
       if (i <= NB)

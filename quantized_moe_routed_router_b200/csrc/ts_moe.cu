@@ -781,11 +781,11 @@ ts_moe_status ts_moe_device_status(ts_moe* h, void* stream) {
   TSM_CUDA(h, cudaMemcpy(&err, h->err, 4, cudaMemcpyDeviceToHost));
   if (!err) return TS_MOE_OK;
   TSM_CUDA(h, cudaMemset(h->counters, 0, h->counters_bytes));
-  char buf[512];
+  char buf[768];
   std::snprintf(buf, sizeof buf, "device error word 0x%x (bit0/1: weight-stage wait gave up, bit2/3: activation-window "
                 "wait gave up, bit4: bad index, bit5: bad route metadata, bit6: grid barrier wait gave up, bit7: "
                 "wait for an expert's activations gave up, bit8: wait for the staged x gave up, bit9: wait for the "
-                "shared FP16 x gave up, bit10: wait for the router logits gave up, bit11: non-finite router bias or per-expert scale)", err);
+                "shared FP16 x gave up, bit10: wait for the router logits gave up, bit11: non-finite router bias or per-expert scale, bit12: wait for the precomputed range tables gave up)", err);
   return fail(h, TS_MOE_EDEVICE, buf);
 }
 
