@@ -196,16 +196,17 @@ ts_moe_status ts_moe_get_info(const ts_moe* h, ts_moe_info* info);
  * kernels, so a timed run without hooks is the throughput number. */
 ts_moe_status ts_moe_set_timing_events(ts_moe* h, void* const* events4);
 
-/* Router GEMV + top-k for callers that cannot allocate device memory.  This
- * entry point has no counterpart in the paper; it is a convenience of this
- * library.  ts_moe_open allocates a weight arena and a workspace, and some
- * callers cannot allocate at all: inference engines that hand every byte of
- * device memory to their own pool when they start and forbid allocations
- * afterwards, and plugins or extensions that are given only a stream and
- * buffers the host application owns.  This call takes the raw router itself
- * and keeps all of its scratch in one file-scope device array of
- * TS_MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
- * until the process exits.  It calls no allocator of any kind.
+/* Router GEMV + top-k for callers that cannot allocate device memory.
+ * This entry point has no counterpart on the llama / gpt-oss state pages; it
+ * is a convenience of this library.  ts_moe_open allocates a weight arena
+ * and a workspace, and some callers cannot allocate at all: inference
+ * engines that hand every byte of device memory to their own pool when they
+ * start and forbid allocations afterwards, and plugins or extensions that
+ * are given only a stream and buffers the host application owns.  This call
+ * takes the raw router itself and keeps all of its scratch in one file-scope
+ * device array of TS_MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads
+ * the library holds until the process exits.  It calls no allocator of any
+ * kind.
  *
  * router: device [E][H] Q8_0 blocks (as in ts_moe_layer_weights.router);
  * router_bias, per_expert_scale: DEVICE [E] float32 or NULL (bias required
