@@ -247,6 +247,25 @@ bool router_slicing(int M, const MatGeom& gR, int E, int nb, bool split, int& S,
 // device iff per_sm >= 1 and nb <= per_sm * sm_count.
 bool coresident(int per_sm, int sm_count, int nb) { return per_sm >= 1 && (long long)nb <= (long long)per_sm * sm_count; }
 
+// The layer-kernel instance of a forward launch: prefill (more than 16
+// tokens), decode with at most 8 tokens (every entry one n8 tile), one token
+// routed with the whole router, or any other decode launch.
+template <int FMT>
+void (*layer_instance(const RouteParams& rp))(LayerParams) {
+  if (rp.M > MAX_TOK) return layer_kernel<FMT, true>;
+  if (rp.M == 1 && rp.whole) return layer_kernel<FMT, false, false, 2>;
+  if (rp.M <= 8) return layer_kernel<FMT, false, false, 1>;
+  return layer_kernel<FMT, false>;
+}
+
+template <int FMT>
+cudaError_t set_narrow_smem(int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(layer_kernel<FMT, false, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(layer_kernel<FMT, false, false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 template <typename... Args>
 cudaError_t launch_pdl(void (*k)(Args...), int grid, int block, size_t smem, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t lc = {};
@@ -270,6 +289,9 @@ ts_moe_status set_smem_attrs(ts_moe* h) {
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  TSM_CUDA(h, set_narrow_smem<0>(bytes));
+  TSM_CUDA(h, set_narrow_smem<1>(bytes));
+  TSM_CUDA(h, set_narrow_smem<2>(bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   TSM_CUDA(h, cudaFuncSetAttribute(layer_kernel<0, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   return TS_MOE_OK;
@@ -760,13 +782,12 @@ ts_moe_status ts_moe_forward(ts_moe* h, int layer, const void* x, int M, void* r
     lp.part_all = lp.rp.M <= MAX_TOK ? h->part_all : nullptr;  // decode launches
     lp.part_nmax = h->part_nmax;
     cudaError_t e;
-    const bool big = lp.rp.M > MAX_TOK;  // a prefill launch: several routing blocks
     if (c.expert_fmt == TS_FMT_MXFP4)
-      e = launch_pdl(big ? layer_kernel<1, true> : layer_kernel<1, false>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(layer_instance<1>(lp.rp), h->nb, NTHREADS, smem, st, lp);
     else if (c.expert_fmt == TS_FMT_INT4_AFFINE)
-      e = launch_pdl(big ? layer_kernel<2, true> : layer_kernel<2, false>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(layer_instance<2>(lp.rp), h->nb, NTHREADS, smem, st, lp);
     else
-      e = launch_pdl(big ? layer_kernel<0, true> : layer_kernel<0, false>, h->nb, NTHREADS, smem, st, lp);
+      e = launch_pdl(layer_instance<0>(lp.rp), h->nb, NTHREADS, smem, st, lp);
     if (e != cudaSuccess) return cuda_fail(h, e, "layer kernel launch");
   }
   if (h->timing) cudaEventRecord(h->ev[1], st);
