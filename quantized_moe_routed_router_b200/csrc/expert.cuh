@@ -912,10 +912,10 @@ TSM_DEV bool produce_phase(LayerSmem& s, const LayerParams& p, long long u0, lon
 // into entries of 16 routes); the other instance is the decode launch.
 // RONLY: the routing of such a launch alone (ts_moe_route), then a grid
 // barrier so that the item counters can be reset; FMT does not matter there.
-// NARROW: decode launches whose entries all have at most 8 columns (1: at
-// most 8 tokens; 2: one token, routed with the whole router).  Such an
-// instance holds only the code those launches run -- one n8 MMA tile per
-// entry, and for one token no sliced routing -- so the once-per-launch phases
+// NARROW: decode launches of one kind (1: at most 8 tokens; 2: one token,
+// whole router; 3: 9 to 16 tokens, router items).  Such an instance holds
+// only the code those launches run -- one n8 MMA tile per entry up to 8
+// tokens, one routing form for 2 and 3 -- so the once-per-launch phases
 // fetch fewer instructions.
 template <int FMT, bool BIG, bool RONLY = false, int NARROW = 0>
 __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
@@ -936,6 +936,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     rp.M = 1;
     rp.whole = 1;
   }
+  if constexpr (NARROW == 3) rp.whole = 0;
   rp.logits = nullptr;  // written below by CTA 0 from the summed items
   if (b != 0) {
     rp.idx_out = nullptr;
@@ -1209,7 +1210,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     int j = 0;
     Seg sg;
     while (next_seg<0>(s, p, u, a1, j, sg)) {
-      if (NARROW == 0 && sg.nc > 8)
+      if ((NARROW == 0 || NARROW == 3) && sg.nc > 8)
         consume_seg<FMT, 0, 2>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
       else
         consume_seg<FMT, 0, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
@@ -1221,7 +1222,7 @@ __global__ void __maxnreg__(120) layer_kernel(const LayerParams p) {
     int j = 0;
     Seg sg;
     while (next_seg<1>(s, p, u, d1, j, sg)) {
-      if (NARROW == 0 && sg.nc > 8)
+      if ((NARROW == 0 || NARROW == 3) && sg.nc > 8)
         consume_seg<FMT, 1, 2>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);
       else
         consume_seg<FMT, 1, 1>(s, p, sg, wi, wph, xi, xph, warp, lane, tid, NB);

@@ -248,22 +248,25 @@ bool router_slicing(int M, const MatGeom& gR, int E, int nb, bool split, int& S,
 bool coresident(int per_sm, int sm_count, int nb) { return per_sm >= 1 && (long long)nb <= (long long)per_sm * sm_count; }
 
 // The layer-kernel instance of a forward launch: prefill (more than 16
-// tokens), decode with at most 8 tokens (every entry one n8 tile), one token
-// routed with the whole router, or any other decode launch.
+// tokens); decode of one token routed with the whole router; decode of at
+// most 8 tokens (every entry one n8 tile); decode of 9 to 16 tokens routed
+// with router items; or any other decode launch.
 template <int FMT>
 void (*layer_instance(const RouteParams& rp))(LayerParams) {
   if (rp.M > MAX_TOK) return layer_kernel<FMT, true>;
-  if (rp.M == 1 && rp.whole) return layer_kernel<FMT, false, false, 2>;
+  if (rp.whole && rp.M == 1) return layer_kernel<FMT, false, false, 2>;
   if (rp.M <= 8) return layer_kernel<FMT, false, false, 1>;
+  if (!rp.whole && rp.M > 8) return layer_kernel<FMT, false, false, 3>;
   return layer_kernel<FMT, false>;
 }
 
 template <int FMT>
 cudaError_t set_narrow_smem(int bytes) {
-  cudaError_t e = cudaFuncSetAttribute(layer_kernel<FMT, false, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       bytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(layer_kernel<FMT, false, false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  const auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(layer_kernel<FMT, false, false, 1>, a, bytes);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(layer_kernel<FMT, false, false, 2>, a, bytes);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(layer_kernel<FMT, false, false, 3>, a, bytes);
+  return e;
 }
 
 template <typename... Args>
